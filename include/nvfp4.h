@@ -1,0 +1,233 @@
+/*
+ * nvfp4.h -- C ABI of the B200 (sm_100a) NVFP4 W4A4 library.
+ *
+ * The operations follow the NVFP4 two-level scaling described in
+ * "How is Qwen3.8-Flash-Next-NVFP4's NVFP4 quantization done? W4A4 two-level
+ * scaling and why only routed experts are quantized" (section "Core: W4A4
+ * two-level scaling"): E2M1 element codes, one E4M3 block scale per 16
+ * contiguous elements of the last dimension, one FP32 global scale per tensor,
+ * 4.5 bits per element. Calibration modes follow Table 1 of "Developing
+ * Nemotron 3.5 Lightning NVFP4 with QAD using NVIDIA Model Optimizer" (max and
+ * four_over_six) and its section "Quantization scale handling during QAD"
+ * (dynamic and frozen scales). The W4A4 GEMM is the operation that "Why W4A4
+ * rather than W4A16" in "Model-Optimizer in practice: recovering
+ * Qwen3.6-35B-A3B W4A4 NVFP4 accuracy with QAD" says only FP4 activations can
+ * reach on Blackwell tensor cores.
+ *
+ * Conventions for every call
+ * --------------------------
+ *  - Pointers are DEVICE pointers unless a comment says otherwise. Calls are
+ *    asynchronous on `stream` (0 = legacy default stream).
+ *  - The caller owns and allocates every buffer. The library allocates no
+ *    device memory; scratch comes from a caller-provided `workspace` whose
+ *    size is returned by the matching *_workspace_bytes query.
+ *  - Return value: an nvfp4_status checked synchronously on the host
+ *    (argument validation, device gate, launch errors). Conditions found on
+ *    the device (non-finite input, a bounded wait that ran out) are recorded
+ *    in a library-owned device status word; read it with
+ *    nvfp4_get_device_status(), which synchronizes `stream`.
+ *  - Requirements: K % 64 == 0; every pointer 16-byte aligned; inputs
+ *    row-major and contiguous. The device must be sm_100 (B200-class);
+ *    other devices get NVFP4_ERR_UNSUPPORTED_DEVICE (the hardware gate of
+ *    "check what your card supports before choosing FP8 / W4A8 / NVFP4").
+ *
+ * Storage formats
+ * ---------------
+ *  codes   [rows][K/2] bytes, two E2M1 codes per byte, element 2j in the low
+ *          nibble of byte j. Code bit 3 is the sign.
+ *  scales  E4M3 block scales in the tiled layout the block-scaled MMA reads:
+ *          512-byte tiles of 128 rows x 4 scales (64 elements of K), tiles
+ *          ordered row-tile-major (tile = (r/128) * (K/64) + c/4), and inside
+ *          a tile the scale of (row r, block c) at byte
+ *          (r%32)*16 + ((r%128)/32)*4 + c%4. Rows are padded to a multiple of
+ *          128 with zero bytes. Size: nvfp4_scale_bytes(rows, K).
+ *  g       one FP32 global scale per tensor: g = amax / (6 * 448).
+ */
+#ifndef NVFP4_H_
+#define NVFP4_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef struct CUstream_st* nvfp4_stream_t; /* same handle as cudaStream_t */
+
+typedef enum {
+  NVFP4_OK = 0,
+  NVFP4_ERR_INVALID_ARG = 1,        /* bad pointer, size, alignment or mode */
+  NVFP4_ERR_UNSUPPORTED_DEVICE = 2, /* not an sm_100 device */
+  NVFP4_ERR_CUDA = 3,               /* a CUDA runtime call failed */
+  NVFP4_ERR_WORKSPACE = 4,          /* workspace missing or too small */
+  NVFP4_ERR_NONFINITE_INPUT = 5,    /* device: amax of an input is Inf/NaN */
+  NVFP4_ERR_TIMEOUT = 6             /* device: a bounded wait ran out */
+} nvfp4_status;
+
+typedef enum {
+  NVFP4_MODE_MAX = 0,           /* every block targets the E2M1 maximum 6 */
+  NVFP4_MODE_FOUR_OVER_SIX = 1  /* per block, target 6 or 4, lower block MSE */
+} nvfp4_mode;
+
+/* Library version (major*10000 + minor*100 + patch). Host only. */
+int nvfp4_version(void);
+
+/* Hardware gate for the CURRENT device: NVFP4_OK on sm_100, else
+ * NVFP4_ERR_UNSUPPORTED_DEVICE (or NVFP4_ERR_CUDA if no device). */
+nvfp4_status nvfp4_check_device(void);
+
+/* Human-readable name of a status code (static string). Host only. */
+const char* nvfp4_status_string(nvfp4_status s);
+
+/* Bytes of the tiled block-scale buffer for a [rows x K] tensor:
+ * ceil(rows/128) * (K/64) * 512. Returns 0 if K % 64 != 0. Host only. */
+size_t nvfp4_scale_bytes(int64_t rows, int64_t K);
+
+/* Workspace bytes nvfp4_quantize / nvfp4_fake_quant need to compute a dynamic
+ * global scale for an [M x K] input (0 is never returned). Host only. */
+size_t nvfp4_quantize_workspace_bytes(int64_t M, int64_t K);
+
+/*
+ * nvfp4_quantize -- NVFP4 quantization of x [M x K] BF16 along K.
+ *   Two-level scaling ("Core: W4A4 two-level scaling", levels 1 and 2):
+ *   g = amax/2688 (or *g_in when given: a static, calibrated global scale);
+ *   per block of 16, s = E4M3(bmax / (Mt * g)) floored at 2^-9, Mt = 6
+ *   (mode MAX) or the better of 6 and 4 by block squared error (mode
+ *   FOUR_OVER_SIX, tie -> 6); codes = E2M1(x * (1 / (g * s))); every
+ *   rounding is to nearest even and saturating (E2M1 at +-6, E4M3 at 448).
+ *   Dynamic activations use g_in = NULL ("the A4 side: dynamic activations");
+ *   static weights pass a precomputed g_in or let the call compute it.
+ * x           [M][K] BF16, device.
+ * g_in        nullable device FP32 scalar: static global scale.
+ * codes       out [M][K/2] bytes.
+ * scales      out nvfp4_scale_bytes(M, K) bytes (tiled layout, padding zeroed).
+ * g_out       out device FP32 scalar: the global scale used.
+ * fos_choice  nullable out [M][K/16] bytes: 1 where the block kept the M=4
+ *             scale, else 0 (always 0 in mode MAX).
+ * workspace   >= nvfp4_quantize_workspace_bytes(M, K) bytes when g_in is
+ *             NULL; may be NULL when g_in is given. Contents need no
+ *             initialisation. Calls that share one workspace must be ordered
+ *             on the GPU (same stream).
+ * M may be 0 (nothing is written except g_out = 1 for a dynamic call).
+ * Device status: NVFP4_ERR_NONFINITE_INPUT if amax is Inf/NaN (outputs are
+ * then unspecified).
+ */
+nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t K, nvfp4_mode mode,
+                            const float* g_in, uint8_t* codes, uint8_t* scales,
+                            float* g_out, uint8_t* fos_choice, void* workspace,
+                            size_t workspace_bytes, nvfp4_stream_t stream);
+
+/*
+ * nvfp4_fake_quant -- quantize-dequantize forward of QAD's simulated
+ *   quantization ("Quantization scale handling during QAD", Figure 2):
+ *   y = BF16(g * s * q) elementwise, with q, s, g as in nvfp4_quantize.
+ *   Scale sources:
+ *     g_frozen = NULL, scales_frozen = NULL : dynamic lane, g and s
+ *        recomputed from x (mode selects MAX / FOUR_OVER_SIX);
+ *     g_frozen set, scales_frozen = NULL : static g, block scales from x;
+ *     both set : frozen lane, s* and g* as captured by an earlier
+ *        nvfp4_quantize (tiled layout); codes saturate at +-6 when x has
+ *        drifted past the frozen range. mode is ignored.
+ * x, y        [M][K] BF16, device (y may not alias x).
+ * workspace   as for nvfp4_quantize (needed only when g_frozen is NULL).
+ */
+nvfp4_status nvfp4_fake_quant(const void* x, int64_t M, int64_t K, nvfp4_mode mode,
+                              const float* g_frozen, const uint8_t* scales_frozen,
+                              void* y, void* workspace, size_t workspace_bytes,
+                              nvfp4_stream_t stream);
+
+/*
+ * nvfp4_gemm -- W4A4 block-scaled GEMM on tcgen05 tensor cores:
+ *   C[m][n] = BF16( (ga*gb) * sum_k (sa*qa)[m][k] * (sb*qb)[n][k] ),
+ *   FP32 accumulation in tensor memory, global-scale product and BF16
+ *   rounding fused in the epilogue ("Why W4A4 rather than W4A16").
+ * Aq, As, ga  activations: codes [M][K/2], tiled scales, FP32 global scale.
+ * Bq, Bs, gb  weights: codes [N][K/2], tiled scales, FP32 global scale.
+ * C           out [M][N] BF16 row-major.
+ * Requirements: M >= 0, N % 16 == 0, K % 64 == 0, K > 0.
+ * Device status: NVFP4_ERR_TIMEOUT if a pipeline wait ran out (C then
+ * unspecified; the context stays usable).
+ */
+nvfp4_status nvfp4_gemm(const uint8_t* Aq, const uint8_t* As, const float* ga,
+                        const uint8_t* Bq, const uint8_t* Bs, const float* gb,
+                        int64_t M, int64_t N, int64_t K, void* C,
+                        nvfp4_stream_t stream);
+
+/*
+ * Routed-expert (MoE) layer in NVFP4 W4A4 -- the layer the pages quantize
+ * first ("2. PTQ": routed experts are 99.2% of the quantized tensors; the
+ * Qwen3.8-Flash-Next page quantizes only the fused gate_up_proj/down_proj of
+ * the routed experts, with top-k routing and dynamic activations).
+ *
+ *   out[t] = sum_j topk_w[t][j] * Down_e( SiLU(Gate_e(x_t)) * Up_e(x_t) ),
+ *   e = topk_ids[t][j]
+ *
+ * with each expert's activations quantized dynamically (its own global scale
+ * over the rows routed to it), h = SiLU(gate)*up rounded to BF16 and
+ * quantized per expert, and the weighted combine done in FP32.
+ * x         [T][H] BF16.
+ * topk_ids  [T][topk] int32 in [0, E); topk_w [T][topk] FP32.
+ * w13_q     [E][2I][H/2] codes; rows [0, I) are gate, [I, 2I) are up.
+ * w13_s     E consecutive tiled scale buffers of nvfp4_scale_bytes(2I, H).
+ * w13_g     [E] FP32 global scales.
+ * w2_q      [E][H][I/2] codes; w2_s E buffers of nvfp4_scale_bytes(H, I);
+ * w2_g      [E] FP32.
+ * out       [T][H] FP32, overwritten.
+ * workspace >= nvfp4_moe_workspace_bytes(T, H, I, E, topk) bytes, no
+ *           initialisation needed; calls sharing it must be stream-ordered.
+ * Requirements: H % 256 == 0, I % 128 == 0, 1 <= topk <= E <= 1024.
+ */
+size_t nvfp4_moe_workspace_bytes(int64_t T, int64_t H, int64_t I, int E, int topk);
+
+nvfp4_status nvfp4_moe_grouped_gemm(const void* x, int64_t T, int64_t H,
+                                    const int32_t* topk_ids, const float* topk_w,
+                                    int topk, int E, int64_t I,
+                                    const uint8_t* w13_q, const uint8_t* w13_s,
+                                    const float* w13_g, const uint8_t* w2_q,
+                                    const uint8_t* w2_s, const float* w2_g,
+                                    float* out, void* workspace, size_t workspace_bytes,
+                                    nvfp4_stream_t stream);
+
+/* Byte offsets of the intermediates the MoE call leaves in its workspace
+ * (for inspection by tests and debuggers). All rows are in expert-major,
+ * 128-padded order; R = padded row capacity. */
+typedef struct {
+  int64_t rows_capacity;    /* R */
+  int64_t counts;           /* int32 [E]   pairs routed to each expert */
+  int64_t offsets;          /* int32 [E+1] first padded row of each expert */
+  int64_t row_pair;         /* int32 [R]   flat pair t*topk+j of a row, -1 = pad */
+  int64_t xq_codes;         /* [R][H/2]    gathered, quantized x */
+  int64_t xq_scales;        /* nvfp4_scale_bytes(R, H) */
+  int64_t xq_g;             /* FP32 [E] */
+  int64_t h;                /* BF16 [R][I]  SiLU(gate)*up */
+  int64_t hq_codes;         /* [R][I/2] */
+  int64_t hq_scales;        /* nvfp4_scale_bytes(R, I) */
+  int64_t hq_g;             /* FP32 [E] */
+  int64_t total_bytes;
+} nvfp4_moe_layout;
+
+nvfp4_status nvfp4_moe_workspace_layout(int64_t T, int64_t H, int64_t I, int E, int topk,
+                                        nvfp4_moe_layout* layout /* host */);
+
+/* Conversion primitives (diagnostics; the quantize kernels use the same
+ * device code). e2m1: code of each FP32 value, one per byte, RNE, saturate
+ * at +-6, sign from the value. e4m3: code of each non-negative FP32 value,
+ * RNE, saturate at 448. n >= 0; in/out device arrays of n elements. */
+nvfp4_status nvfp4_convert_e2m1(const float* in, int64_t n, uint8_t* out, nvfp4_stream_t stream);
+nvfp4_status nvfp4_convert_e4m3(const float* in, int64_t n, uint8_t* out, nvfp4_stream_t stream);
+
+/* Synchronize `stream`, then read (and with clear != 0 reset) the device
+ * status word of the current device. *out is a host pointer. */
+nvfp4_status nvfp4_get_device_status(nvfp4_stream_t stream, int clear, nvfp4_status* out);
+
+/* Test hook for the bounded-wait path: run a kernel on `stream` whose wait
+ * on a flag that nothing sets gives up after `timeout_ns` nanoseconds and
+ * records NVFP4_ERR_TIMEOUT in the device status word. */
+nvfp4_status nvfp4_selftest_timeout(uint64_t timeout_ns, nvfp4_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVFP4_H_ */

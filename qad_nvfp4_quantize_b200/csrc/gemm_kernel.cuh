@@ -1,0 +1,251 @@
+// Block-scaled W4A4 GEMM mainloop for sm_100a (tcgen05 + TMA + TMEM).
+//
+// C = (ga*gb) * sum_k (sa*qa)(sb*qb): E2M1 operands with one UE4M3 scale per
+// 16 elements of K, FP32 accumulation in tensor memory -- the FP4 tensor-core
+// GEMM that "Why W4A4 rather than W4A16" ("Model-Optimizer in practice:
+// recovering Qwen3.6-35B-A3B W4A4 NVFP4 accuracy with QAD") says W4A4 unlocks.
+//
+// One CTA per SM, persistent over output tiles of 128 x 256. Warp roles:
+//   warp 0      TMA producer: codes of A (128 rows) and B (two boxes of 128
+//               rows) and the matching 512-byte scale tiles, 4-stage ring of
+//               256 K-elements per stage, mbarrier transaction counts;
+//   warp 1      allocates tensor memory; one lane copies the scale tiles
+//               shared -> tensor memory (tcgen05.cp) and issues the
+//               block-scaled MMAs (kind::mxf4nvf4, M=128, N=256, K=64);
+//   warps 2..9  epilogue: drain the 128 x 256 FP32 accumulator from tensor
+//               memory into registers, release it to the MMA warp, then scale,
+//               round and store (policy-specific).
+// Tensor memory: columns [0,256) accumulator, [256,272) A scales of one
+// stage (4 columns per MMA), [272,304) B scales (8 columns per MMA).
+// Every mbarrier wait is bounded; on expiry the CTA records
+// NVFP4_ERR_TIMEOUT, drains its in-flight copies and MMAs (bounded) and
+// returns with its tensor memory freed.
+#pragma once
+
+#include "common.cuh"
+
+namespace nvfp4 {
+
+constexpr int kBM = 128;
+constexpr int kBN = 256;
+constexpr int kBK = 256;                       // K elements per stage
+constexpr int kStages = 4;
+constexpr uint32_t kABytes = kBM * kBK / 2;    // 16 KB of codes
+constexpr uint32_t kBHalfBytes = 128 * kBK / 2;
+constexpr uint32_t kBBytes = kBN * kBK / 2;    // 32 KB
+constexpr uint32_t kSFAtom = 512;              // 128 rows x 4 scales
+constexpr uint32_t kSFABytes = 4 * kSFAtom;
+constexpr uint32_t kSFBBytes = 8 * kSFAtom;
+constexpr int kGemmThreads = 320;
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemSFA = 256;
+constexpr uint32_t kTmemSFB = 272;
+
+constexpr uint32_t kSmemA = 0;
+constexpr uint32_t kSmemB = kSmemA + kStages * kABytes;
+constexpr uint32_t kSmemSFA = kSmemB + kStages * kBBytes;
+constexpr uint32_t kSmemSFB = kSmemSFA + kStages * kSFABytes;
+constexpr uint32_t kSmemBar = kSmemSFB + kStages * kSFBBytes;
+constexpr uint32_t kNumBars = 2 * kStages + 3;   // full, empty, acc_full, acc_empty, drain
+constexpr uint32_t kSmemMisc = kSmemBar + kNumBars * 8;
+constexpr uint32_t kGemmSmemBytes = kSmemMisc + 16 + 1024;  // + alignment slack
+
+// Instruction descriptor of kind::mxf4nvf4: A and B E2M1 (format 1), K-major,
+// UE4M3 scales (scale format 0), N >> 3 in bits [17,23), M >> 4 in [24,29).
+__host__ __device__ constexpr uint32_t make_idesc_nvf4(int m, int n) {
+  return (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) | ((uint32_t)(m >> 4) << 24);
+}
+
+// What the producer needs to fetch for one output tile.
+struct TileJob {
+  int32_t a_row;          // first row of A in A's tensor map
+  int32_t b_row0;         // B rows for accumulator columns [0,128)
+  int32_t b_row1;         // B rows for accumulator columns [128,256)
+  const uint8_t* sfa;     // A scale tiles of this 128-row tile, K-group 0
+  const uint8_t* sfb0;    // B scale tiles for b_row0
+  const uint8_t* sfb1;    // B scale tiles for b_row1 (nullptr: none)
+  int32_t expert;
+  int32_t m0, n0;
+};
+
+template <class Prob>
+__global__ void __launch_bounds__(kGemmThreads, 1)
+    nvf4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
+                     const Prob prob, int* status, uint64_t timeout_ns) {
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemBar);
+  uint64_t* full = bars;
+  uint64_t* empty = bars + kStages;
+  uint64_t* acc_full = bars + 2 * kStages;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* drain = acc_full + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kSmemMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSmemMisc + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, 8);  // one arrive per epilogue warp
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tensormap(&tmA);
+    prefetch_tensormap(&tmB);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  const int K = prob.K;
+  const int nkt = (K + kBK - 1) / kBK;
+  const int kgroups = K / 64;
+  const int ntiles = prob.num_tiles();
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t stage = 0, phase = 0;
+      int armed_phase[kStages];
+#pragma unroll
+      for (int s = 0; s < kStages; ++s) armed_phase[s] = -1;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
+        const TileJob job = prob.job(t);
+        for (int kt = 0; kt < nkt; ++kt) {
+          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, timeout_ns)) {
+            ok = false;
+            break;
+          }
+          const int nkb = min(4, kgroups - 4 * kt);
+          const uint32_t sf_bytes = (uint32_t)nkb * kSFAtom;
+          const uint32_t tx = kABytes + kBBytes + sf_bytes * (job.sfb1 ? 3u : 2u);
+          mbar_arrive_expect_tx(&full[stage], tx);
+          armed_phase[stage] = (int)phase;
+          uint8_t* sA = smem + kSmemA + stage * kABytes;
+          uint8_t* sB = smem + kSmemB + stage * kBBytes;
+          tma_load_2d(sA, &tmA, kt * (kBK / 2), job.a_row, &full[stage]);
+          tma_load_2d(sB, &tmB, kt * (kBK / 2), job.b_row0, &full[stage]);
+          tma_load_2d(sB + kBHalfBytes, &tmB, kt * (kBK / 2), job.b_row1, &full[stage]);
+          bulk_load(smem + kSmemSFA + stage * kSFABytes, job.sfa + (size_t)kt * kSFABytes, sf_bytes,
+                    &full[stage]);
+          uint8_t* sSFB = smem + kSmemSFB + stage * kSFBBytes;
+          bulk_load(sSFB, job.sfb0 + (size_t)kt * kSFABytes, sf_bytes, &full[stage]);
+          if (job.sfb1) bulk_load(sSFB + kSFABytes, job.sfb1 + (size_t)kt * kSFABytes, sf_bytes, &full[stage]);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+      }
+      if (!ok) {
+        // let copies already in flight land before the CTA exits
+        record_status(status, NVFP4_ERR_TIMEOUT);
+        for (int s = 0; s < kStages; ++s) {
+          if (armed_phase[s] < 0) continue;
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(&full[s], (uint32_t)armed_phase[s]) &&
+                 globaltimer_ns() - t0 < 1000000ull) {
+          }
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = make_idesc_nvf4(kBM, kBN);
+      uint32_t stage = 0, phase = 0, acc_phase = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
+        if (!mbar_wait_bounded(acc_empty, acc_phase ^ 1, abort_flag, timeout_ns)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int kt = 0; kt < nkt; ++kt) {
+          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, timeout_ns)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const int nkb = min(4, kgroups - 4 * kt);
+          const uint32_t sA = smem_u32(smem + kSmemA + stage * kABytes);
+          const uint32_t sB = smem_u32(smem + kSmemB + stage * kBBytes);
+          const uint32_t sSFA = smem_u32(smem + kSmemSFA + stage * kSFABytes);
+          const uint32_t sSFB = smem_u32(smem + kSmemSFB + stage * kSFBBytes);
+          const uint64_t adesc = smem_desc(sA, 16, 1024, 2);
+          const uint64_t bdesc = smem_desc(sB, 16, 1024, 2);
+          for (int kb = 0; kb < nkb; ++kb) {
+            tc_copy_scales(tmem + kTmemSFA + 4 * kb, smem_desc(sSFA + kb * kSFAtom, 0, 128, 0));
+            tc_copy_scales(tmem + kTmemSFB + 8 * kb, smem_desc(sSFB + kb * kSFAtom, 0, 128, 0));
+            tc_copy_scales(tmem + kTmemSFB + 8 * kb + 4,
+                           smem_desc(sSFB + kSFABytes + kb * kSFAtom, 0, 128, 0));
+            // K advance inside the 128-byte swizzle atom: 32 bytes per MMA
+            tc_mma_nvf4(tmem, adesc + (uint64_t)(2 * kb), bdesc + (uint64_t)(2 * kb), idesc,
+                        tmem + kTmemSFA + 4 * kb, tmem + kTmemSFB + 8 * kb, (kt | kb) != 0);
+          }
+          tc_commit(&empty[stage]);
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+        }
+        if (!ok) break;
+        tc_commit(acc_full);
+        acc_phase ^= 1;
+      }
+      if (!ok) {
+        record_status(status, NVFP4_ERR_TIMEOUT);
+        tc_commit(drain);  // wait (bounded) for MMAs already issued
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < 1000000ull) {
+        }
+      }
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ epilogue
+    const int q = warp & 3;          // tensor-memory lane quarter of this warp
+    const int h = (warp - 2) >> 2;   // which half of the tile's columns
+    uint32_t acc_phase = 0;
+    for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
+      if (!mbar_wait_bounded(acc_full, acc_phase, abort_flag, timeout_ns)) {
+        if (lane == 0) record_status(status, NVFP4_ERR_TIMEOUT);
+        break;
+      }
+      tc_fence_after();
+      uint32_t acc[4][32];
+      const uint32_t lane_addr = tmem + ((uint32_t)(q * 32) << 16);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) tmem_ld32(lane_addr + Prob::tmem_col(h, j), acc[j]);
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);
+      const TileJob job = prob.job(t);
+      prob.store(job, q, h, lane, acc);
+      acc_phase ^= 1;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem, kTmemCols);
+  }
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,53 @@
+// Host-side launchers of the NVFP4 kernels (internal to the library).
+#pragma once
+
+#include <cuda.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+namespace nvfp4 {
+
+constexpr int kMaxPartials = 1024;  // amax pass-1 partial slots in a workspace
+
+int amax_partial_count(int64_t n, int num_sms);
+cudaError_t launch_amax_partial(const void* x, int64_t n, uint32_t* partial, int n_partial,
+                                cudaStream_t s);
+cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, bool fos, const uint32_t* partial,
+                            int n_partial, const float* g_static, uint8_t* codes, uint8_t* scales,
+                            float* g_out, uint8_t* choice, int* status, int num_sms, cudaStream_t s);
+cudaError_t launch_fake_quant(const void* x, int64_t M, int64_t K, bool fos, const uint32_t* partial,
+                              int n_partial, const float* g_static, const uint8_t* scales_frozen,
+                              void* y, int* status, int num_sms, cudaStream_t s);
+cudaError_t launch_convert(const float* in, int64_t n, uint8_t* out, bool e4m3, int num_sms,
+                           cudaStream_t s);
+cudaError_t launch_selftest_timeout(uint64_t timeout_ns, int* status, cudaStream_t s);
+
+// Dense W4A4 GEMM (gemm.cu). Returns cudaErrorInvalidValue if a tensor map
+// cannot be encoded.
+cudaError_t launch_gemm(const uint8_t* Aq, const uint8_t* As, const float* ga, const uint8_t* Bq,
+                        const uint8_t* Bs, const float* gb, int64_t M, int64_t N, int64_t K,
+                        void* C, int* status, int num_sms, cudaStream_t s);
+
+// Routed-expert pipeline (moe.cu).
+struct MoeArgs {
+  const void* x;
+  int64_t T, H, I;
+  const int32_t* topk_ids;
+  const float* topk_w;
+  int topk, E;
+  const uint8_t *w13_q, *w13_s;
+  const float* w13_g;
+  const uint8_t *w2_q, *w2_s;
+  const float* w2_g;
+  float* out;
+  uint8_t* ws;
+};
+int64_t moe_rows_capacity(int64_t T, int topk, int E);
+cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t s);
+
+// Tensor-map encoder from the driver (resolved once through the runtime).
+CUresult encode_tensor_map_2d(CUtensorMap* map, const void* base, uint64_t inner_bytes,
+                              uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner,
+                              uint32_t box_rows);
+
+}  // namespace nvfp4

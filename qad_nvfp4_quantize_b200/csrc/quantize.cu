@@ -1,0 +1,424 @@
+// NVFP4 quantize, four_over_six calibration and fake-quant kernels.
+//
+// The format is the two-level scaling of "How is Qwen3.8-Flash-Next-NVFP4's
+// NVFP4 quantization done?" (section "Core: W4A4 two-level scaling"): an FP32
+// global scale g per tensor (level 2) and an E4M3 block scale per 16
+// contiguous elements (level 1), E2M1 element codes. four_over_six and the
+// frozen-scale fake-quant follow Table 1 and "Quantization scale handling
+// during QAD" of "Developing Nemotron 3.5 Lightning NVFP4 with QAD using
+// NVIDIA Model Optimizer".
+//
+// Work decomposition (HBM-bound streaming): a warp handles a chunk of 256
+// consecutive elements of the flattened [M x K] tensor; lane i loads 16 bytes
+// (8 BF16) with one coalesced 128-bit load, a lane pair forms one 16-element
+// block, the pair's maximum comes from one shuffle. Codes leave as one 32-bit
+// store per lane (128 contiguous bytes per warp); four consecutive block
+// scales (one 64-element group of a row) leave as one 32-bit store into the
+// tiled scale layout.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nvfp4 {
+
+constexpr int kQThreads = 256;  // 8 warps
+constexpr int kAmaxThreads = 256;
+constexpr unsigned kFull = 0xFFFFFFFFu;
+
+__device__ __forceinline__ uint4 ld_stream(const uint4* p) {
+  uint4 v;
+  asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
+// ----------------------------------------------------------------------------
+// amax, pass 1: per-CTA maximum of |x| as a BF16 magnitude (bits & 0x7FFF).
+// Magnitudes of finite BF16 values order like their bit patterns; anything
+// >= 0x7F80 is Inf or NaN, so the maximum also flags non-finite input.
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(kAmaxThreads) amax_partial_kernel(const uint4* __restrict__ x,
+                                                                    int64_t n_vec,
+                                                                    uint32_t* __restrict__ partial) {
+  uint32_t m2 = 0;  // two 16-bit magnitudes
+  const int64_t stride = (int64_t)gridDim.x * blockDim.x;
+  int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  for (; i + 3 * stride < n_vec; i += 4 * stride) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) v[u] = ld_stream(x + i + u * stride);
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      m2 = __vmaxu2(m2, v[u].x & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, v[u].y & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, v[u].z & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, v[u].w & 0x7FFF7FFFu);
+    }
+  }
+  for (; i < n_vec; i += stride) {
+    const uint4 v = ld_stream(x + i);
+    m2 = __vmaxu2(m2, v.x & 0x7FFF7FFFu);
+    m2 = __vmaxu2(m2, v.y & 0x7FFF7FFFu);
+    m2 = __vmaxu2(m2, v.z & 0x7FFF7FFFu);
+    m2 = __vmaxu2(m2, v.w & 0x7FFF7FFFu);
+  }
+  uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFull, m, o));
+  __shared__ uint32_t red[kAmaxThreads / 32];
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t r = 0;
+    for (int w = 0; w < kAmaxThreads / 32; ++w) r = max(r, red[w]);
+    partial[blockIdx.x] = r;
+  }
+}
+
+// Global scale for this call: reduce the pass-1 partials (dynamic) or read the
+// static scale. Every CTA does this redundantly (a few hundred L2 reads), so
+// no atomics and no zero-initialised scratch are needed. Returns g; sets
+// *nonfinite when the amax is Inf/NaN.
+__device__ __forceinline__ float resolve_global_scale(const uint32_t* partial, int n_partial,
+                                                      const float* g_static, bool* nonfinite) {
+  __shared__ float s_g;
+  __shared__ int s_bad;
+  if (threadIdx.x < 32) {
+    float g;
+    int bad = 0;
+    if (g_static) {
+      g = *g_static;
+    } else {
+      uint32_t m = 0;
+      for (int i = threadIdx.x; i < n_partial; i += 32) m = max(m, partial[i]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFull, m, o));
+      bad = m >= 0x7F80u;
+      g = global_scale_from_amax(__uint_as_float(m << 16));
+    }
+    if (threadIdx.x == 0) {
+      s_g = g;
+      s_bad = bad;
+    }
+  }
+  __syncthreads();
+  *nonfinite = s_bad != 0;
+  return s_g;
+}
+
+// Byte offset of scale (row, block column c) in the tiled layout; kgroups =
+// K / 64 is the number of 4-scale tiles per 128-row tile row.
+__device__ __forceinline__ int64_t scale_offset(int64_t row, int64_t c, int64_t kgroups) {
+  return (((row >> 7) * kgroups + (c >> 2)) << 9) + ((row & 31) << 4) + (((row >> 5) & 3) << 2) +
+         (c & 3);
+}
+
+// Per-lane block math. v: this lane's 8 values (half a block); g: global
+// scale; mt: target magnitude (6 or 4). Produces the scale code, packed
+// codes, dequantized values and the block's squared error (pair-wide, summed
+// in element order: the even lane's 8 terms first, then the odd lane's).
+struct HalfBlock {
+  uint32_t sc;      // E4M3 code of the block scale
+  uint32_t q;       // 8 packed E2M1 codes
+  float deq[8];     // g*s*q per element (FP32)
+  float err;        // block squared error (valid on both lanes of the pair)
+};
+
+template <bool kWantErr>
+__device__ __forceinline__ void quantize_half(const float (&v)[8], float bmax, float g, float mt,
+                                              int lane, HalfBlock& hb) {
+  hb.sc = block_scale_code(bmax, g, mt);
+  const float d = __fmul_rn(g, e4m3_value(hb.sc));
+  const float r = __frcp_rn(d);
+  float sv[8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i) sv[i] = __fmul_rn(v[i], r);
+  hb.q = e2m1_pack8(sv);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) hb.deq[i] = __fmul_rn(d, e2m1_value((hb.q >> (4 * i)) & 0xFu));
+  if (kWantErr) {
+    float sq[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      const float df = __fsub_rn(v[i], hb.deq[i]);
+      sq[i] = __fmul_rn(df, df);
+    }
+    float acc = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc = __fadd_rn(acc, sq[i]);
+    const float lo = __shfl_sync(kFull, acc, lane & ~1);  // even partner's partial sum
+    float acc2 = lo;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc2 = __fadd_rn(acc2, sq[i]);
+    hb.err = __shfl_sync(kFull, acc2, lane | 1);
+  } else {
+    hb.err = 0.0f;
+  }
+}
+
+__device__ __forceinline__ void load8(const uint4* x, int64_t vec_idx, bool valid, float (&v)[8]) {
+  uint4 w = make_uint4(0, 0, 0, 0);
+  if (valid) w = ld_stream(x + vec_idx);
+  bf16x2_to_f32(w.x, v[0], v[1]);
+  bf16x2_to_f32(w.y, v[2], v[3]);
+  bf16x2_to_f32(w.z, v[4], v[5]);
+  bf16x2_to_f32(w.w, v[6], v[7]);
+}
+
+__device__ __forceinline__ float block_max(const float (&v)[8]) {
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
+  return fmaxf(m, __shfl_xor_sync(kFull, m, 1));
+}
+
+// Gather the scale codes of the 4 blocks of a 64-element group onto the
+// group's first lane (lanes 8c .. 8c+7 hold blocks 4c .. 4c+3).
+__device__ __forceinline__ uint32_t gather_group_scales(uint32_t sc) {
+  const uint32_t s1 = __shfl_down_sync(kFull, sc, 2);
+  const uint32_t s2 = __shfl_down_sync(kFull, sc, 4);
+  const uint32_t s3 = __shfl_down_sync(kFull, sc, 6);
+  return sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+}
+
+// Zero the scale bytes of the padding rows [M, ceil128(M)).
+__device__ __forceinline__ void zero_pad_scale_rows(uint8_t* scales, int64_t M, int64_t kgroups) {
+  const int64_t pad = ((M + 127) & ~int64_t(127)) - M;
+  const int64_t total = pad * kgroups;
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int64_t row = M + i / kgroups, cg = i % kgroups;
+    *reinterpret_cast<uint32_t*>(scales + scale_offset(row, cg * 4, kgroups)) = 0u;
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Quantize (pass 2). kFos: four_over_six calibration.
+// ----------------------------------------------------------------------------
+template <bool kFos>
+__global__ void __launch_bounds__(kQThreads) quantize_kernel(
+    const uint4* __restrict__ x, int64_t M, int64_t K, const uint32_t* __restrict__ partial,
+    int n_partial, const float* __restrict__ g_static, uint32_t* __restrict__ codes,
+    uint8_t* __restrict__ scales, float* __restrict__ g_out, uint8_t* __restrict__ choice,
+    int* status) {
+  bool bad;
+  const float g = resolve_global_scale(partial, n_partial, g_static, &bad);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if (g_out) *g_out = g;
+    if (bad) record_status(status, NVFP4_ERR_NONFINITE_INPUT);
+  }
+  const int64_t kgroups = K >> 6;
+  const int64_t nblk_row = K >> 4;
+  const int64_t n = M * K;
+  const int64_t n_chunks = (n + 255) >> 8;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (int64_t)blockIdx.x * (kQThreads / 32) + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * (kQThreads / 32);
+
+  for (int64_t ch = warp; ch < n_chunks; ch += nwarps) {
+    const int64_t e0 = (ch << 8) + lane * 8;
+    const bool valid = e0 < n;
+    float v[8];
+    load8(x, e0 >> 3, valid, v);
+    const float bmax = block_max(v);
+    HalfBlock h6;
+    quantize_half<kFos>(v, bmax, g, 6.0f, lane, h6);
+    uint32_t sc = h6.sc, q = h6.q, pick4 = 0;
+    if (kFos) {
+      HalfBlock h4;
+      quantize_half<true>(v, bmax, g, 4.0f, lane, h4);
+      pick4 = h4.err < h6.err;  // tie keeps M = 6
+      if (pick4) {
+        sc = h4.sc;
+        q = h4.q;
+      }
+    }
+    const uint32_t group = gather_group_scales(sc);
+    if (valid) {
+      codes[e0 >> 3] = q;
+      const int64_t fb = e0 >> 4;  // flat block index
+      if ((lane & 7) == 0) {
+        const int64_t row = fb / nblk_row, c = fb - row * nblk_row;
+        *reinterpret_cast<uint32_t*>(scales + scale_offset(row, c, kgroups)) = group;
+      }
+      if (kFos && choice && (lane & 1) == 0) choice[fb] = (uint8_t)pick4;
+    }
+  }
+  if (!kFos && choice) {  // max mode still fills the optional choice map with 0
+    const int64_t nb = n >> 4;
+    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nb;
+         i += (int64_t)gridDim.x * blockDim.x)
+      choice[i] = 0;
+  }
+  zero_pad_scale_rows(scales, M, kgroups);
+}
+
+// ----------------------------------------------------------------------------
+// Fake-quant: y = BF16(g * s * q). Modes: dynamic/static g with computed block
+// scales (max or four_over_six), or frozen g* and s* (tiled layout).
+// ----------------------------------------------------------------------------
+template <bool kFos, bool kFrozen>
+__global__ void __launch_bounds__(kQThreads) fake_quant_kernel(
+    const uint4* __restrict__ x, int64_t M, int64_t K, const uint32_t* __restrict__ partial,
+    int n_partial, const float* __restrict__ g_static, const uint8_t* __restrict__ scales_frozen,
+    uint4* __restrict__ y, int* status) {
+  bool bad;
+  const float g = resolve_global_scale(partial, n_partial, g_static, &bad);
+  if (blockIdx.x == 0 && threadIdx.x == 0 && bad) record_status(status, NVFP4_ERR_NONFINITE_INPUT);
+  const int64_t kgroups = K >> 6;
+  const int64_t nblk_row = K >> 4;
+  const int64_t n = M * K;
+  const int64_t n_chunks = (n + 255) >> 8;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (int64_t)blockIdx.x * (kQThreads / 32) + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * (kQThreads / 32);
+
+  for (int64_t ch = warp; ch < n_chunks; ch += nwarps) {
+    const int64_t e0 = (ch << 8) + lane * 8;
+    const bool valid = e0 < n;
+    float v[8];
+    load8(x, e0 >> 3, valid, v);
+    float out[8];
+    if (kFrozen) {
+      uint32_t sc = 1;
+      if (valid) {
+        const int64_t fb = e0 >> 4;
+        const int64_t row = fb / nblk_row, c = fb - row * nblk_row;
+        sc = scales_frozen[scale_offset(row, c, kgroups)];
+      }
+      const float d = __fmul_rn(g, e4m3_value(sc));
+      const float r = __frcp_rn(d);
+      float sv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sv[i] = __fmul_rn(v[i], r);
+      const uint32_t q = e2m1_pack8(sv);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) out[i] = __fmul_rn(d, e2m1_value((q >> (4 * i)) & 0xFu));
+    } else {
+      const float bmax = block_max(v);
+      HalfBlock h6;
+      quantize_half<kFos>(v, bmax, g, 6.0f, lane, h6);
+      if (kFos) {
+        HalfBlock h4;
+        quantize_half<true>(v, bmax, g, 4.0f, lane, h4);
+        const bool pick4 = h4.err < h6.err;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) out[i] = pick4 ? h4.deq[i] : h6.deq[i];
+      } else {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) out[i] = h6.deq[i];
+      }
+    }
+    if (valid) {
+      uint4 w;
+      w.x = f32x2_to_bf16x2(out[0], out[1]);
+      w.y = f32x2_to_bf16x2(out[2], out[3]);
+      w.z = f32x2_to_bf16x2(out[4], out[5]);
+      w.w = f32x2_to_bf16x2(out[6], out[7]);
+      y[e0 >> 3] = w;
+    }
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Conversion primitives and the bounded-wait self test.
+// ----------------------------------------------------------------------------
+__global__ void convert_e2m1_kernel(const float* __restrict__ in, int64_t n, uint8_t* __restrict__ out) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    out[i] = (uint8_t)e2m1_code(in[i]);
+}
+
+__global__ void convert_e4m3_kernel(const float* __restrict__ in, int64_t n, uint8_t* __restrict__ out) {
+  for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    out[i] = (uint8_t)e4m3_code(in[i]);
+}
+
+__device__ int g_never_set_flag = 0;
+
+__global__ void selftest_timeout_kernel(uint64_t timeout_ns, int* status) {
+  if (threadIdx.x != 0) return;
+  volatile int* flag = &g_never_set_flag;
+  const uint64_t t0 = globaltimer_ns();
+  while (*flag == 0) {
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      record_status(status, NVFP4_ERR_TIMEOUT);
+      return;
+    }
+    __nanosleep(1000);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Host launchers.
+// ----------------------------------------------------------------------------
+static int grid_for(int64_t work_items, int per_block, int max_blocks) {
+  int64_t b = (work_items + per_block - 1) / per_block;
+  if (b < 1) b = 1;
+  if (b > max_blocks) b = max_blocks;
+  return (int)b;
+}
+
+int amax_partial_count(int64_t n, int num_sms) {
+  // about 4 vectors of 8 BF16 per thread per loop trip, 4 CTAs per SM at most
+  return grid_for(n / 8, kAmaxThreads * 16, num_sms * 4 > kMaxPartials ? kMaxPartials : num_sms * 4);
+}
+
+cudaError_t launch_amax_partial(const void* x, int64_t n, uint32_t* partial, int n_partial,
+                                cudaStream_t s) {
+  amax_partial_kernel<<<n_partial, kAmaxThreads, 0, s>>>(static_cast<const uint4*>(x), n / 8, partial);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, bool fos, const uint32_t* partial,
+                            int n_partial, const float* g_static, uint8_t* codes, uint8_t* scales,
+                            float* g_out, uint8_t* choice, int* status, int num_sms, cudaStream_t s) {
+  const int64_t chunks = (M * K + 255) / 256;
+  const int grid = grid_for(chunks, kQThreads / 32 * 2, num_sms * 8);
+  if (fos)
+    quantize_kernel<true><<<grid, kQThreads, 0, s>>>(static_cast<const uint4*>(x), M, K, partial, n_partial,
+                                                      g_static, reinterpret_cast<uint32_t*>(codes), scales,
+                                                      g_out, choice, status);
+  else
+    quantize_kernel<false><<<grid, kQThreads, 0, s>>>(static_cast<const uint4*>(x), M, K, partial, n_partial,
+                                                       g_static, reinterpret_cast<uint32_t*>(codes), scales,
+                                                       g_out, choice, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fake_quant(const void* x, int64_t M, int64_t K, bool fos, const uint32_t* partial,
+                              int n_partial, const float* g_static, const uint8_t* scales_frozen,
+                              void* y, int* status, int num_sms, cudaStream_t s) {
+  const int64_t chunks = (M * K + 255) / 256;
+  const int grid = grid_for(chunks, kQThreads / 32 * 2, num_sms * 8);
+  const uint4* xv = static_cast<const uint4*>(x);
+  uint4* yv = static_cast<uint4*>(y);
+  if (scales_frozen)
+    fake_quant_kernel<false, true><<<grid, kQThreads, 0, s>>>(xv, M, K, partial, n_partial, g_static,
+                                                              scales_frozen, yv, status);
+  else if (fos)
+    fake_quant_kernel<true, false><<<grid, kQThreads, 0, s>>>(xv, M, K, partial, n_partial, g_static,
+                                                              nullptr, yv, status);
+  else
+    fake_quant_kernel<false, false><<<grid, kQThreads, 0, s>>>(xv, M, K, partial, n_partial, g_static,
+                                                               nullptr, yv, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_convert(const float* in, int64_t n, uint8_t* out, bool e4m3, int num_sms,
+                           cudaStream_t s) {
+  const int grid = grid_for(n, 256, num_sms * 8);
+  if (e4m3)
+    convert_e4m3_kernel<<<grid, 256, 0, s>>>(in, n, out);
+  else
+    convert_e2m1_kernel<<<grid, 256, 0, s>>>(in, n, out);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_selftest_timeout(uint64_t timeout_ns, int* status, cudaStream_t s) {
+  selftest_timeout_kernel<<<1, 32, 0, s>>>(timeout_ns, status);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4

@@ -1,0 +1,154 @@
+"""GPU parity of conversions, quantize, four_over_six and fake-quant against
+the CPU oracle (bit-exact), through the C ABI."""
+import numpy as np
+import pytest
+import torch
+
+from oracle import nvfp4_oracle as o
+from qad_nvfp4_quantize_b200 import inputs
+from tests.util import assert_quantized_equal, bf16_np, oracle_quantized, require_gpu, to_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def nv():
+    return require_gpu()
+
+
+def _sweep_values():
+    rng = np.random.default_rng(21)
+    # every finite BF16 bit pattern (as FP32), plus random FP32 values
+    bits = np.arange(0, 1 << 16, dtype=np.uint32) << 16
+    allbf = bits.view(np.float32)
+    allbf = allbf[np.isfinite(allbf)]
+    mids = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0], np.float32)
+    near = np.concatenate([mids, np.nextafter(mids, np.float32(0)), np.nextafter(mids, np.float32(9))])
+    return np.concatenate([allbf, near, -near, rng.uniform(-8, 8, 1 << 20).astype(np.float32),
+                           (rng.standard_normal(1 << 18) * 1e-3).astype(np.float32)])
+
+
+def test_e2m1_conversion_matches_oracle(nv):
+    v = _sweep_values()
+    got = to_np(nv.convert_e2m1(torch.from_numpy(v).cuda()))
+    want = o.e2m1_encode(v)
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, f"{bad.size} differ, e.g. v={v[bad[:5]]} gpu={got[bad[:5]]} oracle={want[bad[:5]]}"
+
+
+def test_e4m3_conversion_matches_oracle(nv):
+    v = np.abs(_sweep_values()) * np.float32(64.0)
+    v = np.concatenate([v, o.e4m3_decode_table().astype(np.float32), np.array([448, 460, 464, 1e30], np.float32)])
+    got = to_np(nv.convert_e4m3(torch.from_numpy(v.astype(np.float32)).cuda()))
+    want = o.e4m3_encode(v.astype(np.float32))
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, f"{bad.size} differ, e.g. t={v[bad[:5]]} gpu={got[bad[:5]]} oracle={want[bad[:5]]}"
+
+
+@pytest.mark.parametrize("which", ["x", "w"])
+def test_quantize_tiny_linear(nv, which):
+    d = inputs.tiny_linear(0)
+    x = d[which]
+    q = nv.quantize(x.cuda(), "max")
+    assert_quantized_equal(q, oracle_quantized(bf16_np(x)), *x.shape)
+
+
+@pytest.mark.parametrize("M,K", [(1, 64), (127, 192), (200, 320), (129, 1024), (385, 5120)])
+def test_quantize_ragged_shapes(nv, M, K):
+    rng = np.random.default_rng(M * 7 + K)
+    x = inputs.to_bf16((rng.standard_t(3, (M, K)) * 0.5).astype(np.float32))
+    for mode in ("max", "four_over_six"):
+        q = nv.quantize(x.cuda(), mode, want_choice=True)
+        assert_quantized_equal(q, oracle_quantized(bf16_np(x), mode), M, K, check_choice=True)
+
+
+def test_quantize_empty(nv):
+    x = torch.empty((0, 256), dtype=torch.bfloat16, device="cuda")
+    q = nv.quantize(x)
+    assert to_np(q.g)[0] == 1.0
+
+
+def test_quantize_static_global_scale(nv):
+    d = inputs.tiny_linear(3)
+    x = bf16_np(d["x"])
+    g = np.float32(0.0007)
+    q = nv.quantize(d["x"].cuda(), "max", g=torch.tensor([g], device="cuda"))
+    assert_quantized_equal(q, oracle_quantized(x, "max", g), *x.shape)
+
+
+def test_quantize_zero_and_tiny_blocks(nv):
+    x = np.zeros((128, 256), np.float32)
+    x[0, 0] = 3.0
+    x[5, 16:32] = 1e-30          # blocks far below the tensor amax: scale floor 2^-9
+    x[7, 32:48] = -0.0
+    xt = inputs.to_bf16(x)
+    for mode in ("max", "four_over_six"):
+        q = nv.quantize(xt.cuda(), mode, want_choice=True)
+        assert_quantized_equal(q, oracle_quantized(bf16_np(xt), mode), 128, 256, check_choice=True)
+
+
+def test_four_over_six_outlier_weights(nv):
+    d = inputs.four_over_six_linear(0, M=16, N=1024, K=2048)
+    w = d["w"]
+    q = nv.quantize(w.cuda(), "four_over_six", want_choice=True)
+    ref = oracle_quantized(bf16_np(w), "four_over_six")
+    assert_quantized_equal(q, ref, *w.shape, check_choice=True)
+    assert 0 < ref["choice"].mean() < 1          # both candidates occur
+
+
+@pytest.mark.parametrize("mode", ["max", "four_over_six"])
+def test_fake_quant_dynamic(nv, mode):
+    d = inputs.four_over_six_linear(1, M=300, N=256, K=1024)
+    x = d["w"]
+    y = nv.fake_quant(x.cuda(), mode)
+    want = o.fake_quant(bf16_np(x), mode)
+    assert np.array_equal(bf16_np(y), want)
+
+
+def test_fake_quant_frozen_and_static(nv):
+    rng = np.random.default_rng(5)
+    w0 = inputs.to_bf16((rng.standard_normal((256, 512)) * 0.02).astype(np.float32))
+    q = nv.quantize(w0.cuda(), "four_over_six")
+    ref = o.quantize(bf16_np(w0), "four_over_six")
+    drift = inputs.to_bf16(bf16_np(w0) * 1.7 + (rng.standard_normal((256, 512)) * 0.01).astype(np.float32))
+    y = nv.fake_quant(drift.cuda(), g=q.g, scales=q.scales)
+    want = o.fake_quant(bf16_np(drift), g_frozen=ref["g"], scales_frozen=ref["scales"])
+    assert np.array_equal(bf16_np(y), want)
+    g = torch.tensor([np.float32(1e-4)], device="cuda")
+    y2 = nv.fake_quant(drift.cuda(), "max", g=g)
+    q2 = o.quantize(bf16_np(drift), "max", np.float32(1e-4))
+    want2 = o.bf16_round(o.dequantize(q2["codes"], q2["scales"], q2["g"]))
+    assert np.array_equal(bf16_np(y2), want2)
+
+
+def test_fake_quant_equals_dequantized_quantize(nv):
+    d = inputs.dense_mlp(2, M=64, N=16, K=512)
+    x = d["x"].cuda()
+    q = nv.quantize(x, "max")
+    y = nv.fake_quant(x, "max")
+    codes = o.unpack_codes(to_np(q.codes))
+    scales = o.scales_from_tiled(to_np(q.scales), 64, 512)
+    assert np.array_equal(bf16_np(y), o.bf16_round(o.dequantize(codes, scales, to_np(q.g)[0])))
+
+
+def test_nonfinite_input_sets_device_status(nv):
+    nv.device_status(clear=True)
+    x = torch.zeros((128, 256), dtype=torch.bfloat16, device="cuda")
+    x[3, 7] = float("inf")
+    nv.quantize(x)
+    assert nv.device_status(clear=True) == 5
+    x[3, 7] = float("nan")
+    nv.quantize(x)
+    assert nv.device_status(clear=True) == 5
+    x[3, 7] = 1.0
+    nv.quantize(x)
+    assert nv.device_status(clear=True) == 0
+
+
+def test_bounded_wait_reports_timeout(nv):
+    nv.device_status(clear=True)
+    nv.selftest_timeout(2_000_000)     # 2 ms on a flag nothing sets
+    assert nv.device_status(clear=True) == 6
+    x = torch.ones((128, 64), dtype=torch.bfloat16, device="cuda")
+    nv.quantize(x)                      # the context is still usable
+    assert nv.device_status(clear=True) == 0
