@@ -1,0 +1,483 @@
+"""Benchmark of the NVFP4 W4A4 hot path on B200.
+
+One step = dynamic NVFP4 quantization of the activations (amax pass +
+quantize/pack) followed by the block-scaled W4A4 GEMM against statically
+max-quantized weights, on the dense transformer MLP workload
+X[4096 x 5120] (Student-t df=3 * 0.5) x W_up[17408 x 5120]^T -> BF16.
+Metric: quant+GEMM TFLOP/s (2*M*N*K per step). Every other hot-path row
+(four_over_six calibration, fake-quant, lm_head decode GEMM, routed-expert
+MoE) is measured on its own workload in the "rows" object of the same line.
+
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+For N > 1 launch with torch.distributed.run; each rank runs an independent
+replica on its own GPU (weak scaling, no data-path collective).
+"""
+from __future__ import annotations
+
+import argparse
+import glob
+import hashlib
+import json
+import os
+import re
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "W4A4 NVFP4 quant+GEMM TFLOPS & % of FP4 tensor peak; quantize GB/s vs HBM"
+UNIT = "TFLOP/s"
+DENSE = dict(M=4096, N=17408, K=5120)
+L2_FLUSH_BYTES = 256 << 20
+FP4_OVER_BF16 = 4.0          # nominal dense ratio (9 PF FP4 / 2.25 PF BF16)
+FALLBACK_HBM_GBS = 6650.0
+FALLBACK_BF16_TFLOPS = 1590.0
+
+
+# ----------------------------------------------------------------------------- helpers
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm=float(p["hbm_gbs"]), bf16=float(p["bf16_tflops"]),
+                    bf16_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])), source="measured")
+    return dict(hbm=FALLBACK_HBM_GBS, bf16=FALLBACK_BF16_TFLOPS, bf16_sustained=1400.0, source="fallback")
+
+
+def kernel_sources_digest():
+    h = hashlib.sha256()
+    for p in sorted(glob.glob(os.path.join(ROOT, "qad_nvfp4_quantize_b200", "csrc", "*"))):
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel_key: str):
+    """DRAM bytes per launch recorded from an ncu capture under profiles/, valid
+    only while the kernel sources are unchanged since the capture."""
+    digest = kernel_sources_digest()
+    for path in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
+        with open(path) as f:
+            for line in f:
+                m = re.match(r"^traffic\s+(\S+)\s+bytes_per_launch=(\d+)\s+sources=(\w+)", line.strip())
+                if m and m.group(1) == kernel_key and m.group(3) == digest:
+                    return int(m.group(2))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi clock / throttle-reason samples while the timed region runs."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except (OSError, FileNotFoundError):
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append((time.time(), line.strip()))
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return self
+
+    def summary(self, t0: float, t1: float):
+        rows = []
+        for ts, line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[5:9]))
+            except ValueError:
+                continue
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        inside = [r for r in rows if t0 - 0.05 <= r[0] <= t1 + 0.05] or rows
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in inside for i, v in enumerate(r[3]) if v.lower() == "active"})
+        loaded = [r[1] for r in inside]
+        return {"sm_mhz": statistics.median(loaded), "sm_max_mhz": max(r[2] for r in inside),
+                "reasons": reasons, "samples": len(inside)}
+
+
+def flush_l2(buf: torch.Tensor):
+    buf.zero_()
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    if world == 1:
+        return 0, 1, 0
+    import datetime
+    import torch.distributed as dist
+    rank = int(os.environ["RANK"])
+    local = int(os.environ.get("LOCAL_RANK", rank))
+    backend = "nccl" if torch.cuda.is_available() else "gloo"
+    if torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return rank, world, local
+
+
+def dist_max(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    dev = torch.device("cuda", torch.cuda.current_device()) if torch.cuda.is_available() else torch.device("cpu")
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------- oracle arm
+
+def oracle_sample_step(x_rows: np.ndarray, wq: dict):
+    """Oracle quant+GEMM of a row sample against the statically quantized W."""
+    from oracle import nvfp4_oracle as o
+    q = o.quantize(x_rows, "max")
+    C, _S = o.gemm_reference(q["codes"], q["scales"], q["g"], wq["codes"], wq["scales"], wq["g"])
+    return C
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return 1
+
+
+def oracle_setup(seed: int, rows: int):
+    from oracle import nvfp4_oracle as o
+    from qad_nvfp4_quantize_b200 import inputs
+    d = inputs.dense_mlp(seed)
+    w = inputs.bf16_to_f32(d["w"])
+    wq = o.quantize(w, "max")
+    x = inputs.bf16_to_f32(d["x"][:rows])
+    return x, wq
+
+
+def cpu_baseline(seed: int, rows: int = 96):
+    x, wq = oracle_setup(seed, rows)
+    t0 = time.perf_counter()
+    oracle_sample_step(x, wq)
+    dt = time.perf_counter() - t0
+    flops = 2.0 * rows * DENSE["N"] * DENSE["K"]
+    return {"value": flops / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+            "sample": f"{rows} of 4096 activation rows: oracle quantize + FP64 GEMM against all 17408 "
+                      f"statically quantized weight rows ({dt:.1f} s)"}
+
+
+def run_reference(args, rank, world):
+    if rank != 0:
+        return 0
+    rows = 32
+    x, wq = oracle_setup(0, rows)
+    for _ in range(args.warmup):
+        oracle_sample_step(x, wq)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_sample_step(x, wq)
+    dt = time.perf_counter() - t0
+    flops = 2.0 * rows * DENSE["N"] * DENSE["K"] * args.steps
+    val = flops / dt / 1e12
+    line = {"metric": METRIC, "value": val, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": dt / args.steps * 1e3, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic", "impl": "reference",
+            "config": {"workload": "dense_mlp", "M": DENSE["M"], "N": DENSE["N"], "K": DENSE["K"],
+                       "step_sample_rows": rows},
+            "cpu_baseline": {"value": val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
+                             "sample": f"{rows} activation rows per step (oracle quantize + FP64 GEMM)"},
+            "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+def parity_gate(nv, x_dev, xq, wq, w_cpu_rows=None):
+    """Verify before timing: quantized activations of sampled rows bit-exact,
+    GEMM of sampled rows within tolerance (oracle on the same inputs)."""
+    from oracle import nvfp4_oracle as o
+    rows = np.array([0, 1, 1000, 2047, 4095])
+    M, K = x_dev.shape
+    x = x_dev.float().cpu().numpy()
+    ref = o.quantize(x, "max")          # full tensor: the global scale depends on every row
+    codes = o.unpack_codes(xq.codes[rows].cpu().numpy())
+    if not np.array_equal(codes, ref["codes"][rows]):
+        return "activation codes differ from the oracle"
+    if xq.g.item() != ref["g"]:
+        return "global scale differs from the oracle"
+    C = nv.gemm(xq, wq)[rows].float().cpu().numpy()
+    wc = o.unpack_codes(wq.codes.cpu().numpy())
+    ws = o.scales_from_tiled(wq.scales.cpu().numpy(), wq.rows, K)
+    C_ref, S = o.gemm_reference(ref["codes"][rows], ref["scales"][rows], ref["g"], wc, ws, wq.g.item())
+    if np.any(np.abs(C - C_ref) > o.gemm_tolerance(C_ref, S)):
+        return "GEMM outside tolerance"
+    return None
+
+
+def time_loop(fn, steps, warmup, flush_buf, stream, marks=0):
+    """Run warmup, then `steps` timed steps with the L2 flushed before each;
+    per-step CUDA events on `stream` exclude the flush. fn(evs) records its own
+    intermediate events into evs (list of `marks` events)."""
+    for _ in range(warmup):
+        flush_l2(flush_buf)
+        fn([torch.cuda.Event(enable_timing=True) for _ in range(marks)])
+    torch.cuda.synchronize()
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
+    mids = [[torch.cuda.Event(enable_timing=True) for _ in range(marks)] for _ in range(steps)]
+    for i in range(steps):
+        flush_l2(flush_buf)
+        starts[i].record(stream)
+        fn(mids[i])
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    total = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    seg = []
+    for i in range(steps):
+        pts = [starts[i]] + mids[i] + [ends[i]]
+        seg.append([pts[j].elapsed_time(pts[j + 1]) for j in range(len(pts) - 1)])
+    return total, seg
+
+
+def measure_rows(nv, peaks, flush_buf, stream, iters=10):
+    """Each other hot-path row on its own workload (device time, L2 flushed)."""
+    from qad_nvfp4_quantize_b200 import inputs
+    rows = {}
+    hbm = peaks["hbm"]
+    fp4_peak = peaks["bf16"] * FP4_OVER_BF16
+
+    # four_over_six static calibration + QAD fake-quant + W4A4 GEMM (W 14336x4096, X 16384x4096)
+    d = inputs.four_over_six_linear(0)
+    w = d["w"].cuda()
+    x = d["x"].cuda()
+    del d
+    wq = nv.quantize(w, "four_over_six", want_choice=True)
+    tot, _ = time_loop(lambda ev: nv.quantize(w, "four_over_six", want_choice=True, out=wq), iters, 2, flush_buf, stream)
+    t = statistics.median(tot) * 1e-3
+    n = w.numel()
+    alg = n * (2 + 0.5 + 1 / 16 + 1 / 16)     # read W, write codes, scales, choice
+    rows["four_over_six_calibration"] = {"workload": "W 14336x4096 BF16, 0.1% entries x20", "ms": t * 1e3,
+                                         "GB/s": alg / t / 1e9, "frac_hbm": alg / t / 1e9 / hbm,
+                                         "algorithmic_bytes": alg}
+    y = torch.empty_like(x)
+    tot, _ = time_loop(lambda ev: nv.fake_quant(x, "max", out=y), iters, 2, flush_buf, stream)
+    t = statistics.median(tot) * 1e-3
+    alg = x.numel() * 4.0
+    rows["fake_quant_dynamic"] = {"workload": "X 16384x4096 BF16 -> BF16", "ms": t * 1e3, "GB/s": alg / t / 1e9,
+                                  "frac_hbm": alg / t / 1e9 / hbm, "algorithmic_bytes": alg}
+    xq = nv.quantize(x)
+    tot, _ = time_loop(lambda ev: nv.quantize(x, out=xq), iters, 2, flush_buf, stream)
+    t = statistics.median(tot) * 1e-3
+    alg = x.numel() * 2.5625
+    rows["quantize_dynamic_cfg5_x"] = {"workload": "X 16384x4096 BF16 (larger than L2)", "ms": t * 1e3,
+                                       "GB/s": alg / t / 1e9, "frac_hbm": alg / t / 1e9 / hbm,
+                                       "algorithmic_bytes": alg}
+    C = torch.empty((x.shape[0], w.shape[0]), dtype=torch.bfloat16, device="cuda")
+    tot, _ = time_loop(lambda ev: nv.gemm(xq, wq, out=C), iters, 2, flush_buf, stream)
+    t = statistics.median(tot) * 1e-3
+    fl = 2.0 * x.shape[0] * w.shape[0] * x.shape[1]
+    rows["gemm_fos_16384x14336x4096"] = {"ms": t * 1e3, "TFLOP/s": fl / t / 1e12, "frac_fp4_peak": fl / t / 1e12 / fp4_peak}
+    del w, x, y, xq, wq, C
+    torch.cuda.empty_cache()
+
+    # lm_head decode: X 128x2048, W 151936x2048 (HBM-bound weight streaming)
+    d = inputs.lm_head(0)
+    w = d["w"].cuda()
+    x = d["x"].cuda()
+    wq = nv.quantize(w)
+    xq = nv.quantize(x)
+    C = torch.empty((128, w.shape[0]), dtype=torch.bfloat16, device="cuda")
+    tot, _ = time_loop(lambda ev: nv.gemm(xq, wq, out=C), iters, 2, flush_buf, stream)
+    t = statistics.median(tot) * 1e-3
+    M, N, K = 128, w.shape[0], 2048
+    alg = N * K * 0.5625 + M * K * 0.5625 + M * N * 2
+    rows["lm_head_gemm"] = {"workload": "128x151936x2048", "ms": t * 1e3, "TFLOP/s": 2.0 * M * N * K / t / 1e12,
+                            "GB/s": alg / t / 1e9, "frac_hbm": alg / t / 1e9 / hbm, "algorithmic_bytes": alg}
+    del w, x, wq, xq, C, d
+    torch.cuda.empty_cache()
+
+    # routed experts: T=8192, H=2048, E=256, top-8, I=512
+    d = inputs.moe_experts(0)
+    x = d["x"].cuda()
+    ids = d["topk_ids"].cuda()
+    tw = d["topk_w"].cuda()
+    w13, g13 = nv.quantize_experts(d["w13"].cuda())
+    w2, g2 = nv.quantize_experts(d["w2"].cuda())
+    del d
+    out, ws = nv.moe_grouped_gemm(x, ids, tw, 512, w13, g13, w2, g2)
+    tot, _ = time_loop(lambda ev: nv.moe_grouped_gemm(x, ids, tw, 512, w13, g13, w2, g2, out=out, workspace=ws),
+                       iters, 2, flush_buf, stream)
+    t = statistics.median(tot) * 1e-3
+    T, H, E, I = 8192, 2048, 256, 512
+    alg = T * H * 2 + E * (2 * I * H + H * I) * 0.5625 + T * H * 4
+    fl = 2.0 * T * 8 * (2 * I * H + H * I)
+    rows["moe_routed_experts"] = {"workload": "T8192 H2048 E256 top8 I512", "ms": t * 1e3,
+                                  "TFLOP/s": fl / t / 1e12, "GB/s": alg / t / 1e9, "frac_hbm": alg / t / 1e9 / hbm,
+                                  "algorithmic_bytes": alg}
+    return rows
+
+
+def run_gpu(args, rank, world, local):
+    import qad_nvfp4_quantize_b200 as nv
+    from qad_nvfp4_quantize_b200 import inputs
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    nv.check_device()
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+    M, N, K = DENSE["M"], DENSE["N"], DENSE["K"]
+
+    d = inputs.dense_mlp(seed=rank)
+    x_host = d["x"].pin_memory()
+    x = d["x"].to(dev)
+    w = d["w"].to(dev)
+    del d
+    wq = nv.quantize(w, "max")                    # static weights, quantized offline
+    del w
+    xq = nv.quantize(x, "max")
+    C = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+    err = parity_gate(nv, x, xq, wq)
+    if err is not None:
+        print(json.dumps({"metric": METRIC, "error": f"parity check failed before timing: {err}"}), flush=True)
+        return 1
+    flush_buf = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=dev)
+
+    def step(ev):
+        nv.quantize(x, "max", out=xq)
+        if ev:
+            ev[0].record(stream)
+        nv.gemm(xq, wq, out=C)
+
+    sampler = ClockSampler(local).start()
+    barrier(world)
+    torch.cuda.synchronize()
+    t_wall0 = time.time()
+    total, seg = time_loop(step, args.steps, args.warmup, flush_buf, stream, marks=1)
+    t_wall1 = time.time()
+    barrier(world)
+    torch.cuda.synchronize()
+    step_ms = dist_max(float(np.mean(total)), world)
+    sampler.stop()
+    clocks = sampler.summary(t_wall0, t_wall1)
+    quant_ms = float(np.mean([s[0] for s in seg]))
+    gemm_ms = float(np.mean([s[1] for s in seg]))
+    flops = 2.0 * M * N * K
+    value = flops * world / (step_ms * 1e-3) / 1e12
+
+    # e2e through the public API with host buffers: H2D of X, quant + GEMM, D2H of C
+    C_host = torch.empty((M, N), dtype=torch.bfloat16, pin_memory=True)
+    x_stage = torch.empty_like(x)
+
+    def e2e_step(ev):
+        x_stage.copy_(x_host, non_blocking=True)
+        nv.quantize(x_stage, "max", out=xq)
+        nv.gemm(xq, wq, out=C)
+        C_host.copy_(C, non_blocking=True)
+
+    e2e_steps = max(3, min(args.steps, 50))
+    e_tot, _ = time_loop(e2e_step, e2e_steps, max(3, min(args.warmup, 5)), flush_buf, stream)
+    e2e_ms = dist_max(float(np.mean(e_tot)), world)
+    e2e_val = flops * world / (e2e_ms * 1e-3) / 1e12
+
+    fp4_peak = peaks["bf16"] * FP4_OVER_BF16
+    achieved = flops / (gemm_ms * 1e-3) / 1e12
+    roofline = {"bound": "tensor", "kernel": "nvf4_gemm_kernel<DenseProblem>", "achieved": achieved,
+                "peak": fp4_peak, "unit": "TFLOP/s", "frac": achieved / fp4_peak,
+                "traffic": recorded_traffic("gemm_dense_mlp"),
+                "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16']} x {FP4_OVER_BF16} (nominal FP4/BF16)",
+                "algorithmic_flops_per_launch": flops}
+    quant_bytes = M * K * 2.5625
+    line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": step_ms, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "nvfp4 (e2m1 x e2m1, ue4m3 block scales, fp32 accumulate)",
+            "data": "synthetic",
+            "config": {"workload": "dense_mlp: X 4096x5120 Student-t(3)*0.5 -> NVFP4 dynamic quantize; "
+                                   "W_up 17408x5120 N(0,0.02) static max NVFP4; C BF16 4096x17408",
+                       "M": M, "N": N, "K": K, "l2": "flushed (256 MiB write) before every step, outside the "
+                                                       "step's events", "parallelism": f"replicas x{world}"},
+            "roofline": roofline,
+            "quantize": {"ms": quant_ms, "GB/s": quant_bytes / (quant_ms * 1e-3) / 1e9,
+                         "frac_hbm": quant_bytes / (quant_ms * 1e-3) / 1e9 / peaks["hbm"],
+                         "algorithmic_bytes": quant_bytes, "peak_GB/s": peaks["hbm"]},
+            "gemm_ms": gemm_ms,
+            "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": x.numel() * 2,
+                    "d2h_bytes_per_step": C.numel() * 2, "ms_per_step": e2e_ms},
+            "gpu_launches": 3 * args.steps,
+            "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"],
+                       "samples": clocks["samples"]},
+            "wall_s_timed_region": t_wall1 - t_wall0}
+    if world == 1 and not args.no_rows:
+        del x_stage, C_host
+        line["rows"] = measure_rows(nv, peaks, flush_buf, stream)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(0)
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-rows", action="store_true", help="skip the per-row measurements")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    rank, world, local = dist_setup()
+    try:
+        if args.impl == "reference":
+            rc = run_reference(args, rank, world)
+        else:
+            rc = run_gpu(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    sys.exit(rc)
+
+
+if __name__ == "__main__":
+    main()

@@ -19,7 +19,7 @@ __all__ = [
     "MODE_MAX", "MODE_FOUR_OVER_SIX", "NVFP4Error", "Quantized", "lib", "library_path",
     "check_device", "scale_bytes", "quantize", "fake_quant", "gemm", "moe_grouped_gemm",
     "moe_workspace_layout", "convert_e2m1", "convert_e4m3", "device_status", "selftest_timeout",
-    "quantize_workspace_bytes", "moe_workspace_bytes",
+    "quantize_workspace_bytes", "moe_workspace_bytes", "quantize_experts",
 ]
 
 MODE_MAX = 0
@@ -209,6 +209,23 @@ def gemm(a: Quantized, b: Quantized, out: Optional[torch.Tensor] = None) -> torc
                           a.rows, b.rows, a.K, _ptr(C), _stream(dev))
     _check(st, "nvfp4_gemm")
     return C
+
+
+def quantize_experts(w: torch.Tensor, mode="max") -> tuple:
+    """Static per-expert weight quantization of w [E, N, K] (BF16, CUDA): one
+    global scale per expert. Returns (Quantized over the E*N rows with the E
+    tiled scale buffers concatenated, g [E] FP32)."""
+    w = _cuda(w, "w", torch.bfloat16)
+    E, N, K = w.shape
+    dev = w.device
+    sb = scale_bytes(N, K)
+    codes = torch.empty((E * N, K // 2), dtype=torch.uint8, device=dev)
+    scales = torch.empty(E * sb, dtype=torch.uint8, device=dev)
+    g = torch.empty(E, dtype=torch.float32, device=dev)
+    for e in range(E):
+        quantize(w[e], mode, out=Quantized(codes[e * N:(e + 1) * N], scales[e * sb:(e + 1) * sb],
+                                           g[e:e + 1], None, N, K))
+    return Quantized(codes, scales, g, None, E * N, K), g
 
 
 def moe_workspace_layout(T: int, H: int, I: int, E: int, topk: int) -> dict:

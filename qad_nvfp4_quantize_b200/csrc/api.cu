@@ -66,6 +66,16 @@ nvfp4_status run_amax(const void* x, int64_t n, void* ws, size_t ws_bytes, int n
 
 }  // namespace
 
+int nvfp4::current_device_context(int* num_sms, int** status) {
+  DeviceInfo* d;
+  const nvfp4_status st = current_device(&d);
+  if (st == NVFP4_OK) {
+    *num_sms = d->num_sms;
+    *status = d->status;
+  }
+  return st;
+}
+
 extern "C" {
 
 int nvfp4_version(void) { return 100; }

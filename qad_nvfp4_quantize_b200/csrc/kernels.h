@@ -45,6 +45,10 @@ struct MoeArgs {
 int64_t moe_rows_capacity(int64_t T, int topk, int E);
 cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t s);
 
+// Current device: the sm_100 gate, SM count and the address of the device
+// status word (api.cu). Returns NVFP4_OK or the gate's error code.
+int current_device_context(int* num_sms, int** status);
+
 // Tensor-map encoder from the driver (resolved once through the runtime).
 CUresult encode_tensor_map_2d(CUtensorMap* map, const void* base, uint64_t inner_bytes,
                               uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner,

@@ -1,0 +1,613 @@
+// Routed-expert (MoE) layer in NVFP4 W4A4.
+//
+// The routed experts are the tensors the pages quantize first: 99.2% of the
+// quantized tensors in "2. PTQ" of "Model-Optimizer in practice: recovering
+// Qwen3.6-35B-A3B W4A4 NVFP4 accuracy with QAD" (fused gate/up and down
+// projections), and the only ones in "How is Qwen3.8-Flash-Next-NVFP4's NVFP4
+// quantization done?" (top-k routing, dynamic activation quantization,
+// section "the A4 side: dynamic activations").
+//
+// Pipeline (all on the caller's stream, no host synchronisation):
+//   1 route      stable counting sort of the T*topk (token, slot) pairs by
+//                expert; expert segments padded to 128 rows; per-m-tile
+//                expert table; per-expert amax slots zeroed.
+//   2 token pass per token: row amax -> per-expert amax (atomicMax over the
+//                experts it is routed to); zero the output row.
+//   3 gather+quantize  each padded row gets its token's x quantized with its
+//                expert's dynamic global scale (pad rows: zero codes/scales).
+//   4 gate_up    grouped tcgen05 GEMM; a tile holds 128 gate and the matching
+//                128 up columns; epilogue h = SiLU(gate)*up -> BF16, plus the
+//                per-expert amax of h.
+//   5 quantize h per expert, dynamic global scale.
+//   6 down       grouped tcgen05 GEMM; epilogue scales by the routing weight
+//                and adds into out[token] in FP32 (vector atomics).
+#include <mutex>
+
+#include "gemm_kernel.cuh"
+#include "kernels.h"
+
+namespace nvfp4 {
+
+namespace {
+
+constexpr unsigned kFullMask = 0xFFFFFFFFu;
+
+int64_t align256(int64_t v) { return (v + 255) & ~int64_t(255); }
+
+int64_t scale_bytes_(int64_t rows, int64_t K) { return ((rows + 127) / 128) * (K / 64) * 512; }
+
+// Byte offset of (row, block column c) in the tiled scale layout.
+__device__ __forceinline__ int64_t sf_offset(int64_t row, int64_t c, int64_t kgroups) {
+  return (((row >> 7) * kgroups + (c >> 2)) << 9) + ((row & 31) << 4) + (((row >> 5) & 3) << 2) + (c & 3);
+}
+
+}  // namespace
+
+// Workspace layout (all regions 256-byte aligned).
+struct MoeLayout {
+  int64_t R, P;
+  int64_t counts, offsets, cursor, row_pair, tile_expert, tile_count, amax_x, amax_h;
+  int64_t xq_codes, xq_scales, xq_g, h, hq_codes, hq_scales, hq_g, total;
+};
+
+int64_t moe_rows_capacity(int64_t T, int topk, int E) {
+  const int64_t P = T * topk;
+  return ((P + (int64_t)E * 127 + 127) / 128) * 128;
+}
+
+static MoeLayout moe_layout(int64_t T, int64_t H, int64_t I, int E, int topk) {
+  MoeLayout L;
+  L.P = T * topk;
+  L.R = moe_rows_capacity(T, topk, E);
+  int64_t o = 0;
+  auto take = [&o](int64_t bytes) {
+    const int64_t at = o;
+    o = align256(o + bytes);
+    return at;
+  };
+  L.counts = take(4 * (int64_t)E);
+  L.offsets = take(4 * ((int64_t)E + 1));
+  L.cursor = take(4 * (int64_t)E);
+  L.row_pair = take(4 * L.R);
+  L.tile_expert = take(4 * (L.R / 128));
+  L.tile_count = take(4);
+  L.amax_x = take(4 * (int64_t)E);
+  L.amax_h = take(4 * (int64_t)E);
+  L.xq_codes = take(L.R * H / 2);
+  L.xq_scales = take(scale_bytes_(L.R, H));
+  L.xq_g = take(4 * (int64_t)E);
+  L.h = take(L.R * I * 2);
+  L.hq_codes = take(L.R * I / 2);
+  L.hq_scales = take(scale_bytes_(L.R, I));
+  L.hq_g = take(4 * (int64_t)E);
+  L.total = o;
+  return L;
+}
+
+// ----------------------------------------------------------------------------
+// 1. Routing: one CTA of 1024 threads (32 warps). Warp w owns the contiguous
+// pair range [w*P/32, (w+1)*P/32); per-warp histograms give each warp its base
+// position inside every expert segment, and inside a warp pairs are ranked
+// with __match_any_sync, so the sort is stable (increasing pair index within
+// an expert, as a counting sort).
+// ----------------------------------------------------------------------------
+constexpr int kRouteThreads = 1024;
+constexpr int kRouteWarps = kRouteThreads / 32;
+
+__global__ void __launch_bounds__(kRouteThreads, 1) moe_route_kernel(
+    const int32_t* __restrict__ topk_ids, int64_t P, int E, int64_t R, int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, int32_t* __restrict__ row_pair, int32_t* __restrict__ tile_expert,
+    int32_t* __restrict__ tile_count, uint32_t* __restrict__ amax_x, uint32_t* __restrict__ amax_h,
+    int* status) {
+  extern __shared__ int32_t sh[];
+  int32_t* wcount = sh;                           // [kRouteWarps][E]
+  int32_t* seg = sh + kRouteWarps * E;            // [E+1] padded offsets
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kRouteWarps * E; i += blockDim.x) wcount[i] = 0;
+  for (int64_t i = threadIdx.x; i < R; i += blockDim.x) row_pair[i] = -1;
+  __syncthreads();
+
+  const int64_t lo = P * warp / kRouteWarps, hi = P * (warp + 1) / kRouteWarps;
+  bool bad = false;
+  for (int64_t p = lo + lane; p < hi; p += 32) {
+    const int e = topk_ids[p];
+    if (e < 0 || e >= E) {
+      bad = true;
+      continue;
+    }
+    atomicAdd(&wcount[warp * E + e], 1);
+  }
+  if (bad) record_status(status, NVFP4_ERR_INVALID_ARG);
+  __syncthreads();
+
+  // per expert: total count, padded segment size; exclusive scan over experts
+  // (thread e handles expert e; E <= 1024) and per-warp bases.
+  int32_t total = 0;
+  if (threadIdx.x < E) {
+    const int e = threadIdx.x;
+    for (int w = 0; w < kRouteWarps; ++w) {
+      const int32_t c = wcount[w * E + e];
+      wcount[w * E + e] = total;  // exclusive prefix over warps
+      total += c;
+    }
+    counts[e] = total;
+    seg[e] = (total + 127) & ~127;
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int32_t run = 0;
+    for (int e = 0; e < E; ++e) {
+      const int32_t sz = seg[e];
+      seg[e] = run;
+      run += sz;
+    }
+    seg[E] = run;
+    *tile_count = run / 128;
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) offsets[e] = seg[e];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    amax_x[e] = 0u;
+    amax_h[e] = 0u;
+    const int32_t t0 = seg[e] / 128, t1 = seg[e + 1] / 128;
+    for (int t = t0; t < t1; ++t) tile_expert[t] = e;
+  }
+  // placement, in pair order within each warp's range
+  for (int64_t base = lo; base < hi; base += 32) {
+    const int64_t p = base + lane;
+    const bool valid = p < hi;
+    int e = valid ? topk_ids[p] : -1;
+    if (e >= E) e = -1;
+    const unsigned same = __match_any_sync(kFullMask, e);
+    const int rank = __popc(same & ((1u << lane) - 1u));
+    const int leader = __ffs(same) - 1;
+    if (e >= 0) {
+      const int32_t pos = seg[e] + wcount[warp * E + e] + rank;
+      row_pair[pos] = (int32_t)p;
+    }
+    __syncwarp();
+    if (e >= 0 && lane == leader) wcount[warp * E + e] += __popc(same);
+    __syncwarp();
+  }
+}
+
+// ----------------------------------------------------------------------------
+// 2. Token pass: row amax of x[t] -> atomicMax into the amax of every expert
+// the token is routed to; zero out[t]. One warp per token.
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) moe_token_pass_kernel(const uint4* __restrict__ x, int64_t T, int64_t H,
+                                                              const int32_t* __restrict__ topk_ids, int topk,
+                                                              int E, uint32_t* __restrict__ amax_x,
+                                                              float4* __restrict__ out) {
+  const int lane = threadIdx.x & 31;
+  const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += nw) {
+    const uint4* row = x + t * (H / 8);
+    uint32_t m2 = 0;
+    for (int64_t i = lane; i < H / 8; i += 32) {
+      const uint4 v = row[i];
+      m2 = __vmaxu2(m2, v.x & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, v.y & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, v.z & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, v.w & 0x7FFF7FFFu);
+    }
+    uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFullMask, m, o));
+    if (lane < topk) {
+      const int e = topk_ids[t * topk + lane];
+      if (e >= 0 && e < E) atomicMax(&amax_x[e], m);
+    }
+    float4* orow = out + t * (H / 4);
+    for (int64_t i = lane; i < H / 4; i += 32) orow[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// 3 / 5. Row-gathered quantization with a per-expert dynamic global scale.
+// A warp quantizes 256 consecutive elements of one padded row (lane = 8
+// elements, lane pair = one 16-element block). Source row of padded row p:
+// kGather ? x[row_pair[p] / topk] : src[p]; pad rows get zero codes and scales.
+// amax_bits[e] is the BF16 magnitude (kGather) or FP32 bits (h) of the amax.
+// ----------------------------------------------------------------------------
+template <bool kGather>
+__global__ void __launch_bounds__(256) moe_quantize_rows_kernel(
+    const uint4* __restrict__ src, int64_t K, int topk, const int32_t* __restrict__ row_pair,
+    const int32_t* __restrict__ tile_expert, const int32_t* __restrict__ tile_count,
+    const uint32_t* __restrict__ amax_bits, int E, uint32_t* __restrict__ codes, uint8_t* __restrict__ scales,
+    float* __restrict__ g_out, int* status) {
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = (int64_t)(*tile_count) * 128;
+  const int64_t chunks_per_row = (K + 255) / 256;
+  const int64_t kgroups = K / 64;
+  const int64_t n_chunks = rows * chunks_per_row;
+  if (blockIdx.x == 0) {
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      const uint32_t a = amax_bits[e];
+      const float amax = kGather ? __uint_as_float(a << 16) : __uint_as_float(a);
+      if (kGather ? a >= 0x7F80u : !(amax <= 3.0e38f)) record_status(status, NVFP4_ERR_NONFINITE_INPUT);
+      g_out[e] = global_scale_from_amax(amax);
+    }
+  }
+  const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
+  for (int64_t ch = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); ch < n_chunks; ch += nw) {
+    const int64_t p = ch / chunks_per_row;
+    const int64_t col0 = (ch - p * chunks_per_row) * 256;
+    const int32_t pair = row_pair[p];
+    const int e = tile_expert[p >> 7];
+    const uint32_t a = amax_bits[e];
+    const float g = global_scale_from_amax(kGather ? __uint_as_float(a << 16) : __uint_as_float(a));
+    const int64_t e0 = col0 + lane * 8;  // element within the row
+    const bool in_row = e0 < K;          // K % 64 == 0: whole 64-element groups
+    const bool active = pair >= 0 && in_row;
+    float v[8];
+    {
+      uint4 w = make_uint4(0, 0, 0, 0);
+      if (active) {
+        const int64_t srow = kGather ? (int64_t)(pair / topk) : p;
+        w = src[(srow * K + e0) >> 3];
+      }
+      bf16x2_to_f32(w.x, v[0], v[1]);
+      bf16x2_to_f32(w.y, v[2], v[3]);
+      bf16x2_to_f32(w.z, v[4], v[5]);
+      bf16x2_to_f32(w.w, v[6], v[7]);
+    }
+    float m = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
+    const float bmax = fmaxf(m, __shfl_xor_sync(kFullMask, m, 1));  // all lanes, uniform
+    uint32_t q = 0, sc = 0;
+    if (active) {
+      sc = block_scale_code(bmax, g, 6.0f);
+      const float d = __fmul_rn(g, e4m3_value(sc));
+      const float r = __frcp_rn(d);
+      float sv[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) sv[i] = __fmul_rn(v[i], r);
+      q = e2m1_pack8(sv);
+    }
+    const uint32_t s1 = __shfl_down_sync(kFullMask, sc, 2);
+    const uint32_t s2 = __shfl_down_sync(kFullMask, sc, 4);
+    const uint32_t s3 = __shfl_down_sync(kFullMask, sc, 6);
+    if (!in_row) continue;
+    codes[(p * K + e0) >> 3] = q;
+    if ((lane & 7) == 0)
+      *reinterpret_cast<uint32_t*>(scales + sf_offset(p, e0 >> 4, kgroups)) = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// 4. gate_up grouped GEMM problem. Tiles are n-fastest: the I/128 column tiles
+// of one m-tile run on neighbouring CTAs (A read once), and the m-tiles of an
+// expert are adjacent (its weight tiles are re-read from L2).
+// ----------------------------------------------------------------------------
+struct GateUpProblem {
+  int K;             // H
+  int I;
+  int n_tiles;       // I / 128
+  int kgroups;       // H / 64
+  int64_t sf_expert_bytes;
+  const int32_t* tile_count;
+  const int32_t* tile_expert;
+  const uint8_t* sfa;      // xq scales
+  const uint8_t* sfb;      // w13 scales
+  const float* ga;         // xq_g [E]
+  const float* gb;         // w13_g [E]
+  __nv_bfloat16* h;        // [R][I]
+  uint32_t* amax_h;
+
+  __device__ __forceinline__ int num_tiles() const { return (*tile_count) * n_tiles; }
+
+  __device__ __forceinline__ TileJob job(int t) const {
+    const int mt = t / n_tiles, nt = t - mt * n_tiles;
+    const int e = tile_expert[mt];
+    const size_t rt = (size_t)kgroups * kSFAtom;
+    TileJob j;
+    j.a_row = mt * 128;
+    j.b_row0 = e * 2 * I + nt * 128;
+    j.b_row1 = e * 2 * I + I + nt * 128;
+    j.sfa = sfa + (size_t)mt * rt;
+    const uint8_t* sfe = sfb + (size_t)e * sf_expert_bytes;
+    j.sfb0 = sfe + (size_t)nt * rt;
+    j.sfb1 = sfe + (size_t)(I / 128 + nt) * rt;
+    j.expert = e;
+    j.m0 = mt * 128;
+    j.n0 = nt * 128;
+    return j;
+  }
+
+  // gate columns [h*64, h*64+64) and the matching up columns 128 later
+  __device__ static constexpr uint32_t tmem_col(int h, int j) {
+    return (uint32_t)(j < 2 ? h * 64 + 32 * j : 128 + h * 64 + 32 * (j - 2));
+  }
+
+  __device__ __forceinline__ void store(const TileJob& job, int q, int hh, int lane,
+                                        const uint32_t (&acc)[4][32]) const {
+    const int row = job.m0 + q * 32 + lane;
+    const float alpha = __fmul_rn(ga[job.expert], gb[job.expert]);
+    __nv_bfloat16* hrow = h + (size_t)row * I + job.n0 + hh * 64;
+    uint32_t mx = 0;
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+#pragma unroll
+      for (int c = 0; c < 32; c += 8) {
+        uint32_t packed[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          float hv[2];
+#pragma unroll
+          for (int k = 0; k < 2; ++k) {
+            const float z = __fmul_rn(__uint_as_float(acc[j][c + 2 * u + k]), alpha);
+            const float up = __fmul_rn(__uint_as_float(acc[j + 2][c + 2 * u + k]), alpha);
+            const float silu = __fdiv_rn(z, __fadd_rn(1.0f, expf(-z)));
+            hv[k] = __fmul_rn(silu, up);
+          }
+          packed[u] = f32x2_to_bf16x2(hv[0], hv[1]);
+          mx = __vmaxu2(mx, packed[u] & 0x7FFF7FFFu);
+        }
+        *reinterpret_cast<uint4*>(hrow + 32 * j + c) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+      }
+    }
+    uint32_t m = max(mx & 0xFFFFu, mx >> 16);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFullMask, m, o));
+    if (lane == 0) atomicMax(&amax_h[job.expert], m << 16);  // FP32 bits of the BF16 amax
+  }
+};
+
+// ----------------------------------------------------------------------------
+// 6. down grouped GEMM problem: out[token] += w * (g_h * g_w2) * acc.
+// ----------------------------------------------------------------------------
+struct DownProblem {
+  int K;             // I
+  int H;
+  int n_tiles;       // ceil(H / 256)
+  int kgroups;       // I / 64
+  int topk;
+  int64_t sf_expert_bytes;
+  const int32_t* tile_count;
+  const int32_t* tile_expert;
+  const int32_t* row_pair;
+  const float* topk_w;
+  const uint8_t* sfa;      // hq scales
+  const uint8_t* sfb;      // w2 scales
+  const float* ga;         // hq_g [E]
+  const float* gb;         // w2_g [E]
+  float* out;
+
+  __device__ __forceinline__ int num_tiles() const { return (*tile_count) * n_tiles; }
+
+  __device__ __forceinline__ TileJob job(int t) const {
+    const int mt = t / n_tiles, nt = t - mt * n_tiles;
+    const int e = tile_expert[mt];
+    const size_t rt = (size_t)kgroups * kSFAtom;
+    TileJob j;
+    j.a_row = mt * 128;
+    j.b_row0 = e * H + nt * 256;
+    j.b_row1 = e * H + nt * 256 + 128;
+    j.sfa = sfa + (size_t)mt * rt;
+    const uint8_t* sfe = sfb + (size_t)e * sf_expert_bytes;
+    j.sfb0 = sfe + (size_t)(2 * nt) * rt;
+    j.sfb1 = (nt * 256 + 128 < H) ? sfe + (size_t)(2 * nt + 1) * rt : nullptr;
+    j.expert = e;
+    j.m0 = mt * 128;
+    j.n0 = nt * 256;
+    return j;
+  }
+
+  __device__ static constexpr uint32_t tmem_col(int h, int j) { return (uint32_t)(h * 128 + 32 * j); }
+
+  __device__ __forceinline__ void store(const TileJob& job, int q, int hh, int lane,
+                                        const uint32_t (&acc)[4][32]) const {
+    const int row = job.m0 + q * 32 + lane;
+    const int32_t pair = row_pair[row];
+    if (pair < 0) return;
+    const float alpha = __fmul_rn(ga[job.expert], gb[job.expert]);
+    const float w = topk_w[pair];
+    float* orow = out + (size_t)(pair / topk) * H;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int n = job.n0 + hh * 128 + 32 * j;
+      if (n >= H) break;
+#pragma unroll
+      for (int c = 0; c < 32; c += 4) {
+        float4 v;
+        v.x = __fmul_rn(__fmul_rn(__uint_as_float(acc[j][c + 0]), alpha), w);
+        v.y = __fmul_rn(__fmul_rn(__uint_as_float(acc[j][c + 1]), alpha), w);
+        v.z = __fmul_rn(__fmul_rn(__uint_as_float(acc[j][c + 2]), alpha), w);
+        v.w = __fmul_rn(__fmul_rn(__uint_as_float(acc[j][c + 3]), alpha), w);
+        atomicAdd(reinterpret_cast<float4*>(orow + n + c), v);
+      }
+    }
+  }
+};
+
+template <class Prob>
+static cudaError_t prepare_moe_kernel() {
+  static std::once_flag once;
+  static cudaError_t err = cudaSuccess;
+  std::call_once(once, [] {
+    err = cudaFuncSetAttribute(nvf4_gemm_kernel<Prob>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               (int)kGemmSmemBytes);
+  });
+  return err;
+}
+
+constexpr uint64_t kMoeTimeoutNs = 2000000000ull;
+
+cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t s) {
+  const MoeLayout L = moe_layout(a.T, a.H, a.I, a.E, a.topk);
+  uint8_t* ws = a.ws;
+  auto I32 = [ws](int64_t off) { return reinterpret_cast<int32_t*>(ws + off); };
+  auto U32 = [ws](int64_t off) { return reinterpret_cast<uint32_t*>(ws + off); };
+  auto F32 = [ws](int64_t off) { return reinterpret_cast<float*>(ws + off); };
+  const int64_t P = L.P, R = L.R;
+  cudaError_t e;
+
+  // 1. route
+  const size_t route_smem = (size_t)(kRouteWarps * a.E + a.E + 1) * sizeof(int32_t);
+  static std::once_flag once;
+  static cudaError_t attr_err = cudaSuccess;
+  std::call_once(once, [] {
+    attr_err = cudaFuncSetAttribute(moe_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  });
+  if (attr_err != cudaSuccess) return attr_err;
+  moe_route_kernel<<<1, kRouteThreads, route_smem, s>>>(a.topk_ids, P, a.E, R, I32(L.counts), I32(L.offsets),
+                                                         I32(L.row_pair), I32(L.tile_expert), I32(L.tile_count),
+                                                         U32(L.amax_x), U32(L.amax_h), status);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  // 2. token pass
+  {
+    int64_t blocks = (a.T + 7) / 8;
+    if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
+    if (blocks < 1) blocks = 1;
+    moe_token_pass_kernel<<<(int)blocks, 256, 0, s>>>(static_cast<const uint4*>(a.x), a.T, a.H, a.topk_ids,
+                                                       a.topk, a.E, U32(L.amax_x), reinterpret_cast<float4*>(a.out));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+
+  const int qgrid = num_sms * 8;
+  // 3. gather + quantize x per expert
+  moe_quantize_rows_kernel<true><<<qgrid, 256, 0, s>>>(
+      static_cast<const uint4*>(a.x), a.H, a.topk, I32(L.row_pair), I32(L.tile_expert), I32(L.tile_count),
+      U32(L.amax_x), a.E, U32(L.xq_codes), ws + L.xq_scales, F32(L.xq_g), status);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  // 4. gate_up grouped GEMM
+  {
+    CUtensorMap tmA, tmB;
+    if (encode_tensor_map_2d(&tmA, ws + L.xq_codes, a.H / 2, R, a.H / 2, kBK / 2, kBM) != CUDA_SUCCESS ||
+        encode_tensor_map_2d(&tmB, a.w13_q, a.H / 2, (uint64_t)a.E * 2 * a.I, a.H / 2, kBK / 2, 128) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    GateUpProblem p;
+    p.K = (int)a.H;
+    p.I = (int)a.I;
+    p.n_tiles = (int)(a.I / 128);
+    p.kgroups = (int)(a.H / 64);
+    p.sf_expert_bytes = scale_bytes_(2 * a.I, a.H);
+    p.tile_count = I32(L.tile_count);
+    p.tile_expert = I32(L.tile_expert);
+    p.sfa = ws + L.xq_scales;
+    p.sfb = a.w13_s;
+    p.ga = F32(L.xq_g);
+    p.gb = a.w13_g;
+    p.h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
+    p.amax_h = U32(L.amax_h);
+    if ((e = prepare_moe_kernel<GateUpProblem>()) != cudaSuccess) return e;
+    int64_t max_tiles = (R / 128) * p.n_tiles;
+    const int grid = (int)(max_tiles < num_sms ? max_tiles : num_sms);
+    nvf4_gemm_kernel<GateUpProblem><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB, p, status, kMoeTimeoutNs);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+
+  // 5. quantize h per expert
+  moe_quantize_rows_kernel<false><<<qgrid, 256, 0, s>>>(
+      reinterpret_cast<const uint4*>(ws + L.h), a.I, a.topk, I32(L.row_pair), I32(L.tile_expert),
+      I32(L.tile_count), U32(L.amax_h), a.E, U32(L.hq_codes), ws + L.hq_scales, F32(L.hq_g), status);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+
+  // 6. down grouped GEMM + weighted FP32 combine
+  {
+    CUtensorMap tmA, tmB;
+    if (encode_tensor_map_2d(&tmA, ws + L.hq_codes, a.I / 2, R, a.I / 2, kBK / 2, kBM) != CUDA_SUCCESS ||
+        encode_tensor_map_2d(&tmB, a.w2_q, a.I / 2, (uint64_t)a.E * a.H, a.I / 2, kBK / 2, 128) != CUDA_SUCCESS)
+      return cudaErrorInvalidValue;
+    DownProblem p;
+    p.K = (int)a.I;
+    p.H = (int)a.H;
+    p.n_tiles = (int)((a.H + 255) / 256);
+    p.kgroups = (int)(a.I / 64);
+    p.topk = a.topk;
+    p.sf_expert_bytes = scale_bytes_(a.H, a.I);
+    p.tile_count = I32(L.tile_count);
+    p.tile_expert = I32(L.tile_expert);
+    p.row_pair = I32(L.row_pair);
+    p.topk_w = a.topk_w;
+    p.sfa = ws + L.hq_scales;
+    p.sfb = a.w2_s;
+    p.ga = F32(L.hq_g);
+    p.gb = a.w2_g;
+    p.out = a.out;
+    if ((e = prepare_moe_kernel<DownProblem>()) != cudaSuccess) return e;
+    int64_t max_tiles = (R / 128) * p.n_tiles;
+    const int grid = (int)(max_tiles < num_sms ? max_tiles : num_sms);
+    nvf4_gemm_kernel<DownProblem><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB, p, status, kMoeTimeoutNs);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace nvfp4
+
+// ----------------------------------------------------------------------------
+// C ABI of the MoE layer.
+// ----------------------------------------------------------------------------
+extern "C" {
+
+size_t nvfp4_moe_workspace_bytes(int64_t T, int64_t H, int64_t I, int E, int topk) {
+  if (T < 0 || H <= 0 || I <= 0 || E <= 0 || topk <= 0) return 0;
+  return (size_t)nvfp4::moe_layout(T, H, I, E, topk).total;
+}
+
+nvfp4_status nvfp4_moe_grouped_gemm(const void* x, int64_t T, int64_t H, const int32_t* topk_ids,
+                                    const float* topk_w, int topk, int E, int64_t I, const uint8_t* w13_q,
+                                    const uint8_t* w13_s, const float* w13_g, const uint8_t* w2_q,
+                                    const uint8_t* w2_s, const float* w2_g, float* out, void* workspace,
+                                    size_t workspace_bytes, nvfp4_stream_t stream) {
+  if (T < 0 || H <= 0 || I <= 0 || H % 256 || I % 128 || topk < 1 || E < 1 || E > 1024 || topk > E ||
+      T * topk >= (1ll << 31) || (int64_t)E * 2 * I >= (1ll << 31) || (int64_t)E * H >= (1ll << 31))
+    return NVFP4_ERR_INVALID_ARG;
+  auto al = [](const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; };
+  if (!w13_q || !w13_s || !w13_g || !w2_q || !w2_s || !w2_g || !al(w13_q) || !al(w13_s) || !al(w2_q) || !al(w2_s))
+    return NVFP4_ERR_INVALID_ARG;
+  if (T > 0 && (!x || !topk_ids || !topk_w || !out || !al(x) || !al(out))) return NVFP4_ERR_INVALID_ARG;
+  if (!workspace || !al(workspace) || workspace_bytes < nvfp4_moe_workspace_bytes(T, H, I, E, topk))
+    return NVFP4_ERR_WORKSPACE;
+  int num_sms = 0;
+  int* status = nullptr;
+  const int st = nvfp4::current_device_context(&num_sms, &status);
+  if (st != NVFP4_OK) return (nvfp4_status)st;
+  if (T == 0) return NVFP4_OK;
+  nvfp4::MoeArgs a;
+  a.x = x;
+  a.T = T;
+  a.H = H;
+  a.I = I;
+  a.topk_ids = topk_ids;
+  a.topk_w = topk_w;
+  a.topk = topk;
+  a.E = E;
+  a.w13_q = w13_q;
+  a.w13_s = w13_s;
+  a.w13_g = w13_g;
+  a.w2_q = w2_q;
+  a.w2_s = w2_s;
+  a.w2_g = w2_g;
+  a.out = out;
+  a.ws = static_cast<uint8_t*>(workspace);
+  return nvfp4::launch_moe(a, status, num_sms, reinterpret_cast<cudaStream_t>(stream)) == cudaSuccess
+             ? NVFP4_OK
+             : NVFP4_ERR_CUDA;
+}
+
+nvfp4_status nvfp4_moe_workspace_layout(int64_t T, int64_t H, int64_t I, int E, int topk,
+                                        nvfp4_moe_layout* out) {
+  if (!out || T < 0 || H <= 0 || I <= 0 || E <= 0 || topk <= 0) return NVFP4_ERR_INVALID_ARG;
+  const nvfp4::MoeLayout L = nvfp4::moe_layout(T, H, I, E, topk);
+  out->rows_capacity = L.R;
+  out->counts = L.counts;
+  out->offsets = L.offsets;
+  out->row_pair = L.row_pair;
+  out->xq_codes = L.xq_codes;
+  out->xq_scales = L.xq_scales;
+  out->xq_g = L.xq_g;
+  out->h = L.h;
+  out->hq_codes = L.hq_codes;
+  out->hq_scales = L.hq_scales;
+  out->hq_g = L.hq_g;
+  out->total_bytes = L.total;
+  return NVFP4_OK;
+}
+
+}  // extern "C"
