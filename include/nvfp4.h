@@ -62,7 +62,8 @@ typedef enum {
   NVFP4_ERR_CUDA = 3,               /* a CUDA runtime call failed */
   NVFP4_ERR_WORKSPACE = 4,          /* workspace missing or too small */
   NVFP4_ERR_NONFINITE_INPUT = 5,    /* device: amax of an input is Inf/NaN */
-  NVFP4_ERR_TIMEOUT = 6             /* device: a bounded wait ran out */
+  NVFP4_ERR_TIMEOUT = 6,            /* device: a bounded wait ran out */
+  NVFP4_ERR_TOO_LARGE = 7           /* input larger than nvfp4_quantize_noalloc's static scratch */
 } nvfp4_status;
 
 typedef enum {
@@ -209,6 +210,27 @@ typedef struct {
 
 nvfp4_status nvfp4_moe_workspace_layout(int64_t T, int64_t H, int64_t I, int E, int topk,
                                         nvfp4_moe_layout* layout /* host */);
+
+/*
+ * nvfp4_quantize_noalloc -- nvfp4_quantize without a workspace argument, for
+ *   callers that cannot allocate device memory: an inference plugin whose
+ *   enqueue step receives only its input and output pointers, or code that
+ *   runs where the device allocator is unavailable or forbidden. (The pages
+ *   have no counterpart; this is a deployment convenience.) Same arguments,
+ *   outputs and device status as nvfp4_quantize.
+ * Scratch: the dynamic global scale is reduced through a library-owned static
+ *   device array of 4096 32-bit slots (16 KiB, held on every GPU that loads
+ *   the library until exit), one slot per 2^18 input elements: M*K may be at
+ *   most 2^30, larger inputs return NVFP4_ERR_TOO_LARGE before any launch.
+ * The call allocates nothing. The first call on a device looks up the array's
+ *   device address (make it before any stream capture on that device). All
+ *   calls on a device share the array: calls whose kernels overlap on the GPU
+ *   race and must be ordered (same stream). Nothing in the array needs to be
+ *   cleared between calls.
+ */
+nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t M, int64_t K, nvfp4_mode mode,
+                                    const float* g_in, uint8_t* codes, uint8_t* scales,
+                                    float* g_out, uint8_t* fos_choice, nvfp4_stream_t stream);
 
 /* Conversion primitives (diagnostics; the quantize kernels use the same
  * device code). e2m1: code of each FP32 value, one per byte, RNE, saturate

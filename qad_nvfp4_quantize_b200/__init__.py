@@ -19,7 +19,7 @@ __all__ = [
     "MODE_MAX", "MODE_FOUR_OVER_SIX", "NVFP4Error", "Quantized", "lib", "library_path",
     "check_device", "scale_bytes", "quantize", "fake_quant", "gemm", "moe_grouped_gemm",
     "moe_workspace_layout", "convert_e2m1", "convert_e4m3", "device_status", "selftest_timeout",
-    "quantize_workspace_bytes", "moe_workspace_bytes", "quantize_experts",
+    "quantize_workspace_bytes", "moe_workspace_bytes", "quantize_experts", "quantize_noalloc",
 ]
 
 MODE_MAX = 0
@@ -31,7 +31,8 @@ _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libnvfp4.so")
 
 _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported device", 3: "CUDA error",
-           4: "workspace missing or too small", 5: "non-finite input", 6: "device wait timed out"}
+           4: "workspace missing or too small", 5: "non-finite input", 6: "device wait timed out",
+           7: "input too large for the no-alloc entry point (M*K > 2^30)"}
 
 
 class NVFP4Error(RuntimeError):
@@ -58,6 +59,7 @@ _SIGS = {
     "nvfp4_quantize_workspace_bytes": (SZ, [I64, I64]),
     "nvfp4_quantize": (I32, [P, I64, I64, I32, P, P, P, P, P, P, SZ, P]),
     "nvfp4_fake_quant": (I32, [P, I64, I64, I32, P, P, P, P, SZ, P]),
+    "nvfp4_quantize_noalloc": (I32, [P, I64, I64, I32, P, P, P, P, P, P]),
     "nvfp4_gemm": (I32, [P, P, P, P, P, P, I64, I64, I64, P, P]),
     "nvfp4_moe_workspace_bytes": (SZ, [I64, I64, I64, I32, I32]),
     "nvfp4_moe_grouped_gemm": (I32, [P, I64, I64, P, P, I32, I32, I64, P, P, P, P, P, P, P, P, SZ, P]),
@@ -177,6 +179,26 @@ def quantize(x: torch.Tensor, mode="max", g: Optional[torch.Tensor] = None, want
     st = lib().nvfp4_quantize(_ptr(x), M, K, _MODES[mode], _ptr(g), _ptr(out.codes), _ptr(out.scales),
                               _ptr(out.g), _ptr(out.choice), _ptr(ws), ws_bytes, _stream(dev))
     _check(st, "nvfp4_quantize")
+    return out
+
+
+def quantize_noalloc(x: torch.Tensor, mode="max", g: Optional[torch.Tensor] = None,
+                     want_choice: bool = False, out: Optional[Quantized] = None) -> Quantized:
+    """nvfp4_quantize_noalloc: like quantize(), but the library reduces the
+    global scale through its own static device scratch instead of a caller
+    workspace (for callers that cannot allocate; M*K <= 2^30). Pass ``out`` to
+    make the call itself allocation-free."""
+    x = _cuda(x, "x", torch.bfloat16)
+    M, K = x.shape
+    dev = x.device
+    if out is None:
+        out = Quantized(torch.empty((M, K // 2), dtype=torch.uint8, device=dev),
+                        torch.empty(max(scale_bytes(M, K), 16), dtype=torch.uint8, device=dev),
+                        torch.empty(1, dtype=torch.float32, device=dev),
+                        torch.empty((M, K // 16), dtype=torch.uint8, device=dev) if want_choice else None, M, K)
+    st = lib().nvfp4_quantize_noalloc(_ptr(x), M, K, _MODES[mode], _ptr(g), _ptr(out.codes), _ptr(out.scales),
+                                      _ptr(out.g), _ptr(out.choice), _stream(dev))
+    _check(st, "nvfp4_quantize_noalloc")
     return out
 
 

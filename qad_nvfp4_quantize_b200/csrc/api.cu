@@ -94,6 +94,7 @@ const char* nvfp4_status_string(nvfp4_status s) {
     case NVFP4_ERR_WORKSPACE: return "workspace missing or too small";
     case NVFP4_ERR_NONFINITE_INPUT: return "non-finite input";
     case NVFP4_ERR_TIMEOUT: return "device wait timed out";
+    case NVFP4_ERR_TOO_LARGE: return "input larger than the no-alloc entry point's static scratch (M*K > 2^30)";
   }
   return "unknown status";
 }
