@@ -53,10 +53,18 @@ def load_peaks():
     return dict(hbm=FALLBACK_HBM_GBS, bf16=FALLBACK_BF16_TFLOPS, bf16_sustained=1400.0, source="fallback")
 
 
-def kernel_sources_digest():
+KERNEL_SOURCES = {
+    "gemm_dense_mlp": ["common.cuh", "gemm_kernel.cuh", "gemm.cu"],
+    "quantize_dense_mlp": ["common.cuh", "quantize.cu"],
+}
+
+
+def kernel_sources_digest(kernel_key: str):
+    """Digest of the sources a kernel is built from (its traffic figure is
+    stale once any of them changes)."""
     h = hashlib.sha256()
-    for p in sorted(glob.glob(os.path.join(ROOT, "qad_nvfp4_quantize_b200", "csrc", "*"))):
-        with open(p, "rb") as f:
+    for name in KERNEL_SOURCES[kernel_key]:
+        with open(os.path.join(ROOT, "qad_nvfp4_quantize_b200", "csrc", name), "rb") as f:
             h.update(f.read())
     return h.hexdigest()[:16]
 
@@ -64,7 +72,7 @@ def kernel_sources_digest():
 def recorded_traffic(kernel_key: str):
     """DRAM bytes per launch recorded from an ncu capture under profiles/, valid
     only while the kernel sources are unchanged since the capture."""
-    digest = kernel_sources_digest()
+    digest = kernel_sources_digest(kernel_key)
     for path in glob.glob(os.path.join(ROOT, "profiles", "*.md")):
         with open(path) as f:
             for line in f:

@@ -286,4 +286,75 @@ NVFP4_DEVINL uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo
   return d;
 }
 
+// ----------------------------------------------------------------------------
+// Warp-converged issue. The producer and MMA roles run their loops on all 32
+// lanes (so loop state and descriptors stay warp-uniform) and each issuing
+// instruction is predicated on elect.sync, which picks the same single lane
+// every time for a full mask.
+// ----------------------------------------------------------------------------
+#define NVFP4_ELECT_BEGIN "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
+#define NVFP4_ELECT_END "\n\t}"
+
+NVFP4_DEVINL void mbar_arrive_expect_tx_elect(uint64_t* bar, uint32_t bytes) {
+  asm volatile(NVFP4_ELECT_BEGIN "@e mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" NVFP4_ELECT_END
+               ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+
+NVFP4_DEVINL void tma_load_2d_elect(void* smem_dst, const CUtensorMap* map, int32_t x, int32_t y, uint64_t* bar) {
+  asm volatile(NVFP4_ELECT_BEGIN
+               "@e cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+               " [%0], [%1, {%2, %3}], [%4];" NVFP4_ELECT_END
+               ::"r"(smem_u32(smem_dst)), "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+               : "memory");
+}
+
+NVFP4_DEVINL void bulk_load_elect(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(NVFP4_ELECT_BEGIN
+               "@e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
+               NVFP4_ELECT_END
+               ::"r"(smem_u32(smem_dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
+}
+
+NVFP4_DEVINL void tc_copy_scales_elect(uint32_t taddr, uint64_t sdesc) {
+  asm volatile(NVFP4_ELECT_BEGIN "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" NVFP4_ELECT_END
+               ::"r"(taddr), "l"(sdesc) : "memory");
+}
+
+NVFP4_DEVINL void tc_mma_nvf4_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                    uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
+  asm volatile(NVFP4_ELECT_BEGIN ".reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+               "@e tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;"
+               NVFP4_ELECT_END
+               ::"r"(d_tmem), "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
+               : "memory");
+}
+
+NVFP4_DEVINL void tc_commit_elect(uint64_t* bar) {
+  asm volatile(NVFP4_ELECT_BEGIN
+               "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" NVFP4_ELECT_END
+               ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Warp-converged bounded wait: every lane observes the phase; the timeout
+// decision is lane 0's, broadcast, so the warp leaves the loop together.
+NVFP4_DEVINL bool mbar_wait_warp(uint64_t* bar, uint32_t parity, volatile int* abort, uint64_t limit_ns) {
+  uint64_t t0 = 0;
+  uint32_t spins = 0;
+  const int lane = threadIdx.x & 31;
+  while (true) {
+    const bool done = mbar_try_wait(bar, parity);
+    if (__all_sync(0xFFFFFFFFu, done)) return true;
+    if (((++spins) & 63u) == 0) {
+      int stop = 0;
+      if (lane == 0) {
+        const uint64_t now = globaltimer_ns();
+        if (t0 == 0) t0 = now;
+        stop = (*abort != 0) || (now - t0 > limit_ns);
+        if (stop) *abort = 1;
+      }
+      if (__shfl_sync(0xFFFFFFFFu, stop, 0)) return false;
+    }
+  }
+}
+
 }  // namespace nvfp4

@@ -15,8 +15,10 @@
 //   warps 2..9  epilogue: drain the 128 x 256 FP32 accumulator from tensor
 //               memory into registers, release it to the MMA warp, then scale,
 //               round and store (policy-specific).
-// Tensor memory: columns [0,256) accumulator, [256,272) A scales of one
-// stage (4 columns per MMA), [272,304) B scales (8 columns per MMA).
+// Tensor memory: columns [0,256) accumulator; from column 256 each pipeline
+// stage owns 48 columns of scales -- 16 for A (4 per MMA) then 32 for B (8 per
+// MMA) -- so the scale copy of one stage never overwrites columns that MMAs of
+// the previous stages may still read.
 // Every mbarrier wait is bounded; on expiry the CTA records
 // NVFP4_ERR_TIMEOUT, drains its in-flight copies and MMAs (bounded) and
 // returns with its tensor memory freed.
@@ -38,8 +40,10 @@ constexpr uint32_t kSFABytes = 4 * kSFAtom;
 constexpr uint32_t kSFBBytes = 8 * kSFAtom;
 constexpr int kGemmThreads = 320;
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kTmemSFA = 256;
-constexpr uint32_t kTmemSFB = 272;
+constexpr uint32_t kTmemSF = 256;         // first scale column
+constexpr uint32_t kTmemSFStage = 48;     // scale columns per stage
+constexpr uint32_t kTmemSFBOff = 16;      // B scales after A scales inside a stage
+static_assert(kTmemSF + kStages * kTmemSFStage <= kTmemCols, "tensor memory budget");
 
 constexpr uint32_t kSmemA = 0;
 constexpr uint32_t kSmemB = kSmemA + kStages * kABytes;
@@ -115,100 +119,111 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (lane == 0) {
-      uint32_t stage = 0, phase = 0;
-      int armed_phase[kStages];
-#pragma unroll
-      for (int s = 0; s < kStages; ++s) armed_phase[s] = -1;
-      bool ok = true;
-      for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
-        const TileJob job = prob.job(t);
-        for (int kt = 0; kt < nkt; ++kt) {
-          if (!mbar_wait_bounded(&empty[stage], phase ^ 1, abort_flag, timeout_ns)) {
-            ok = false;
-            break;
-          }
-          const int nkb = min(4, kgroups - 4 * kt);
-          const uint32_t sf_bytes = (uint32_t)nkb * kSFAtom;
-          const uint32_t tx = kABytes + kBBytes + sf_bytes * (job.sfb1 ? 3u : 2u);
-          mbar_arrive_expect_tx(&full[stage], tx);
-          armed_phase[stage] = (int)phase;
-          uint8_t* sA = smem + kSmemA + stage * kABytes;
-          uint8_t* sB = smem + kSmemB + stage * kBBytes;
-          tma_load_2d(sA, &tmA, kt * (kBK / 2), job.a_row, &full[stage]);
-          tma_load_2d(sB, &tmB, kt * (kBK / 2), job.b_row0, &full[stage]);
-          tma_load_2d(sB + kBHalfBytes, &tmB, kt * (kBK / 2), job.b_row1, &full[stage]);
-          bulk_load(smem + kSmemSFA + stage * kSFABytes, job.sfa + (size_t)kt * kSFABytes, sf_bytes,
-                    &full[stage]);
-          uint8_t* sSFB = smem + kSmemSFB + stage * kSFBBytes;
-          bulk_load(sSFB, job.sfb0 + (size_t)kt * kSFABytes, sf_bytes, &full[stage]);
-          if (job.sfb1) bulk_load(sSFB + kSFABytes, job.sfb1 + (size_t)kt * kSFABytes, sf_bytes, &full[stage]);
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1;
-          }
+    // The whole warp runs the loop (warp-uniform state); elect.sync issues.
+    uint32_t stage = 0, phase = 0;
+    uint32_t armed = 0;  // bit s: stage s armed; bit 8+s: its phase
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
+      const TileJob job = prob.job(t);
+      for (int kt = 0; kt < nkt; ++kt) {
+        if (!mbar_wait_warp(&empty[stage], phase ^ 1, abort_flag, timeout_ns)) {
+          ok = false;
+          break;
+        }
+        const int nkb = min(4, kgroups - 4 * kt);
+        const uint32_t sf_bytes = (uint32_t)nkb * kSFAtom;
+        const uint32_t tx = kABytes + kBBytes + sf_bytes * (job.sfb1 ? 3u : 2u);
+        mbar_arrive_expect_tx_elect(&full[stage], tx);
+        armed = (armed & ~(0x101u << stage)) | (1u << stage) | (phase << (8 + stage));
+        uint8_t* sA = smem + kSmemA + stage * kABytes;
+        uint8_t* sB = smem + kSmemB + stage * kBBytes;
+        tma_load_2d_elect(sA, &tmA, kt * (kBK / 2), job.a_row, &full[stage]);
+        tma_load_2d_elect(sB, &tmB, kt * (kBK / 2), job.b_row0, &full[stage]);
+        tma_load_2d_elect(sB + kBHalfBytes, &tmB, kt * (kBK / 2), job.b_row1, &full[stage]);
+        bulk_load_elect(smem + kSmemSFA + stage * kSFABytes, job.sfa + (size_t)kt * kSFABytes, sf_bytes,
+                        &full[stage]);
+        uint8_t* sSFB = smem + kSmemSFB + stage * kSFBBytes;
+        bulk_load_elect(sSFB, job.sfb0 + (size_t)kt * kSFABytes, sf_bytes, &full[stage]);
+        if (job.sfb1) bulk_load_elect(sSFB + kSFABytes, job.sfb1 + (size_t)kt * kSFABytes, sf_bytes, &full[stage]);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1;
         }
       }
-      if (!ok) {
-        // let copies already in flight land before the CTA exits
-        record_status(status, NVFP4_ERR_TIMEOUT);
-        for (int s = 0; s < kStages; ++s) {
-          if (armed_phase[s] < 0) continue;
-          const uint64_t t0 = globaltimer_ns();
-          while (!mbar_try_wait(&full[s], (uint32_t)armed_phase[s]) &&
-                 globaltimer_ns() - t0 < 1000000ull) {
-          }
+    }
+    if (!ok && lane == 0) {
+      // let copies already in flight land before the CTA exits
+      record_status(status, NVFP4_ERR_TIMEOUT);
+      for (int s = 0; s < kStages; ++s) {
+        if (!((armed >> s) & 1u)) continue;
+        const uint32_t ph = (armed >> (8 + s)) & 1u;
+        const uint64_t t0 = globaltimer_ns();
+        while (!mbar_try_wait(&full[s], ph) && globaltimer_ns() - t0 < 1000000ull) {
         }
       }
     }
     __syncwarp();
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = make_idesc_nvf4(kBM, kBN);
-      uint32_t stage = 0, phase = 0, acc_phase = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
-        if (!mbar_wait_bounded(acc_empty, acc_phase ^ 1, abort_flag, timeout_ns)) {
+    // Warp-converged loop; scale copies, MMAs and commits issued by one
+    // elected lane (the same lane each time, so they stay in issue order).
+    constexpr uint32_t idesc = make_idesc_nvf4(kBM, kBN);
+    uint32_t stage = 0, phase = 0, acc_phase = 0;
+    bool ok = true;
+    for (int t = blockIdx.x; ok && t < ntiles; t += gridDim.x) {
+      if (!mbar_wait_warp(acc_empty, acc_phase ^ 1, abort_flag, timeout_ns)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      for (int kt = 0; kt < nkt; ++kt) {
+        if (!mbar_wait_warp(&full[stage], phase, abort_flag, timeout_ns)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        for (int kt = 0; kt < nkt; ++kt) {
-          if (!mbar_wait_bounded(&full[stage], phase, abort_flag, timeout_ns)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const int nkb = min(4, kgroups - 4 * kt);
-          const uint32_t sA = smem_u32(smem + kSmemA + stage * kABytes);
-          const uint32_t sB = smem_u32(smem + kSmemB + stage * kBBytes);
-          const uint32_t sSFA = smem_u32(smem + kSmemSFA + stage * kSFABytes);
-          const uint32_t sSFB = smem_u32(smem + kSmemSFB + stage * kSFBBytes);
-          const uint64_t adesc = smem_desc(sA, 16, 1024, 2);
-          const uint64_t bdesc = smem_desc(sB, 16, 1024, 2);
-          for (int kb = 0; kb < nkb; ++kb) {
-            tc_copy_scales(tmem + kTmemSFA + 4 * kb, smem_desc(sSFA + kb * kSFAtom, 0, 128, 0));
-            tc_copy_scales(tmem + kTmemSFB + 8 * kb, smem_desc(sSFB + kb * kSFAtom, 0, 128, 0));
-            tc_copy_scales(tmem + kTmemSFB + 8 * kb + 4,
-                           smem_desc(sSFB + kSFABytes + kb * kSFAtom, 0, 128, 0));
+        const int nkb = min(4, kgroups - 4 * kt);
+        const uint32_t sA = smem_u32(smem + kSmemA + stage * kABytes);
+        const uint32_t sB = smem_u32(smem + kSmemB + stage * kBBytes);
+        const uint32_t sSFA = smem_u32(smem + kSmemSFA + stage * kSFABytes);
+        const uint32_t sSFB = smem_u32(smem + kSmemSFB + stage * kSFBBytes);
+        const uint64_t adesc = smem_desc(sA, 16, 1024, 2);
+        const uint64_t bdesc = smem_desc(sB, 16, 1024, 2);
+        const uint32_t tsfa = tmem + kTmemSF + stage * kTmemSFStage;
+        const uint32_t tsfb = tsfa + kTmemSFBOff;
+        if (nkb == 4) {
+#pragma unroll
+          for (int kb = 0; kb < 4; ++kb) {
+            tc_copy_scales_elect(tsfa + 4 * kb, smem_desc(sSFA + kb * kSFAtom, 0, 128, 0));
+            tc_copy_scales_elect(tsfb + 8 * kb, smem_desc(sSFB + kb * kSFAtom, 0, 128, 0));
+            tc_copy_scales_elect(tsfb + 8 * kb + 4, smem_desc(sSFB + kSFABytes + kb * kSFAtom, 0, 128, 0));
             // K advance inside the 128-byte swizzle atom: 32 bytes per MMA
-            tc_mma_nvf4(tmem, adesc + (uint64_t)(2 * kb), bdesc + (uint64_t)(2 * kb), idesc,
-                        tmem + kTmemSFA + 4 * kb, tmem + kTmemSFB + 8 * kb, (kt | kb) != 0);
+            tc_mma_nvf4_elect(tmem, adesc + (uint64_t)(2 * kb), bdesc + (uint64_t)(2 * kb), idesc, tsfa + 4 * kb,
+                              tsfb + 8 * kb, (kt | kb) != 0);
           }
-          tc_commit(&empty[stage]);
-          if (++stage == kStages) {
-            stage = 0;
-            phase ^= 1;
+        } else {
+          for (int kb = 0; kb < nkb; ++kb) {
+            tc_copy_scales_elect(tsfa + 4 * kb, smem_desc(sSFA + kb * kSFAtom, 0, 128, 0));
+            tc_copy_scales_elect(tsfb + 8 * kb, smem_desc(sSFB + kb * kSFAtom, 0, 128, 0));
+            tc_copy_scales_elect(tsfb + 8 * kb + 4, smem_desc(sSFB + kSFABytes + kb * kSFAtom, 0, 128, 0));
+            tc_mma_nvf4_elect(tmem, adesc + (uint64_t)(2 * kb), bdesc + (uint64_t)(2 * kb), idesc, tsfa + 4 * kb,
+                              tsfb + 8 * kb, (kt | kb) != 0);
           }
         }
-        if (!ok) break;
-        tc_commit(acc_full);
-        acc_phase ^= 1;
+        tc_commit_elect(&empty[stage]);
+        if (++stage == kStages) {
+          stage = 0;
+          phase ^= 1;
+        }
       }
-      if (!ok) {
+      if (!ok) break;
+      tc_commit_elect(acc_full);
+      acc_phase ^= 1;
+    }
+    if (!ok) {
+      tc_commit_elect(drain);  // wait (bounded) for MMAs already issued
+      if (lane == 0) {
         record_status(status, NVFP4_ERR_TIMEOUT);
-        tc_commit(drain);  // wait (bounded) for MMAs already issued
         const uint64_t t0 = globaltimer_ns();
         while (!mbar_try_wait(drain, 0) && globaltimer_ns() - t0 < 1000000ull) {
         }
@@ -221,7 +236,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     const int h = (warp - 2) >> 2;   // which half of the tile's columns
     uint32_t acc_phase = 0;
     for (int t = blockIdx.x; t < ntiles; t += gridDim.x) {
-      if (!mbar_wait_bounded(acc_full, acc_phase, abort_flag, timeout_ns)) {
+      if (!mbar_wait_warp(acc_full, acc_phase, abort_flag, timeout_ns)) {
         if (lane == 0) record_status(status, NVFP4_ERR_TIMEOUT);
         break;
       }

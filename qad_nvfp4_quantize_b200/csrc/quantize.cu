@@ -23,6 +23,7 @@ namespace nvfp4 {
 constexpr int kQThreads = 256;  // 8 warps
 constexpr int kAmaxThreads = 256;
 constexpr unsigned kFull = 0xFFFFFFFFu;
+constexpr int kUnroll = 4;  // chunks of 256 elements in flight per warp
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   uint4 v;
@@ -90,7 +91,16 @@ __device__ __forceinline__ float resolve_global_scale(const uint32_t* partial, i
       g = *g_static;
     } else {
       uint32_t m = 0;
-      for (int i = threadIdx.x; i < n_partial; i += 32) m = max(m, partial[i]);
+      for (int base = 0; base < n_partial; base += 8 * 32) {  // 8 independent loads per lane
+        uint32_t v[8];
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int i = base + u * 32 + (int)threadIdx.x;
+          v[u] = i < n_partial ? partial[i] : 0u;
+        }
+#pragma unroll
+        for (int u = 0; u < 8; ++u) m = max(m, v[u]);
+      }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFull, m, o));
       bad = m >= 0x7F80u;
@@ -215,33 +225,42 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(
   const int64_t warp = (int64_t)blockIdx.x * (kQThreads / 32) + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * (kQThreads / 32);
 
-  for (int64_t ch = warp; ch < n_chunks; ch += nwarps) {
-    const int64_t e0 = (ch << 8) + lane * 8;
-    const bool valid = e0 < n;
-    float v[8];
-    load8(x, e0 >> 3, valid, v);
-    const float bmax = block_max(v);
-    HalfBlock h6;
-    quantize_half<kFos>(v, bmax, g, 6.0f, lane, h6);
-    uint32_t sc = h6.sc, q = h6.q, pick4 = 0;
-    if (kFos) {
-      HalfBlock h4;
-      quantize_half<true>(v, bmax, g, 4.0f, lane, h4);
-      pick4 = h4.err < h6.err;  // tie keeps M = 6
-      if (pick4) {
-        sc = h4.sc;
-        q = h4.q;
-      }
+  // kUnroll chunks per trip with all loads issued first (memory-level parallelism)
+  for (int64_t ch0 = warp; ch0 < n_chunks; ch0 += kUnroll * nwarps) {
+    float vv[kUnroll][8];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t e0 = ((ch0 + u * nwarps) << 8) + lane * 8;
+      load8(x, e0 >> 3, e0 < n, vv[u]);
     }
-    const uint32_t group = gather_group_scales(sc);
-    if (valid) {
-      codes[e0 >> 3] = q;
-      const int64_t fb = e0 >> 4;  // flat block index
-      if ((lane & 7) == 0) {
-        const int64_t row = fb / nblk_row, c = fb - row * nblk_row;
-        *reinterpret_cast<uint32_t*>(scales + scale_offset(row, c, kgroups)) = group;
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      if (ch0 + u * nwarps >= n_chunks) break;  // warp-uniform
+      const int64_t e0 = ((ch0 + u * nwarps) << 8) + lane * 8;
+      const bool valid = e0 < n;
+      const float bmax = block_max(vv[u]);
+      HalfBlock h6;
+      quantize_half<kFos>(vv[u], bmax, g, 6.0f, lane, h6);
+      uint32_t sc = h6.sc, q = h6.q, pick4 = 0;
+      if (kFos) {
+        HalfBlock h4;
+        quantize_half<true>(vv[u], bmax, g, 4.0f, lane, h4);
+        pick4 = h4.err < h6.err;  // tie keeps M = 6
+        if (pick4) {
+          sc = h4.sc;
+          q = h4.q;
+        }
       }
-      if (kFos && choice && (lane & 1) == 0) choice[fb] = (uint8_t)pick4;
+      const uint32_t group = gather_group_scales(sc);
+      if (valid) {
+        codes[e0 >> 3] = q;
+        const int64_t fb = e0 >> 4;  // flat block index
+        if ((lane & 7) == 0) {
+          const int64_t row = fb / nblk_row, c = fb - row * nblk_row;
+          *reinterpret_cast<uint32_t*>(scales + scale_offset(row, c, kgroups)) = group;
+        }
+        if (kFos && choice && (lane & 1) == 0) choice[fb] = (uint8_t)pick4;
+      }
     }
   }
   if (!kFos && choice) {  // max mode still fills the optional choice map with 0
@@ -273,49 +292,57 @@ __global__ void __launch_bounds__(kQThreads) fake_quant_kernel(
   const int64_t warp = (int64_t)blockIdx.x * (kQThreads / 32) + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * (kQThreads / 32);
 
-  for (int64_t ch = warp; ch < n_chunks; ch += nwarps) {
-    const int64_t e0 = (ch << 8) + lane * 8;
-    const bool valid = e0 < n;
-    float v[8];
-    load8(x, e0 >> 3, valid, v);
-    float out[8];
-    if (kFrozen) {
-      uint32_t sc = 1;
-      if (valid) {
-        const int64_t fb = e0 >> 4;
-        const int64_t row = fb / nblk_row, c = fb - row * nblk_row;
-        sc = scales_frozen[scale_offset(row, c, kgroups)];
-      }
-      const float d = __fmul_rn(g, e4m3_value(sc));
-      const float r = __frcp_rn(d);
-      float sv[8];
+  for (int64_t ch0 = warp; ch0 < n_chunks; ch0 += kUnroll * nwarps) {
+    float vv[kUnroll][8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) sv[i] = __fmul_rn(v[i], r);
-      const uint32_t q = e2m1_pack8(sv);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) out[i] = __fmul_rn(d, e2m1_value((q >> (4 * i)) & 0xFu));
-    } else {
-      const float bmax = block_max(v);
-      HalfBlock h6;
-      quantize_half<kFos>(v, bmax, g, 6.0f, lane, h6);
-      if (kFos) {
-        HalfBlock h4;
-        quantize_half<true>(v, bmax, g, 4.0f, lane, h4);
-        const bool pick4 = h4.err < h6.err;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) out[i] = pick4 ? h4.deq[i] : h6.deq[i];
-      } else {
-#pragma unroll
-        for (int i = 0; i < 8; ++i) out[i] = h6.deq[i];
-      }
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t e0 = ((ch0 + u * nwarps) << 8) + lane * 8;
+      load8(x, e0 >> 3, e0 < n, vv[u]);
     }
-    if (valid) {
-      uint4 w;
-      w.x = f32x2_to_bf16x2(out[0], out[1]);
-      w.y = f32x2_to_bf16x2(out[2], out[3]);
-      w.z = f32x2_to_bf16x2(out[4], out[5]);
-      w.w = f32x2_to_bf16x2(out[6], out[7]);
-      y[e0 >> 3] = w;
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      if (ch0 + u * nwarps >= n_chunks) break;  // warp-uniform
+      const int64_t e0 = ((ch0 + u * nwarps) << 8) + lane * 8;
+      const bool valid = e0 < n;
+      float out[8];
+      if (kFrozen) {
+        uint32_t sc = 1;
+        if (valid) {
+          const int64_t fb = e0 >> 4;
+          const int64_t row = fb / nblk_row, c = fb - row * nblk_row;
+          sc = scales_frozen[scale_offset(row, c, kgroups)];
+        }
+        const float d = __fmul_rn(g, e4m3_value(sc));
+        const float r = __frcp_rn(d);
+        float sv[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) sv[i] = __fmul_rn(vv[u][i], r);
+        const uint32_t q = e2m1_pack8(sv);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) out[i] = __fmul_rn(d, e2m1_value((q >> (4 * i)) & 0xFu));
+      } else {
+        const float bmax = block_max(vv[u]);
+        HalfBlock h6;
+        quantize_half<kFos>(vv[u], bmax, g, 6.0f, lane, h6);
+        if (kFos) {
+          HalfBlock h4;
+          quantize_half<true>(vv[u], bmax, g, 4.0f, lane, h4);
+          const bool pick4 = h4.err < h6.err;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) out[i] = pick4 ? h4.deq[i] : h6.deq[i];
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) out[i] = h6.deq[i];
+        }
+      }
+      if (valid) {
+        uint4 w;
+        w.x = f32x2_to_bf16x2(out[0], out[1]);
+        w.y = f32x2_to_bf16x2(out[2], out[3]);
+        w.z = f32x2_to_bf16x2(out[4], out[5]);
+        w.w = f32x2_to_bf16x2(out[6], out[7]);
+        y[e0 >> 3] = w;
+      }
     }
   }
 }
@@ -371,11 +398,20 @@ cudaError_t launch_amax_partial(const void* x, int64_t n, uint32_t* partial, int
   return cudaGetLastError();
 }
 
+template <class Kern>
+static int resident_blocks(Kern k) {
+  int b = 0;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, k, kQThreads, 0) != cudaSuccess || b < 1) b = 1;
+  return b;
+}
+
 cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, bool fos, const uint32_t* partial,
                             int n_partial, const float* g_static, uint8_t* codes, uint8_t* scales,
                             float* g_out, uint8_t* choice, int* status, int num_sms, cudaStream_t s) {
   const int64_t chunks = (M * K + 255) / 256;
-  const int grid = grid_for(chunks, kQThreads / 32 * 2, num_sms * 8);
+  static const int occ_max = resident_blocks(quantize_kernel<false>);
+  static const int occ_fos = resident_blocks(quantize_kernel<true>);
+  const int grid = grid_for(chunks, kQThreads / 32 * kUnroll, num_sms * (fos ? occ_fos : occ_max));
   if (fos)
     quantize_kernel<true><<<grid, kQThreads, 0, s>>>(static_cast<const uint4*>(x), M, K, partial, n_partial,
                                                       g_static, reinterpret_cast<uint32_t*>(codes), scales,
@@ -391,7 +427,8 @@ cudaError_t launch_fake_quant(const void* x, int64_t M, int64_t K, bool fos, con
                               int n_partial, const float* g_static, const uint8_t* scales_frozen,
                               void* y, int* status, int num_sms, cudaStream_t s) {
   const int64_t chunks = (M * K + 255) / 256;
-  const int grid = grid_for(chunks, kQThreads / 32 * 2, num_sms * 8);
+  static const int occ = resident_blocks(fake_quant_kernel<true, false>);
+  const int grid = grid_for(chunks, kQThreads / 32 * kUnroll, num_sms * occ);
   const uint4* xv = static_cast<const uint4*>(x);
   uint4* yv = static_cast<uint4*>(y);
   if (scales_frozen)
