@@ -23,7 +23,7 @@ namespace nvfp4 {
 constexpr int kQThreads = 256;  // 8 warps
 constexpr int kAmaxThreads = 256;
 constexpr unsigned kFull = 0xFFFFFFFFu;
-constexpr int kUnroll = 4;  // chunks of 256 elements in flight per warp
+constexpr int kUnroll = 2;  // chunks of 512 elements in flight per warp
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   uint4 v;
@@ -38,7 +38,7 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
 // Magnitudes of finite BF16 values order like their bit patterns; anything
 // >= 0x7F80 is Inf or NaN, so the maximum also flags non-finite input.
 // ----------------------------------------------------------------------------
-__global__ void __launch_bounds__(kAmaxThreads) amax_partial_kernel(const uint4* __restrict__ x,
+__global__ void __launch_bounds__(kAmaxThreads, 8) amax_partial_kernel(const uint4* __restrict__ x,
                                                                     int64_t n_vec,
                                                                     uint32_t* __restrict__ partial) {
   uint32_t m2 = 0;  // two 16-bit magnitudes
@@ -123,71 +123,95 @@ __device__ __forceinline__ int64_t scale_offset(int64_t row, int64_t c, int64_t 
          (c & 3);
 }
 
-// Per-lane block math. v: this lane's 8 values (half a block); g: global
-// scale; mt: target magnitude (6 or 4). Produces the scale code, packed
-// codes, dequantized values and the block's squared error (pair-wide, summed
-// in element order: the even lane's 8 terms first, then the odd lane's).
-struct HalfBlock {
-  uint32_t sc;      // E4M3 code of the block scale
-  uint32_t q;       // 8 packed E2M1 codes
-  float deq[8];     // g*s*q per element (FP32)
-  float err;        // block squared error (valid on both lanes of the pair)
+// A warp's unit of work: 512 consecutive elements of one row ("chunk"), one
+// 16-element block per lane. Chunks never straddle rows; a row of K elements
+// has ceil(K/512) chunks and the last one may be partial. The row division is
+// warp-uniform.
+struct Chunk {
+  int64_t row;
+  int32_t col;        // this lane's first element within the row
+  bool valid;         // col < K
+  int64_t vec;        // 16-byte vector index of the block's first 8 elements
 };
 
-template <bool kWantErr>
-__device__ __forceinline__ void quantize_half(const float (&v)[8], float bmax, float g, float mt,
-                                              int lane, HalfBlock& hb) {
-  hb.sc = block_scale_code(bmax, g, mt);
-  const float d = __fmul_rn(g, e4m3_value(hb.sc));
+__device__ __forceinline__ Chunk chunk_at(int64_t ch, int32_t cpr, int64_t K, int lane) {
+  Chunk c;
+  const uint32_t chu = (uint32_t)ch;  // the launcher keeps chunk counts below 2^31
+  const uint32_t r = chu / (uint32_t)cpr;
+  c.row = r;
+  c.col = (int32_t)(chu - r * (uint32_t)cpr) * 512 + lane * 16;
+  c.valid = c.col < K;
+  c.vec = (c.row * K + c.col) >> 3;
+  return c;
+}
+
+__device__ __forceinline__ void load16(const uint4* x, int64_t vec, bool valid, float (&v)[16]) {
+  uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+  if (valid) {
+    a = ld_stream(x + vec);
+    b = ld_stream(x + vec + 1);
+  }
+  bf16x2_to_f32(a.x, v[0], v[1]);
+  bf16x2_to_f32(a.y, v[2], v[3]);
+  bf16x2_to_f32(a.z, v[4], v[5]);
+  bf16x2_to_f32(a.w, v[6], v[7]);
+  bf16x2_to_f32(b.x, v[8], v[9]);
+  bf16x2_to_f32(b.y, v[10], v[11]);
+  bf16x2_to_f32(b.z, v[12], v[13]);
+  bf16x2_to_f32(b.w, v[14], v[15]);
+}
+
+// One 16-element block: scale code, packed codes (two 32-bit words, element 2j
+// in the low nibble of byte j) and, when requested, the dequantized values
+// and the block's squared error summed in element order.
+struct Block {
+  uint32_t sc;
+  uint32_t q0, q1;
+  float deq[16];
+  float err;
+};
+
+template <bool kDeq, bool kErr>
+__device__ __forceinline__ void quantize_block(const float (&v)[16], float bmax, float g, float mt, Block& b) {
+  b.sc = block_scale_code(bmax, g, mt);
+  const float d = __fmul_rn(g, e4m3_value(b.sc));
   const float r = __frcp_rn(d);
-  float sv[8];
+  float sv[16];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) sv[i] = __fmul_rn(v[i], r);
-  hb.q = e2m1_pack8(sv);
+  for (int i = 0; i < 16; ++i) sv[i] = __fmul_rn(v[i], r);
+  b.q0 = e2m1_pack8(sv);
+  b.q1 = e2m1_pack8(sv + 8);
+  if (kDeq || kErr) {
 #pragma unroll
-  for (int i = 0; i < 8; ++i) hb.deq[i] = __fmul_rn(d, e2m1_value((hb.q >> (4 * i)) & 0xFu));
-  if (kWantErr) {
-    float sq[8];
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      const float df = __fsub_rn(v[i], hb.deq[i]);
-      sq[i] = __fmul_rn(df, df);
-    }
+    for (int i = 0; i < 16; ++i)
+      b.deq[i] = __fmul_rn(d, e2m1_value(((i < 8 ? b.q0 : b.q1) >> (4 * (i & 7))) & 0xFu));
+  }
+  if (kErr) {
     float acc = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc = __fadd_rn(acc, sq[i]);
-    const float lo = __shfl_sync(kFull, acc, lane & ~1);  // even partner's partial sum
-    float acc2 = lo;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) acc2 = __fadd_rn(acc2, sq[i]);
-    hb.err = __shfl_sync(kFull, acc2, lane | 1);
+    for (int i = 0; i < 16; ++i) {
+      const float df = __fsub_rn(v[i], b.deq[i]);
+      acc = __fadd_rn(acc, __fmul_rn(df, df));
+    }
+    b.err = acc;
   } else {
-    hb.err = 0.0f;
+    b.err = 0.0f;
   }
 }
 
-__device__ __forceinline__ void load8(const uint4* x, int64_t vec_idx, bool valid, float (&v)[8]) {
-  uint4 w = make_uint4(0, 0, 0, 0);
-  if (valid) w = ld_stream(x + vec_idx);
-  bf16x2_to_f32(w.x, v[0], v[1]);
-  bf16x2_to_f32(w.y, v[2], v[3]);
-  bf16x2_to_f32(w.z, v[4], v[5]);
-  bf16x2_to_f32(w.w, v[6], v[7]);
-}
-
-__device__ __forceinline__ float block_max(const float (&v)[8]) {
+__device__ __forceinline__ float abs_max16(const float (&v)[16]) {
   float m = 0.0f;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
-  return fmaxf(m, __shfl_xor_sync(kFull, m, 1));
+  for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
+  return m;
 }
 
 // Gather the scale codes of the 4 blocks of a 64-element group onto the
-// group's first lane (lanes 8c .. 8c+7 hold blocks 4c .. 4c+3).
+// group's first lane (lanes 4c .. 4c+3 hold blocks 4c .. 4c+3).
 __device__ __forceinline__ uint32_t gather_group_scales(uint32_t sc) {
-  const uint32_t s1 = __shfl_down_sync(kFull, sc, 2);
-  const uint32_t s2 = __shfl_down_sync(kFull, sc, 4);
-  const uint32_t s3 = __shfl_down_sync(kFull, sc, 6);
+  const uint32_t s1 = __shfl_down_sync(kFull, sc, 1);
+  const uint32_t s2 = __shfl_down_sync(kFull, sc, 2);
+  const uint32_t s3 = __shfl_down_sync(kFull, sc, 3);
   return sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
 }
 
@@ -208,7 +232,7 @@ __device__ __forceinline__ void zero_pad_scale_rows(uint8_t* scales, int64_t M, 
 template <bool kFos>
 __global__ void __launch_bounds__(kQThreads) quantize_kernel(
     const uint4* __restrict__ x, int64_t M, int64_t K, const uint32_t* __restrict__ partial,
-    int n_partial, const float* __restrict__ g_static, uint32_t* __restrict__ codes,
+    int n_partial, const float* __restrict__ g_static, uint2* __restrict__ codes,
     uint8_t* __restrict__ scales, float* __restrict__ g_out, uint8_t* __restrict__ choice,
     int* status) {
   bool bad;
@@ -218,53 +242,49 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(
     if (bad) record_status(status, NVFP4_ERR_NONFINITE_INPUT);
   }
   const int64_t kgroups = K >> 6;
-  const int64_t nblk_row = K >> 4;
-  const int64_t n = M * K;
-  const int64_t n_chunks = (n + 255) >> 8;
+  const int32_t cpr = (int32_t)((K + 511) >> 9);
+  const int64_t n_chunks = M * cpr;
   const int lane = threadIdx.x & 31;
   const int64_t warp = (int64_t)blockIdx.x * (kQThreads / 32) + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * (kQThreads / 32);
 
   // kUnroll chunks per trip with all loads issued first (memory-level parallelism)
   for (int64_t ch0 = warp; ch0 < n_chunks; ch0 += kUnroll * nwarps) {
-    float vv[kUnroll][8];
+    float vv[kUnroll][16];
+    Chunk cc[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const int64_t e0 = ((ch0 + u * nwarps) << 8) + lane * 8;
-      load8(x, e0 >> 3, e0 < n, vv[u]);
+      cc[u] = chunk_at(ch0 + u * nwarps, cpr, K, lane);
+      load16(x, cc[u].vec, cc[u].valid && ch0 + u * nwarps < n_chunks, vv[u]);
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       if (ch0 + u * nwarps >= n_chunks) break;  // warp-uniform
-      const int64_t e0 = ((ch0 + u * nwarps) << 8) + lane * 8;
-      const bool valid = e0 < n;
-      const float bmax = block_max(vv[u]);
-      HalfBlock h6;
-      quantize_half<kFos>(vv[u], bmax, g, 6.0f, lane, h6);
-      uint32_t sc = h6.sc, q = h6.q, pick4 = 0;
+      const float bmax = abs_max16(vv[u]);
+      Block b6;
+      quantize_block<false, kFos>(vv[u], bmax, g, 6.0f, b6);
+      uint32_t sc = b6.sc, q0 = b6.q0, q1 = b6.q1, pick4 = 0;
       if (kFos) {
-        HalfBlock h4;
-        quantize_half<true>(vv[u], bmax, g, 4.0f, lane, h4);
-        pick4 = h4.err < h6.err;  // tie keeps M = 6
+        Block b4;
+        quantize_block<false, true>(vv[u], bmax, g, 4.0f, b4);
+        pick4 = b4.err < b6.err;  // tie keeps M = 6
         if (pick4) {
-          sc = h4.sc;
-          q = h4.q;
+          sc = b4.sc;
+          q0 = b4.q0;
+          q1 = b4.q1;
         }
       }
       const uint32_t group = gather_group_scales(sc);
-      if (valid) {
-        codes[e0 >> 3] = q;
-        const int64_t fb = e0 >> 4;  // flat block index
-        if ((lane & 7) == 0) {
-          const int64_t row = fb / nblk_row, c = fb - row * nblk_row;
-          *reinterpret_cast<uint32_t*>(scales + scale_offset(row, c, kgroups)) = group;
-        }
-        if (kFos && choice && (lane & 1) == 0) choice[fb] = (uint8_t)pick4;
+      if (cc[u].valid) {
+        codes[cc[u].vec >> 1] = make_uint2(q0, q1);
+        if ((lane & 3) == 0)
+          *reinterpret_cast<uint32_t*>(scales + scale_offset(cc[u].row, cc[u].col >> 4, kgroups)) = group;
+        if (kFos && choice) choice[cc[u].vec >> 1] = (uint8_t)pick4;
       }
     }
   }
   if (!kFos && choice) {  // max mode still fills the optional choice map with 0
-    const int64_t nb = n >> 4;
+    const int64_t nb = (M * K) >> 4;
     for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nb;
          i += (int64_t)gridDim.x * blockDim.x)
       choice[i] = 0;
@@ -285,63 +305,61 @@ __global__ void __launch_bounds__(kQThreads) fake_quant_kernel(
   const float g = resolve_global_scale(partial, n_partial, g_static, &bad);
   if (blockIdx.x == 0 && threadIdx.x == 0 && bad) record_status(status, NVFP4_ERR_NONFINITE_INPUT);
   const int64_t kgroups = K >> 6;
-  const int64_t nblk_row = K >> 4;
-  const int64_t n = M * K;
-  const int64_t n_chunks = (n + 255) >> 8;
+  const int32_t cpr = (int32_t)((K + 511) >> 9);
+  const int64_t n_chunks = M * cpr;
   const int lane = threadIdx.x & 31;
   const int64_t warp = (int64_t)blockIdx.x * (kQThreads / 32) + (threadIdx.x >> 5);
   const int64_t nwarps = (int64_t)gridDim.x * (kQThreads / 32);
 
   for (int64_t ch0 = warp; ch0 < n_chunks; ch0 += kUnroll * nwarps) {
-    float vv[kUnroll][8];
+    float vv[kUnroll][16];
+    Chunk cc[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const int64_t e0 = ((ch0 + u * nwarps) << 8) + lane * 8;
-      load8(x, e0 >> 3, e0 < n, vv[u]);
+      cc[u] = chunk_at(ch0 + u * nwarps, cpr, K, lane);
+      load16(x, cc[u].vec, cc[u].valid && ch0 + u * nwarps < n_chunks, vv[u]);
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       if (ch0 + u * nwarps >= n_chunks) break;  // warp-uniform
-      const int64_t e0 = ((ch0 + u * nwarps) << 8) + lane * 8;
-      const bool valid = e0 < n;
-      float out[8];
+      float out[16];
       if (kFrozen) {
-        uint32_t sc = 1;
-        if (valid) {
-          const int64_t fb = e0 >> 4;
-          const int64_t row = fb / nblk_row, c = fb - row * nblk_row;
-          sc = scales_frozen[scale_offset(row, c, kgroups)];
-        }
+        const uint32_t sc = cc[u].valid ? scales_frozen[scale_offset(cc[u].row, cc[u].col >> 4, kgroups)] : 1u;
         const float d = __fmul_rn(g, e4m3_value(sc));
         const float r = __frcp_rn(d);
-        float sv[8];
+        float sv[16];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) sv[i] = __fmul_rn(vv[u][i], r);
-        const uint32_t q = e2m1_pack8(sv);
+        for (int i = 0; i < 16; ++i) sv[i] = __fmul_rn(vv[u][i], r);
+        const uint32_t q0 = e2m1_pack8(sv), q1 = e2m1_pack8(sv + 8);
 #pragma unroll
-        for (int i = 0; i < 8; ++i) out[i] = __fmul_rn(d, e2m1_value((q >> (4 * i)) & 0xFu));
+        for (int i = 0; i < 16; ++i) out[i] = __fmul_rn(d, e2m1_value(((i < 8 ? q0 : q1) >> (4 * (i & 7))) & 0xFu));
       } else {
-        const float bmax = block_max(vv[u]);
-        HalfBlock h6;
-        quantize_half<kFos>(vv[u], bmax, g, 6.0f, lane, h6);
+        const float bmax = abs_max16(vv[u]);
+        Block b6;
+        quantize_block<true, kFos>(vv[u], bmax, g, 6.0f, b6);
         if (kFos) {
-          HalfBlock h4;
-          quantize_half<true>(vv[u], bmax, g, 4.0f, lane, h4);
-          const bool pick4 = h4.err < h6.err;
+          Block b4;
+          quantize_block<true, true>(vv[u], bmax, g, 4.0f, b4);
+          const bool pick4 = b4.err < b6.err;
 #pragma unroll
-          for (int i = 0; i < 8; ++i) out[i] = pick4 ? h4.deq[i] : h6.deq[i];
+          for (int i = 0; i < 16; ++i) out[i] = pick4 ? b4.deq[i] : b6.deq[i];
         } else {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) out[i] = h6.deq[i];
+          for (int i = 0; i < 16; ++i) out[i] = b6.deq[i];
         }
       }
-      if (valid) {
-        uint4 w;
-        w.x = f32x2_to_bf16x2(out[0], out[1]);
-        w.y = f32x2_to_bf16x2(out[2], out[3]);
-        w.z = f32x2_to_bf16x2(out[4], out[5]);
-        w.w = f32x2_to_bf16x2(out[6], out[7]);
-        y[e0 >> 3] = w;
+      if (cc[u].valid) {
+        uint4 w0, w1;
+        w0.x = f32x2_to_bf16x2(out[0], out[1]);
+        w0.y = f32x2_to_bf16x2(out[2], out[3]);
+        w0.z = f32x2_to_bf16x2(out[4], out[5]);
+        w0.w = f32x2_to_bf16x2(out[6], out[7]);
+        w1.x = f32x2_to_bf16x2(out[8], out[9]);
+        w1.y = f32x2_to_bf16x2(out[10], out[11]);
+        w1.z = f32x2_to_bf16x2(out[12], out[13]);
+        w1.w = f32x2_to_bf16x2(out[14], out[15]);
+        y[cc[u].vec] = w0;
+        y[cc[u].vec + 1] = w1;
       }
     }
   }
@@ -389,7 +407,7 @@ static int grid_for(int64_t work_items, int per_block, int max_blocks) {
 
 int amax_partial_count(int64_t n, int num_sms) {
   // about 4 vectors of 8 BF16 per thread per loop trip, 4 CTAs per SM at most
-  return grid_for(n / 8, kAmaxThreads * 16, num_sms * 4 > kMaxPartials ? kMaxPartials : num_sms * 4);
+  return grid_for(n / 8, kAmaxThreads * 16, num_sms * 6 > kMaxPartials ? kMaxPartials : num_sms * 6);
 }
 
 cudaError_t launch_amax_partial(const void* x, int64_t n, uint32_t* partial, int n_partial,
@@ -408,17 +426,18 @@ static int resident_blocks(Kern k) {
 cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, bool fos, const uint32_t* partial,
                             int n_partial, const float* g_static, uint8_t* codes, uint8_t* scales,
                             float* g_out, uint8_t* choice, int* status, int num_sms, cudaStream_t s) {
-  const int64_t chunks = (M * K + 255) / 256;
+  const int64_t chunks = M * ((K + 511) / 512);
+  if (chunks >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
   static const int occ_max = resident_blocks(quantize_kernel<false>);
   static const int occ_fos = resident_blocks(quantize_kernel<true>);
   const int grid = grid_for(chunks, kQThreads / 32 * kUnroll, num_sms * (fos ? occ_fos : occ_max));
   if (fos)
     quantize_kernel<true><<<grid, kQThreads, 0, s>>>(static_cast<const uint4*>(x), M, K, partial, n_partial,
-                                                      g_static, reinterpret_cast<uint32_t*>(codes), scales,
+                                                      g_static, reinterpret_cast<uint2*>(codes), scales,
                                                       g_out, choice, status);
   else
     quantize_kernel<false><<<grid, kQThreads, 0, s>>>(static_cast<const uint4*>(x), M, K, partial, n_partial,
-                                                       g_static, reinterpret_cast<uint32_t*>(codes), scales,
+                                                       g_static, reinterpret_cast<uint2*>(codes), scales,
                                                        g_out, choice, status);
   return cudaGetLastError();
 }
@@ -426,7 +445,8 @@ cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, bool fos, const
 cudaError_t launch_fake_quant(const void* x, int64_t M, int64_t K, bool fos, const uint32_t* partial,
                               int n_partial, const float* g_static, const uint8_t* scales_frozen,
                               void* y, int* status, int num_sms, cudaStream_t s) {
-  const int64_t chunks = (M * K + 255) / 256;
+  const int64_t chunks = M * ((K + 511) / 512);
+  if (chunks >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
   static const int occ = resident_blocks(fake_quant_kernel<true, false>);
   const int grid = grid_for(chunks, kQThreads / 32 * kUnroll, num_sms * occ);
   const uint4* xv = static_cast<const uint4*>(x);
