@@ -86,7 +86,10 @@ const char* nvfp4_status_string(nvfp4_status s);
 size_t nvfp4_scale_bytes(int64_t rows, int64_t K);
 
 /* Workspace bytes nvfp4_quantize / nvfp4_fake_quant need to compute a dynamic
- * global scale for an [M x K] input (0 is never returned). Host only. */
+ * global scale for an [M x K] input (0 is never returned). The workspace
+ * holds a grid-wide barrier: zero-fill it once before its first use; every
+ * completed call leaves it ready for the next (after a call that reported
+ * NVFP4_ERR_TIMEOUT, zero-fill it again). Host only. */
 size_t nvfp4_quantize_workspace_bytes(int64_t M, int64_t K);
 
 /*
@@ -107,12 +110,15 @@ size_t nvfp4_quantize_workspace_bytes(int64_t M, int64_t K);
  * fos_choice  nullable out [M][K/16] bytes: 1 where the block kept the M=4
  *             scale, else 0 (always 0 in mode MAX).
  * workspace   >= nvfp4_quantize_workspace_bytes(M, K) bytes when g_in is
- *             NULL; may be NULL when g_in is given. Contents need no
- *             initialisation. Calls that share one workspace must be ordered
- *             on the GPU (same stream).
+ *             NULL (zero-filled before its first use, see above); may be
+ *             NULL when g_in is given. Calls that share one workspace must
+ *             be ordered on the GPU (same stream).
+ * A dynamic call is a single cooperative launch of one CTA per SM: each CTA
+ *   reduces the amax of its slice while keeping most of the slice in shared
+ *   memory, the CTAs meet at a grid-wide barrier, then quantize.
  * M may be 0 (nothing is written except g_out = 1 for a dynamic call).
  * Device status: NVFP4_ERR_NONFINITE_INPUT if amax is Inf/NaN (outputs are
- * then unspecified).
+ * then unspecified); NVFP4_ERR_TIMEOUT if the grid barrier wait ran out.
  */
 nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t K, nvfp4_mode mode,
                             const float* g_in, uint8_t* codes, uint8_t* scales,

@@ -131,6 +131,7 @@ def moe_workspace_bytes(T: int, H: int, I: int, E: int, topk: int) -> int:
 
 
 # Per-device scratch for the amax reduction (the library itself never allocates).
+# It holds a grid barrier and must start zero-filled.
 _ws_cache: dict = {}
 
 
@@ -138,7 +139,7 @@ def _workspace(device: torch.device, nbytes: int) -> torch.Tensor:
     key = (device.index, "q")
     ws = _ws_cache.get(key)
     if ws is None or ws.numel() < nbytes:
-        ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+        ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
         _ws_cache[key] = ws
     return ws
 

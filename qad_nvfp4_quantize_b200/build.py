@@ -21,7 +21,10 @@ OBJDIR = os.path.join(HERE, "_build")
 LIB = os.path.join(HERE, "libnvfp4.so")
 
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
-FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-Xcompiler", "-fPIC", "-DNDEBUG", f"-I{INCLUDE}"]
+# -fmad=false: no multiply is fused into a following add or subtract, packed
+# f32x2 operations included, so every FP32 product and sum of the method is
+# rounded on its own (the four_over_six error sum depends on it bit for bit).
+FLAGS = ["-O3", "-lineinfo", "-std=c++17", "-fmad=false", "-Xcompiler", "-fPIC", "-DNDEBUG", f"-I{INCLUDE}"]
 
 
 def _nvcc() -> str:
@@ -41,6 +44,10 @@ def build(verbose: bool = False, force: bool = False) -> str:
     nvcc = _nvcc()
     os.makedirs(OBJDIR, exist_ok=True)
     srcs = sorted(glob.glob(os.path.join(CSRC, "*.cu")))
+    stamp = os.path.join(OBJDIR, "flags.txt")
+    flags_line = " ".join([*ARCH, *FLAGS])
+    if not os.path.exists(stamp) or open(stamp).read() != flags_line:
+        force = True  # compiler flags changed since the objects were built
     newest_header = max((os.path.getmtime(h) for h in _headers()), default=0.0)
     jobs = []
     objs = []
@@ -62,6 +69,8 @@ def build(verbose: bool = False, force: bool = False) -> str:
         list(ex.map(run, jobs))
     if jobs or force or not os.path.exists(LIB):
         run([nvcc, *ARCH, "-shared", "-o", LIB, *objs])
+    with open(stamp, "w") as f:
+        f.write(flags_line)
     return LIB
 
 

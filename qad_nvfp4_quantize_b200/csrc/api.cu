@@ -107,7 +107,8 @@ size_t nvfp4_scale_bytes(int64_t rows, int64_t K) {
 size_t nvfp4_quantize_workspace_bytes(int64_t M, int64_t K) {
   (void)M;
   (void)K;
-  return (size_t)nvfp4::kMaxPartials * sizeof(uint32_t);
+  // partial maxima, then the two grid-barrier words (padded to 256 bytes)
+  return (size_t)nvfp4::kMaxPartials * sizeof(uint32_t) + 256;
 }
 
 nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t K, nvfp4_mode mode, const float* g_in,
@@ -123,12 +124,19 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t K, nvfp4_mode mode
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const uint32_t* partial = nullptr;
   int np = 0;
+  const bool fos = mode == NVFP4_MODE_FOUR_OVER_SIX;
   if (!g_in) {
+    if (!workspace || workspace_bytes < nvfp4_quantize_workspace_bytes(M, K) || !aligned16(workspace))
+      return NVFP4_ERR_WORKSPACE;
+    // one launch: amax, grid barrier and quantization with X kept on chip
+    const cudaError_t e = nvfp4::launch_quantize_fused(x, M, K, fos, static_cast<uint32_t*>(workspace), codes,
+                                                       scales, g_out, fos_choice, d->status, d->num_sms, s);
+    if (e != cudaErrorNotSupported) return launched(e);
     st = run_amax(x, M * K, workspace, workspace_bytes, d->num_sms, s, &partial, &np);
     if (st != NVFP4_OK) return st;
   }
-  return launched(nvfp4::launch_quantize(x, M, K, mode == NVFP4_MODE_FOUR_OVER_SIX, partial, np, g_in,
-                                         codes, scales, g_out, fos_choice, d->status, d->num_sms, s));
+  return launched(nvfp4::launch_quantize(x, M, K, fos, partial, np, g_in, codes, scales, g_out, fos_choice,
+                                         d->status, d->num_sms, s));
 }
 
 nvfp4_status nvfp4_fake_quant(const void* x, int64_t M, int64_t K, nvfp4_mode mode, const float* g_frozen,
@@ -144,12 +152,18 @@ nvfp4_status nvfp4_fake_quant(const void* x, int64_t M, int64_t K, nvfp4_mode mo
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const uint32_t* partial = nullptr;
   int np = 0;
+  const bool fos = mode == NVFP4_MODE_FOUR_OVER_SIX;
   if (!g_frozen) {
+    if (!workspace || workspace_bytes < nvfp4_quantize_workspace_bytes(M, K) || !aligned16(workspace))
+      return NVFP4_ERR_WORKSPACE;
+    const cudaError_t e =
+        nvfp4::launch_fake_quant_fused(x, M, K, fos, static_cast<uint32_t*>(workspace), y, d->status, d->num_sms, s);
+    if (e != cudaErrorNotSupported) return launched(e);
     st = run_amax(x, M * K, workspace, workspace_bytes, d->num_sms, s, &partial, &np);
     if (st != NVFP4_OK) return st;
   }
-  return launched(nvfp4::launch_fake_quant(x, M, K, mode == NVFP4_MODE_FOUR_OVER_SIX, partial, np, g_frozen,
-                                           scales_frozen, y, d->status, d->num_sms, s));
+  return launched(nvfp4::launch_fake_quant(x, M, K, fos, partial, np, g_frozen, scales_frozen, y, d->status,
+                                           d->num_sms, s));
 }
 
 nvfp4_status nvfp4_gemm(const uint8_t* Aq, const uint8_t* As, const float* ga, const uint8_t* Bq,

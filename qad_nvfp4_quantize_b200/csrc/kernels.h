@@ -18,6 +18,15 @@ cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, bool fos, const
 cudaError_t launch_fake_quant(const void* x, int64_t M, int64_t K, bool fos, const uint32_t* partial,
                               int n_partial, const float* g_static, const uint8_t* scales_frozen,
                               void* y, int* status, int num_sms, cudaStream_t s);
+// Fused single-launch dynamic quantize / fake-quant (amax, grid barrier,
+// quantization). ws: kMaxPartials partial slots followed by two barrier
+// words that must be zero before the first use. Returns
+// cudaErrorNotSupported when the cooperative launch is not possible.
+cudaError_t launch_quantize_fused(const void* x, int64_t M, int64_t K, bool fos, uint32_t* ws, uint8_t* codes,
+                                  uint8_t* scales, float* g_out, uint8_t* choice, int* status, int num_sms,
+                                  cudaStream_t s);
+cudaError_t launch_fake_quant_fused(const void* x, int64_t M, int64_t K, bool fos, uint32_t* ws, void* y,
+                                    int* status, int num_sms, cudaStream_t s);
 cudaError_t launch_convert(const float* in, int64_t n, uint8_t* out, bool e4m3, int num_sms,
                            cudaStream_t s);
 cudaError_t launch_selftest_timeout(uint64_t timeout_ns, int* status, cudaStream_t s);

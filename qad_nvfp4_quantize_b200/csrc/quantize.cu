@@ -24,6 +24,7 @@ constexpr int kQThreads = 256;  // 8 warps
 constexpr int kAmaxThreads = 256;
 constexpr unsigned kFull = 0xFFFFFFFFu;
 constexpr int kUnroll = 2;  // chunks of 512 elements in flight per warp
+constexpr uint64_t kFusedTimeoutNs = 2000000000ull;  // grid-barrier wait bound
 
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   uint4 v;
@@ -145,65 +146,125 @@ __device__ __forceinline__ Chunk chunk_at(int64_t ch, int32_t cpr, int64_t K, in
   return c;
 }
 
-__device__ __forceinline__ void load16(const uint4* x, int64_t vec, bool valid, float (&v)[16]) {
+// Two FP32 values in one 64-bit register (element 2j in the low half), for
+// the packed sm_100 f32x2 instructions; each half is an IEEE FP32 operation.
+typedef unsigned long long f32x2;
+
+__device__ __forceinline__ f32x2 pack2(float lo, float hi) {
+  f32x2 r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack2(f32x2 v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ f32x2 mul2(f32x2 a, f32x2 b) {
+  f32x2 r;
+  asm("mul.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+__device__ __forceinline__ f32x2 sub2(f32x2 a, f32x2 b) {
+  f32x2 r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+// BF16 pair (one 32-bit word) -> FP32 pair, exact.
+__device__ __forceinline__ f32x2 bf16x2_unpack(uint32_t w) {
+  return pack2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
+}
+// FP32 pair -> one byte of two E2M1 codes (low element in the low nibble).
+__device__ __forceinline__ uint32_t e2m1x2(f32x2 v) {
+  float lo, hi;
+  unpack2(v, lo, hi);
+  uint16_t out;
+  asm("{\n\t.reg .b8 q;\n\tcvt.rn.satfinite.e2m1x2.f32 q, %2, %1;\n\tcvt.u16.u8 %0, q;\n\t}"
+      : "=h"(out) : "f"(lo), "f"(hi));
+  return out & 0xFFu;
+}
+// Byte of two E2M1 codes -> their two values as FP32 (exact, through f16x2).
+__device__ __forceinline__ f32x2 e2m1x2_value(uint32_t byte) {
+  float lo, hi;
+  asm("{\n\t.reg .b8 t;\n\t.reg .b32 h2;\n\t.reg .b16 a, b;\n\t"
+      "cvt.u8.u32 t, %2;\n\tcvt.rn.f16x2.e2m1x2 h2, t;\n\t"
+      "mov.b32 {a, b}, h2;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
+      : "=f"(lo), "=f"(hi) : "r"(byte));
+  return pack2(lo, hi);
+}
+
+// A lane's 16-element block as 8 raw BF16 words.
+struct Raw16 {
+  uint32_t w[8];
+};
+
+__device__ __forceinline__ void load_raw16(const uint4* x, int64_t vec, bool valid, Raw16& r) {
   uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
   if (valid) {
     a = ld_stream(x + vec);
     b = ld_stream(x + vec + 1);
   }
-  bf16x2_to_f32(a.x, v[0], v[1]);
-  bf16x2_to_f32(a.y, v[2], v[3]);
-  bf16x2_to_f32(a.z, v[4], v[5]);
-  bf16x2_to_f32(a.w, v[6], v[7]);
-  bf16x2_to_f32(b.x, v[8], v[9]);
-  bf16x2_to_f32(b.y, v[10], v[11]);
-  bf16x2_to_f32(b.z, v[12], v[13]);
-  bf16x2_to_f32(b.w, v[14], v[15]);
+  r.w[0] = a.x; r.w[1] = a.y; r.w[2] = a.z; r.w[3] = a.w;
+  r.w[4] = b.x; r.w[5] = b.y; r.w[6] = b.z; r.w[7] = b.w;
 }
 
-// One 16-element block: scale code, packed codes (two 32-bit words, element 2j
-// in the low nibble of byte j) and, when requested, the dequantized values
-// and the block's squared error summed in element order.
+// max |x| of the block (BF16 magnitudes order like their bit patterns).
+__device__ __forceinline__ float block_absmax(const Raw16& r) {
+  uint32_t m2 = 0;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) m2 = __vmaxu2(m2, r.w[i] & 0x7FFF7FFFu);
+  return __uint_as_float(max(m2 & 0xFFFFu, m2 >> 16) << 16);
+}
+
+// One 16-element block: scale code, packed codes (two 32-bit words, element
+// 2j in the low nibble of byte j) and, when requested, the dequantized values
+// (pairs) and the block's squared error summed in element order.
 struct Block {
   uint32_t sc;
   uint32_t q0, q1;
-  float deq[16];
+  f32x2 deq[8];
   float err;
 };
 
 template <bool kDeq, bool kErr>
-__device__ __forceinline__ void quantize_block(const float (&v)[16], float bmax, float g, float mt, Block& b) {
+__device__ __forceinline__ void quantize_block(const Raw16& raw, float bmax, float g, float mt, Block& b) {
   b.sc = block_scale_code(bmax, g, mt);
   const float d = __fmul_rn(g, e4m3_value(b.sc));
   const float r = __frcp_rn(d);
-  float sv[16];
+  const f32x2 rr = pack2(r, r);
+  uint32_t bytes[8];
 #pragma unroll
-  for (int i = 0; i < 16; ++i) sv[i] = __fmul_rn(v[i], r);
-  b.q0 = e2m1_pack8(sv);
-  b.q1 = e2m1_pack8(sv + 8);
-  if (kDeq || kErr) {
+  for (int i = 0; i < 8; ++i) bytes[i] = e2m1x2(mul2(bf16x2_unpack(raw.w[i]), rr));
+  b.q0 = bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24);
+  b.q1 = bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24);
+  if (kErr) {
+    // Scalar products here: with a packed multiply feeding the packed
+    // subtraction below, the compiler was seen to fuse the two into one
+    // fused multiply-add (one rounding of x - d*q where the method rounds
+    // d*q first), which flips near-tie four_over_six choices.
 #pragma unroll
-    for (int i = 0; i < 16; ++i)
-      b.deq[i] = __fmul_rn(d, e2m1_value(((i < 8 ? b.q0 : b.q1) >> (4 * (i & 7))) & 0xFu));
+    for (int i = 0; i < 8; ++i) {
+      float lo, hi;
+      unpack2(e2m1x2_value(bytes[i]), lo, hi);
+      b.deq[i] = pack2(__fmul_rn(d, lo), __fmul_rn(d, hi));
+    }
+  } else if (kDeq) {
+    const f32x2 dd = pack2(d, d);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) b.deq[i] = mul2(dd, e2m1x2_value(bytes[i]));
   }
   if (kErr) {
     float acc = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const float df = __fsub_rn(v[i], b.deq[i]);
-      acc = __fadd_rn(acc, __fmul_rn(df, df));
+    for (int i = 0; i < 8; ++i) {
+      const f32x2 df = sub2(bf16x2_unpack(raw.w[i]), b.deq[i]);
+      float lo, hi;
+      unpack2(mul2(df, df), lo, hi);
+      acc = __fadd_rn(acc, lo);  // element order: 2i, then 2i+1
+      acc = __fadd_rn(acc, hi);
     }
     b.err = acc;
   } else {
     b.err = 0.0f;
   }
-}
-
-__device__ __forceinline__ float abs_max16(const float (&v)[16]) {
-  float m = 0.0f;
-#pragma unroll
-  for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(v[i]));
-  return m;
 }
 
 // Gather the scale codes of the 4 blocks of a 64-element group onto the
@@ -227,21 +288,126 @@ __device__ __forceinline__ void zero_pad_scale_rows(uint8_t* scales, int64_t M, 
 }
 
 // ----------------------------------------------------------------------------
-// Quantize (pass 2). kFos: four_over_six calibration.
+// Per-block operations. Each maps one lane's 16-element block (with the
+// chunk it belongs to and the global scale) to the call's outputs.
 // ----------------------------------------------------------------------------
+
+// Quantize: codes, tiled block scales and (four_over_six) the choice map.
 template <bool kFos>
-__global__ void __launch_bounds__(kQThreads) quantize_kernel(
-    const uint4* __restrict__ x, int64_t M, int64_t K, const uint32_t* __restrict__ partial,
-    int n_partial, const float* __restrict__ g_static, uint2* __restrict__ codes,
-    uint8_t* __restrict__ scales, float* __restrict__ g_out, uint8_t* __restrict__ choice,
-    int* status) {
+struct QuantOp {
+  uint2* codes;
+  uint8_t* scales;
+  uint8_t* choice;
+  int64_t M, K;
+
+  __device__ __forceinline__ void operator()(const Raw16& v, const Chunk& c, float g, int lane) const {
+    const float bmax = block_absmax(v);
+    Block b6;
+    quantize_block<false, kFos>(v, bmax, g, 6.0f, b6);
+    uint32_t sc = b6.sc, q0 = b6.q0, q1 = b6.q1, pick4 = 0;
+    if (kFos) {
+      Block b4;
+      quantize_block<false, true>(v, bmax, g, 4.0f, b4);
+      pick4 = b4.err < b6.err;  // tie keeps M = 6
+      if (pick4) {
+        sc = b4.sc;
+        q0 = b4.q0;
+        q1 = b4.q1;
+      }
+    }
+    const uint32_t group = gather_group_scales(sc);
+    if (c.valid) {
+      codes[c.vec >> 1] = make_uint2(q0, q1);
+      if ((lane & 3) == 0)
+        *reinterpret_cast<uint32_t*>(scales + scale_offset(c.row, c.col >> 4, K >> 6)) = group;
+      if (kFos && choice) choice[c.vec >> 1] = (uint8_t)pick4;
+    }
+  }
+
+  // Work independent of the values: zero padding-row scales; a max-mode call
+  // that asked for a choice map gets zeros.
+  __device__ __forceinline__ void finish() const {
+    if (!kFos && choice) {
+      const int64_t nb = (M * K) >> 4;
+      for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nb;
+           i += (int64_t)gridDim.x * blockDim.x)
+        choice[i] = 0;
+    }
+    zero_pad_scale_rows(scales, M, K >> 6);
+  }
+};
+
+// Fake-quant with block scales computed from the values (max or four_over_six).
+template <bool kFos>
+struct FakeOp {
+  uint4* y;
+  int64_t M, K;
+
+  __device__ __forceinline__ void operator()(const Raw16& v, const Chunk& c, float g, int lane) const {
+    (void)lane;
+    const float bmax = block_absmax(v);
+    Block b6;
+    quantize_block<true, kFos>(v, bmax, g, 6.0f, b6);
+    if (kFos) {
+      Block b4;
+      quantize_block<true, true>(v, bmax, g, 4.0f, b4);
+      if (b4.err < b6.err) {
+        store_bf16x16(y, c, b4.deq);
+        return;
+      }
+    }
+    store_bf16x16(y, c, b6.deq);
+  }
+  __device__ __forceinline__ void finish() const {}
+
+  __device__ static __forceinline__ uint32_t to_bf16x2(f32x2 v) {
+    float lo, hi;
+    unpack2(v, lo, hi);
+    return f32x2_to_bf16x2(lo, hi);
+  }
+
+  __device__ static __forceinline__ void store_bf16x16(uint4* y, const Chunk& c, const f32x2 (&out)[8]) {
+    if (!c.valid) return;
+    y[c.vec] = make_uint4(to_bf16x2(out[0]), to_bf16x2(out[1]), to_bf16x2(out[2]), to_bf16x2(out[3]));
+    y[c.vec + 1] = make_uint4(to_bf16x2(out[4]), to_bf16x2(out[5]), to_bf16x2(out[6]), to_bf16x2(out[7]));
+  }
+};
+
+// Fake-quant with frozen block scales s* (tiled layout) and frozen g*.
+struct FrozenFakeOp {
+  uint4* y;
+  const uint8_t* scales_frozen;
+  int64_t M, K;
+
+  __device__ __forceinline__ void operator()(const Raw16& v, const Chunk& c, float g, int lane) const {
+    (void)lane;
+    const uint32_t sc = c.valid ? scales_frozen[scale_offset(c.row, c.col >> 4, K >> 6)] : 1u;
+    const float d = __fmul_rn(g, e4m3_value(sc));
+    const float r = __frcp_rn(d);
+    const f32x2 rr = pack2(r, r), dd = pack2(d, d);
+    f32x2 out[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) out[i] = mul2(dd, e2m1x2_value(e2m1x2(mul2(bf16x2_unpack(v.w[i]), rr))));
+    FakeOp<false>::store_bf16x16(y, c, out);
+  }
+  __device__ __forceinline__ void finish() const {}
+};
+
+// ----------------------------------------------------------------------------
+// Streaming pass with a known global scale (static g, or g reduced from the
+// partials of a separate amax pass): grid-stride over 512-element chunks.
+// ----------------------------------------------------------------------------
+template <class Op>
+__global__ void __launch_bounds__(kQThreads) stream_pass_kernel(const uint4* __restrict__ x, int64_t M, int64_t K,
+                                                                 const uint32_t* __restrict__ partial, int n_partial,
+                                                                 const float* __restrict__ g_static, Op op,
+                                                                 float* __restrict__ g_out, int* status) {
   bool bad;
   const float g = resolve_global_scale(partial, n_partial, g_static, &bad);
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     if (g_out) *g_out = g;
     if (bad) record_status(status, NVFP4_ERR_NONFINITE_INPUT);
   }
-  const int64_t kgroups = K >> 6;
   const int32_t cpr = (int32_t)((K + 511) >> 9);
   const int64_t n_chunks = M * cpr;
   const int lane = threadIdx.x & 31;
@@ -250,119 +416,191 @@ __global__ void __launch_bounds__(kQThreads) quantize_kernel(
 
   // kUnroll chunks per trip with all loads issued first (memory-level parallelism)
   for (int64_t ch0 = warp; ch0 < n_chunks; ch0 += kUnroll * nwarps) {
-    float vv[kUnroll][16];
+    Raw16 vv[kUnroll];
     Chunk cc[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       cc[u] = chunk_at(ch0 + u * nwarps, cpr, K, lane);
-      load16(x, cc[u].vec, cc[u].valid && ch0 + u * nwarps < n_chunks, vv[u]);
+      load_raw16(x, cc[u].vec, cc[u].valid && ch0 + u * nwarps < n_chunks, vv[u]);
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       if (ch0 + u * nwarps >= n_chunks) break;  // warp-uniform
-      const float bmax = abs_max16(vv[u]);
-      Block b6;
-      quantize_block<false, kFos>(vv[u], bmax, g, 6.0f, b6);
-      uint32_t sc = b6.sc, q0 = b6.q0, q1 = b6.q1, pick4 = 0;
-      if (kFos) {
-        Block b4;
-        quantize_block<false, true>(vv[u], bmax, g, 4.0f, b4);
-        pick4 = b4.err < b6.err;  // tie keeps M = 6
-        if (pick4) {
-          sc = b4.sc;
-          q0 = b4.q0;
-          q1 = b4.q1;
-        }
-      }
-      const uint32_t group = gather_group_scales(sc);
-      if (cc[u].valid) {
-        codes[cc[u].vec >> 1] = make_uint2(q0, q1);
-        if ((lane & 3) == 0)
-          *reinterpret_cast<uint32_t*>(scales + scale_offset(cc[u].row, cc[u].col >> 4, kgroups)) = group;
-        if (kFos && choice) choice[cc[u].vec >> 1] = (uint8_t)pick4;
-      }
+      op(vv[u], cc[u], g, lane);
     }
   }
-  if (!kFos && choice) {  // max mode still fills the optional choice map with 0
-    const int64_t nb = (M * K) >> 4;
-    for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < nb;
-         i += (int64_t)gridDim.x * blockDim.x)
-      choice[i] = 0;
-  }
-  zero_pad_scale_rows(scales, M, kgroups);
+  op.finish();
 }
 
 // ----------------------------------------------------------------------------
-// Fake-quant: y = BF16(g * s * q). Modes: dynamic/static g with computed block
-// scales (max or four_over_six), or frozen g* and s* (tiled layout).
+// Fused dynamic pass: amax and quantization in one persistent launch.
+//
+// One CTA per SM (cooperative launch, so all CTAs are resident). CTA c owns a
+// contiguous range of chunks. Phase 1 streams the range once, reducing the
+// BF16 magnitude maximum and keeping the first kKeepChunks chunks (up to
+// 200 KB) in shared memory. The CTA maxima meet at a grid-wide barrier (two
+// words in the workspace, returned to zero by every completed barrier, so the
+// workspace must be zero before its first use). Phase 2 walks the range
+// backwards: the chunks that were not kept -- read last in phase 1, so the
+// most likely to still be in L2 -- are read again from global memory, the
+// kept ones come from shared memory. X therefore crosses HBM about once.
 // ----------------------------------------------------------------------------
-template <bool kFos, bool kFrozen>
-__global__ void __launch_bounds__(kQThreads) fake_quant_kernel(
-    const uint4* __restrict__ x, int64_t M, int64_t K, const uint32_t* __restrict__ partial,
-    int n_partial, const float* __restrict__ g_static, const uint8_t* __restrict__ scales_frozen,
-    uint4* __restrict__ y, int* status) {
-  bool bad;
-  const float g = resolve_global_scale(partial, n_partial, g_static, &bad);
-  if (blockIdx.x == 0 && threadIdx.x == 0 && bad) record_status(status, NVFP4_ERR_NONFINITE_INPUT);
-  const int64_t kgroups = K >> 6;
+constexpr int kFusedThreads = 1024;
+constexpr int kFusedWarps = kFusedThreads / 32;
+constexpr int kKeepChunks = 200;                       // 1 KB of BF16 per chunk
+constexpr int kFusedSmem = kKeepChunks * 1024;
+constexpr int kFusedUnroll = 2;
+
+// Grid-wide barrier on bar[0] (arrivals) and bar[1] (generation). Returns
+// false if the wait ran out (the status is recorded by the caller).
+__device__ __forceinline__ bool grid_barrier(uint32_t* bar, uint64_t timeout_ns) {
+  __shared__ int s_ok;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    volatile uint32_t* vgen = bar + 1;
+    const uint32_t gen = *vgen;
+    __threadfence();
+    int ok = 1;
+    if (atomicAdd(bar, 1u) == gridDim.x - 1) {
+      atomicExch(bar, 0u);
+      __threadfence();
+      atomicAdd(bar + 1, 1u);
+    } else {
+      const uint64_t t0 = globaltimer_ns();
+      while (*vgen == gen) {
+        if (globaltimer_ns() - t0 > timeout_ns) {
+          ok = 0;
+          break;
+        }
+        __nanosleep(64);
+      }
+    }
+    __threadfence();
+    s_ok = ok;
+  }
+  __syncthreads();
+  return s_ok != 0;
+}
+
+template <class Op>
+__global__ void __launch_bounds__(kFusedThreads, 1) fused_dynamic_kernel(const uint4* __restrict__ x, int64_t M,
+                                                                           int64_t K, uint32_t* partial, uint32_t* bar,
+                                                                           Op op, float* g_out, int* status,
+                                                                           uint64_t timeout_ns) {
+  extern __shared__ uint4 keep[];
+  __shared__ uint32_t red[kFusedWarps];
+  __shared__ float s_g;
+  __shared__ int s_bad;
+  const int lane = threadIdx.x & 31;
+  const int warp = threadIdx.x >> 5;
   const int32_t cpr = (int32_t)((K + 511) >> 9);
   const int64_t n_chunks = M * cpr;
-  const int lane = threadIdx.x & 31;
-  const int64_t warp = (int64_t)blockIdx.x * (kQThreads / 32) + (threadIdx.x >> 5);
-  const int64_t nwarps = (int64_t)gridDim.x * (kQThreads / 32);
+  const int64_t per = (n_chunks + gridDim.x - 1) / gridDim.x;
+  const int64_t lo = (int64_t)blockIdx.x * per;
+  const int64_t hi = lo + per < n_chunks ? lo + per : n_chunks;
+  const int64_t nkeep = hi - lo < kKeepChunks ? (hi - lo > 0 ? hi - lo : 0) : kKeepChunks;
 
-  for (int64_t ch0 = warp; ch0 < n_chunks; ch0 += kUnroll * nwarps) {
-    float vv[kUnroll][16];
-    Chunk cc[kUnroll];
+  // ---- phase 1: magnitude maximum, keep the first nkeep chunks
+  uint32_t m2 = 0;
+  for (int64_t base = lo + warp; base < hi; base += kFusedUnroll * kFusedWarps) {
+    uint4 a[kFusedUnroll], b[kFusedUnroll];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      cc[u] = chunk_at(ch0 + u * nwarps, cpr, K, lane);
-      load16(x, cc[u].vec, cc[u].valid && ch0 + u * nwarps < n_chunks, vv[u]);
-    }
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      if (ch0 + u * nwarps >= n_chunks) break;  // warp-uniform
-      float out[16];
-      if (kFrozen) {
-        const uint32_t sc = cc[u].valid ? scales_frozen[scale_offset(cc[u].row, cc[u].col >> 4, kgroups)] : 1u;
-        const float d = __fmul_rn(g, e4m3_value(sc));
-        const float r = __frcp_rn(d);
-        float sv[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) sv[i] = __fmul_rn(vv[u][i], r);
-        const uint32_t q0 = e2m1_pack8(sv), q1 = e2m1_pack8(sv + 8);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) out[i] = __fmul_rn(d, e2m1_value(((i < 8 ? q0 : q1) >> (4 * (i & 7))) & 0xFu));
-      } else {
-        const float bmax = abs_max16(vv[u]);
-        Block b6;
-        quantize_block<true, kFos>(vv[u], bmax, g, 6.0f, b6);
-        if (kFos) {
-          Block b4;
-          quantize_block<true, true>(vv[u], bmax, g, 4.0f, b4);
-          const bool pick4 = b4.err < b6.err;
-#pragma unroll
-          for (int i = 0; i < 16; ++i) out[i] = pick4 ? b4.deq[i] : b6.deq[i];
-        } else {
-#pragma unroll
-          for (int i = 0; i < 16; ++i) out[i] = b6.deq[i];
+    for (int u = 0; u < kFusedUnroll; ++u) {
+      const int64_t ch = base + u * kFusedWarps;
+      a[u] = b[u] = make_uint4(0, 0, 0, 0);
+      if (ch < hi) {
+        const Chunk c = chunk_at(ch, cpr, K, lane);
+        if (c.valid) {
+          a[u] = ld_stream(x + c.vec);
+          b[u] = ld_stream(x + c.vec + 1);
         }
       }
-      if (cc[u].valid) {
-        uint4 w0, w1;
-        w0.x = f32x2_to_bf16x2(out[0], out[1]);
-        w0.y = f32x2_to_bf16x2(out[2], out[3]);
-        w0.z = f32x2_to_bf16x2(out[4], out[5]);
-        w0.w = f32x2_to_bf16x2(out[6], out[7]);
-        w1.x = f32x2_to_bf16x2(out[8], out[9]);
-        w1.y = f32x2_to_bf16x2(out[10], out[11]);
-        w1.z = f32x2_to_bf16x2(out[12], out[13]);
-        w1.w = f32x2_to_bf16x2(out[14], out[15]);
-        y[cc[u].vec] = w0;
-        y[cc[u].vec + 1] = w1;
+    }
+#pragma unroll
+    for (int u = 0; u < kFusedUnroll; ++u) {
+      m2 = __vmaxu2(m2, a[u].x & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, a[u].y & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, a[u].z & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, a[u].w & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, b[u].x & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, b[u].y & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, b[u].z & 0x7FFF7FFFu);
+      m2 = __vmaxu2(m2, b[u].w & 0x7FFF7FFFu);
+      const int64_t k = base + u * kFusedWarps - lo;
+      if (k < nkeep) {  // lane-contiguous halves: conflict-free 512-byte rows
+        keep[k * 64 + lane] = a[u];
+        keep[k * 64 + 32 + lane] = b[u];
       }
     }
   }
+  uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFull, m, o));
+  if (lane == 0) red[warp] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t r = 0;
+    for (int w = 0; w < kFusedWarps; ++w) r = max(r, red[w]);
+    partial[blockIdx.x] = r;
+  }
+
+  // ---- grid-wide maximum -> global scale
+  if (!grid_barrier(bar, timeout_ns) && threadIdx.x == 0) record_status(status, NVFP4_ERR_TIMEOUT);
+  if (threadIdx.x < 32) {
+    uint32_t mm = 0;
+    for (int base = 0; base < (int)gridDim.x; base += 8 * 32) {
+      uint32_t v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        const int i = base + u * 32 + lane;
+        v[u] = i < (int)gridDim.x ? __ldcg(partial + i) : 0u;
+      }
+#pragma unroll
+      for (int u = 0; u < 8; ++u) mm = max(mm, v[u]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) mm = max(mm, __shfl_xor_sync(kFull, mm, o));
+    if (lane == 0) {
+      s_g = global_scale_from_amax(__uint_as_float(mm << 16));
+      s_bad = mm >= 0x7F80u;
+    }
+  }
+  __syncthreads();
+  const float g = s_g;
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    if (g_out) *g_out = g;
+    if (s_bad) record_status(status, NVFP4_ERR_NONFINITE_INPUT);
+  }
+
+  // ---- phase 2: backwards, re-read chunks that were not kept, then kept ones
+  for (int64_t top = hi - 1 - warp; top >= lo; top -= kFusedUnroll * kFusedWarps) {
+    Raw16 vv[kFusedUnroll];
+    Chunk cc[kFusedUnroll];
+#pragma unroll
+    for (int u = 0; u < kFusedUnroll; ++u) {
+      const int64_t ch = top - u * kFusedWarps;
+      uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+      cc[u] = chunk_at(ch >= lo ? ch : lo, cpr, K, lane);
+      if (ch >= lo && cc[u].valid) {
+        const int64_t k = ch - lo;
+        if (k < nkeep) {
+          a = keep[k * 64 + lane];
+          b = keep[k * 64 + 32 + lane];
+        } else {
+          a = ld_stream(x + cc[u].vec);
+          b = ld_stream(x + cc[u].vec + 1);
+        }
+      }
+      vv[u].w[0] = a.x; vv[u].w[1] = a.y; vv[u].w[2] = a.z; vv[u].w[3] = a.w;
+      vv[u].w[4] = b.x; vv[u].w[5] = b.y; vv[u].w[6] = b.z; vv[u].w[7] = b.w;
+    }
+#pragma unroll
+    for (int u = 0; u < kFusedUnroll; ++u) {
+      if (top - u * kFusedWarps < lo) break;  // warp-uniform
+      op(vv[u], cc[u], g, lane);
+    }
+  }
+  op.finish();
 }
 
 // ----------------------------------------------------------------------------
@@ -417,50 +655,87 @@ cudaError_t launch_amax_partial(const void* x, int64_t n, uint32_t* partial, int
 }
 
 template <class Kern>
-static int resident_blocks(Kern k) {
+static int resident_blocks(Kern k, int threads, size_t smem) {
   int b = 0;
-  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, k, kQThreads, 0) != cudaSuccess || b < 1) b = 1;
+  if (cudaOccupancyMaxActiveBlocksPerMultiprocessor(&b, k, threads, smem) != cudaSuccess || b < 1) b = 0;
   return b;
+}
+
+template <class Op>
+static cudaError_t launch_stream(const void* x, int64_t M, int64_t K, const uint32_t* partial, int n_partial,
+                                 const float* g_static, const Op& op, float* g_out, int* status, int num_sms,
+                                 cudaStream_t s) {
+  const int64_t chunks = M * ((K + 511) / 512);
+  if (chunks >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+  static const int occ = resident_blocks(stream_pass_kernel<Op>, kQThreads, 0);
+  const int grid = grid_for(chunks, kQThreads / 32 * kUnroll, num_sms * (occ > 0 ? occ : 1));
+  stream_pass_kernel<Op><<<grid, kQThreads, 0, s>>>(static_cast<const uint4*>(x), M, K, partial, n_partial, g_static,
+                                                     op, g_out, status);
+  return cudaGetLastError();
+}
+
+// Fused dynamic launch; returns cudaErrorNotSupported when a cooperative
+// launch of one CTA per SM is not possible (the caller then runs two passes).
+template <class Op>
+static cudaError_t launch_fused(const void* x, int64_t M, int64_t K, uint32_t* ws, const Op& op, float* g_out,
+                                int* status, int num_sms, cudaStream_t s) {
+  const int64_t chunks = M * ((K + 511) / 512);
+  if (chunks >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+  static cudaError_t attr = cudaFuncSetAttribute(fused_dynamic_kernel<Op>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                 kFusedSmem);
+  static const int occ = attr == cudaSuccess ? resident_blocks(fused_dynamic_kernel<Op>, kFusedThreads, kFusedSmem) : 0;
+  if (occ < 1 || num_sms > kMaxPartials) return cudaErrorNotSupported;
+  const uint4* xv = static_cast<const uint4*>(x);
+  uint32_t* partial = ws;
+  uint32_t* bar = ws + kMaxPartials;
+  uint64_t timeout_ns = kFusedTimeoutNs;
+  void* args[] = {(void*)&xv, (void*)&M, (void*)&K, (void*)&partial, (void*)&bar, (void*)&op, (void*)&g_out,
+                  (void*)&status, (void*)&timeout_ns};
+  const cudaError_t e = cudaLaunchCooperativeKernel((const void*)fused_dynamic_kernel<Op>, dim3(num_sms),
+                                                    dim3(kFusedThreads), args, kFusedSmem, s);
+  if (e == cudaErrorCooperativeLaunchTooLarge) {
+    (void)cudaGetLastError();
+    return cudaErrorNotSupported;
+  }
+  return e;
 }
 
 cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, bool fos, const uint32_t* partial,
                             int n_partial, const float* g_static, uint8_t* codes, uint8_t* scales,
                             float* g_out, uint8_t* choice, int* status, int num_sms, cudaStream_t s) {
-  const int64_t chunks = M * ((K + 511) / 512);
-  if (chunks >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
-  static const int occ_max = resident_blocks(quantize_kernel<false>);
-  static const int occ_fos = resident_blocks(quantize_kernel<true>);
-  const int grid = grid_for(chunks, kQThreads / 32 * kUnroll, num_sms * (fos ? occ_fos : occ_max));
+  uint2* c = reinterpret_cast<uint2*>(codes);
   if (fos)
-    quantize_kernel<true><<<grid, kQThreads, 0, s>>>(static_cast<const uint4*>(x), M, K, partial, n_partial,
-                                                      g_static, reinterpret_cast<uint2*>(codes), scales,
-                                                      g_out, choice, status);
-  else
-    quantize_kernel<false><<<grid, kQThreads, 0, s>>>(static_cast<const uint4*>(x), M, K, partial, n_partial,
-                                                       g_static, reinterpret_cast<uint2*>(codes), scales,
-                                                       g_out, choice, status);
-  return cudaGetLastError();
+    return launch_stream(x, M, K, partial, n_partial, g_static, QuantOp<true>{c, scales, choice, M, K}, g_out, status,
+                         num_sms, s);
+  return launch_stream(x, M, K, partial, n_partial, g_static, QuantOp<false>{c, scales, choice, M, K}, g_out, status,
+                       num_sms, s);
 }
 
 cudaError_t launch_fake_quant(const void* x, int64_t M, int64_t K, bool fos, const uint32_t* partial,
                               int n_partial, const float* g_static, const uint8_t* scales_frozen,
                               void* y, int* status, int num_sms, cudaStream_t s) {
-  const int64_t chunks = M * ((K + 511) / 512);
-  if (chunks >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
-  static const int occ = resident_blocks(fake_quant_kernel<true, false>);
-  const int grid = grid_for(chunks, kQThreads / 32 * kUnroll, num_sms * occ);
-  const uint4* xv = static_cast<const uint4*>(x);
   uint4* yv = static_cast<uint4*>(y);
   if (scales_frozen)
-    fake_quant_kernel<false, true><<<grid, kQThreads, 0, s>>>(xv, M, K, partial, n_partial, g_static,
-                                                              scales_frozen, yv, status);
-  else if (fos)
-    fake_quant_kernel<true, false><<<grid, kQThreads, 0, s>>>(xv, M, K, partial, n_partial, g_static,
-                                                              nullptr, yv, status);
-  else
-    fake_quant_kernel<false, false><<<grid, kQThreads, 0, s>>>(xv, M, K, partial, n_partial, g_static,
-                                                               nullptr, yv, status);
-  return cudaGetLastError();
+    return launch_stream(x, M, K, partial, n_partial, g_static, FrozenFakeOp{yv, scales_frozen, M, K}, nullptr,
+                         status, num_sms, s);
+  if (fos)
+    return launch_stream(x, M, K, partial, n_partial, g_static, FakeOp<true>{yv, M, K}, nullptr, status, num_sms, s);
+  return launch_stream(x, M, K, partial, n_partial, g_static, FakeOp<false>{yv, M, K}, nullptr, status, num_sms, s);
+}
+
+cudaError_t launch_quantize_fused(const void* x, int64_t M, int64_t K, bool fos, uint32_t* ws, uint8_t* codes,
+                                  uint8_t* scales, float* g_out, uint8_t* choice, int* status, int num_sms,
+                                  cudaStream_t s) {
+  uint2* c = reinterpret_cast<uint2*>(codes);
+  if (fos) return launch_fused(x, M, K, ws, QuantOp<true>{c, scales, choice, M, K}, g_out, status, num_sms, s);
+  return launch_fused(x, M, K, ws, QuantOp<false>{c, scales, choice, M, K}, g_out, status, num_sms, s);
+}
+
+cudaError_t launch_fake_quant_fused(const void* x, int64_t M, int64_t K, bool fos, uint32_t* ws, void* y,
+                                    int* status, int num_sms, cudaStream_t s) {
+  uint4* yv = static_cast<uint4*>(y);
+  if (fos) return launch_fused(x, M, K, ws, FakeOp<true>{yv, M, K}, nullptr, status, num_sms, s);
+  return launch_fused(x, M, K, ws, FakeOp<false>{yv, M, K}, nullptr, status, num_sms, s);
 }
 
 cudaError_t launch_convert(const float* in, int64_t n, uint8_t* out, bool e4m3, int num_sms,

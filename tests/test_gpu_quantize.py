@@ -87,6 +87,52 @@ def test_quantize_zero_and_tiny_blocks(nv):
         assert_quantized_equal(q, oracle_quantized(bf16_np(xt), mode), 128, 256, check_choice=True)
 
 
+def _fma_choice(blocks: np.ndarray, g: np.float32) -> np.ndarray:
+    """four_over_six choice as a kernel that fused d*q into the subtraction
+    (one rounding of x - d*q) would take it: used only to find blocks whose
+    choice depends on the products being rounded separately."""
+    bmax = np.max(np.abs(blocks), axis=1)
+    errs = []
+    for mt in (6.0, 4.0):
+        sc = o.block_scale_codes(bmax, g, mt)
+        d = (np.float32(g) * o.e4m3_decode(sc).astype(np.float32)).astype(np.float32)
+        q = o.e2m1_encode(blocks * (np.float32(1) / d)[:, None])
+        # float64 holds x - d*q exactly here; one rounding to FP32 as an FMA does
+        df = (blocks.astype(np.float64) - d.astype(np.float64)[:, None] *
+              o.e2m1_decode(q).astype(np.float64)).astype(np.float32)
+        sq = df * df
+        e = np.zeros(len(blocks), np.float32)
+        for i in range(16):
+            e = e + sq[:, i]
+        errs.append(e)
+    return (errs[1] < errs[0]).astype(np.uint8)
+
+
+def test_four_over_six_near_ties_round_each_product(nv):
+    # Blocks whose M=4 / M=6 errors agree to the last few ULPs: the choice flips
+    # if any product of the error sum is fused with the following subtraction.
+    rng = np.random.default_rng(46)
+    amax = np.float32(87.5)
+    g = np.float32(amax / np.float32(2688.0))
+    t = np.clip(rng.standard_t(3, (1 << 19, 16)) * 0.5, -80.0, 80.0).astype(np.float32)
+    cand = bf16_np(inputs.to_bf16(t))
+    ref = o.quantize(cand, "four_over_six", g)["choice"][:, 0]
+    flips = np.nonzero(ref != _fma_choice(cand, g))[0]
+    assert flips.size >= 4, flips.size
+    picked = cand[flips[: 4 * (flips.size // 4)]]
+    top = np.zeros((4, 16), np.float32)
+    top[0, 0] = amax  # the tensor's maximum, so the dynamic g equals g
+    x = np.ascontiguousarray(np.concatenate([picked, cand[:256], top]).reshape(-1, 64))
+    assert o.global_scale(x)[0] == g
+    xt = torch.from_numpy(x).to(torch.bfloat16)
+    q = nv.quantize(xt.cuda(), "four_over_six", want_choice=True)
+    assert_quantized_equal(q, oracle_quantized(x, "four_over_six"), x.shape[0], 64, check_choice=True)
+    # the same blocks through fake-quant, whose output follows the choice
+    y = to_np(nv.fake_quant(xt.cuda(), "four_over_six").view(torch.int16))
+    y_ref = torch.from_numpy(o.fake_quant(x, "four_over_six")).to(torch.bfloat16).view(torch.int16).numpy()
+    np.testing.assert_array_equal(y, y_ref)
+
+
 def test_four_over_six_outlier_weights(nv):
     d = inputs.four_over_six_linear(0, M=16, N=1024, K=2048)
     w = d["w"]
