@@ -104,6 +104,13 @@ class ClockSampler:
             self.proc = None
         return self
 
+    def wait_first(self, timeout_s: float):
+        """Block until the first sample has arrived (nvidia-smi takes a moment to start)."""
+        t_end = time.time() + timeout_s
+        while self.proc is not None and not self.lines and time.time() < t_end:
+            time.sleep(0.01)
+        return self
+
     def _read(self):
         for line in self.proc.stdout:
             self.lines.append((time.time(), line.strip()))
@@ -261,14 +268,18 @@ def parity_gate(nv, x_dev, xq, wq, w_cpu_rows=None):
     return None
 
 
-def time_loop(fn, steps, warmup, flush_buf, stream, marks=0):
+def time_loop(fn, steps, warmup, flush_buf, stream, marks=0, launches=None):
     """Run warmup, then `steps` timed steps with the L2 flushed before each;
     per-step CUDA events on `stream` exclude the flush. fn(evs) records its own
-    intermediate events into evs (list of `marks` events)."""
+    intermediate events into evs (list of `marks` events). With `launches` (a
+    dict), launches["timed"] receives the library's kernel launches issued by
+    the timed steps."""
+    import qad_nvfp4_quantize_b200 as nv
     for _ in range(warmup):
         flush_l2(flush_buf)
         fn([torch.cuda.Event(enable_timing=True) for _ in range(marks)])
     torch.cuda.synchronize()
+    n0 = nv.kernel_launches()
     starts = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     ends = [torch.cuda.Event(enable_timing=True) for _ in range(steps)]
     mids = [[torch.cuda.Event(enable_timing=True) for _ in range(marks)] for _ in range(steps)]
@@ -278,6 +289,8 @@ def time_loop(fn, steps, warmup, flush_buf, stream, marks=0):
         fn(mids[i])
         ends[i].record(stream)
     torch.cuda.synchronize()
+    if launches is not None:
+        launches["timed"] = nv.kernel_launches() - n0
     total = [s.elapsed_time(e) for s, e in zip(starts, ends)]
     seg = []
     for i in range(steps):
@@ -396,10 +409,12 @@ def run_gpu(args, rank, world, local):
         nv.gemm(xq, wq, out=C)
 
     sampler = ClockSampler(local).start()
+    sampler.wait_first(3.0)
     barrier(world)
     torch.cuda.synchronize()
     t_wall0 = time.time()
-    total, seg = time_loop(step, args.steps, args.warmup, flush_buf, stream, marks=1)
+    launches = {}
+    total, seg = time_loop(step, args.steps, args.warmup, flush_buf, stream, marks=1, launches=launches)
     t_wall1 = time.time()
     barrier(world)
     torch.cuda.synchronize()
@@ -445,11 +460,12 @@ def run_gpu(args, rank, world, local):
             "roofline": roofline,
             "quantize": {"ms": quant_ms, "GB/s": quant_bytes / (quant_ms * 1e-3) / 1e9,
                          "frac_hbm": quant_bytes / (quant_ms * 1e-3) / 1e9 / peaks["hbm"],
-                         "algorithmic_bytes": quant_bytes, "peak_GB/s": peaks["hbm"]},
+                         "algorithmic_bytes": quant_bytes, "peak_GB/s": peaks["hbm"],
+                         "traffic": recorded_traffic("quantize_dense_mlp")},
             "gemm_ms": gemm_ms,
             "e2e": {"value": e2e_val, "unit": UNIT, "h2d_bytes_per_step": x.numel() * 2,
                     "d2h_bytes_per_step": C.numel() * 2, "ms_per_step": e2e_ms},
-            "gpu_launches": 3 * args.steps,
+            "gpu_launches": launches["timed"],
             "clocks": {"sm_mhz": clocks["sm_mhz"], "sm_max_mhz": clocks["sm_max_mhz"], "reasons": clocks["reasons"],
                        "samples": clocks["samples"]},
             "wall_s_timed_region": t_wall1 - t_wall0}
@@ -466,7 +482,7 @@ def run_gpu(args, rank, world, local):
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-rows", action="store_true", help="skip the per-row measurements")

@@ -254,6 +254,12 @@ nvfp4_status nvfp4_get_device_status(nvfp4_stream_t stream, int clear, nvfp4_sta
  * records NVFP4_ERR_TIMEOUT in the device status word. */
 nvfp4_status nvfp4_selftest_timeout(uint64_t timeout_ns, nvfp4_stream_t stream);
 
+/* Number of kernels this library has launched in the process so far, summed
+ * over all devices and threads (a host-side counter incremented at every
+ * launch; it counts launches issued, not completed). Diagnostic only: the
+ * method itself has no counterpart. Never fails. */
+uint64_t nvfp4_kernel_launches(void);
+
 #ifdef __cplusplus
 }
 #endif

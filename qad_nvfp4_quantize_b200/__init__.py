@@ -68,6 +68,7 @@ _SIGS = {
     "nvfp4_convert_e4m3": (I32, [P, I64, P, P]),
     "nvfp4_get_device_status": (I32, [P, I32, ctypes.POINTER(ctypes.c_int)]),
     "nvfp4_selftest_timeout": (I32, [U64, P]),
+    "nvfp4_kernel_launches": (U64, []),
 }
 
 
@@ -304,6 +305,11 @@ def device_status(clear: bool = True, device=None) -> int:
     v = ctypes.c_int(0)
     _check(lib().nvfp4_get_device_status(_stream(dev), int(clear), ctypes.byref(v)), "nvfp4_get_device_status")
     return v.value
+
+
+def kernel_launches() -> int:
+    """Kernels this library has launched in the process so far (nvfp4_kernel_launches)."""
+    return int(lib().nvfp4_kernel_launches())
 
 
 def selftest_timeout(timeout_ns: int, device=None) -> None:

@@ -1,5 +1,6 @@
 // C ABI entry points (include/nvfp4.h): argument validation, the sm_100
 // hardware gate, the device status word, and dispatch to the kernels.
+#include <atomic>
 #include <mutex>
 
 #include "common.cuh"
@@ -64,7 +65,11 @@ nvfp4_status run_amax(const void* x, int64_t n, void* ws, size_t ws_bytes, int n
   return NVFP4_OK;
 }
 
+std::atomic<uint64_t> g_launches{0};
+
 }  // namespace
+
+void nvfp4::note_launch() { g_launches.fetch_add(1, std::memory_order_relaxed); }
 
 int nvfp4::current_device_context(int* num_sms, int** status) {
   DeviceInfo* d;
@@ -212,6 +217,8 @@ nvfp4_status nvfp4_get_device_status(nvfp4_stream_t stream, int clear, nvfp4_sta
   *out = static_cast<nvfp4_status>(v);
   return NVFP4_OK;
 }
+
+uint64_t nvfp4_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
 nvfp4_status nvfp4_selftest_timeout(uint64_t timeout_ns, nvfp4_stream_t stream) {
   if (timeout_ns > 10000000000ull) return NVFP4_ERR_INVALID_ARG;  // at most 10 s

@@ -144,6 +144,7 @@ cudaError_t launch_gemm(const uint8_t* Aq, const uint8_t* As, const float* ga, c
   if (e != cudaSuccess) return e;
   const int tiles = p.m_tiles * p.n_tiles;
   const int grid = tiles < num_sms ? tiles : num_sms;
+  note_launch();
   nvf4_gemm_kernel<DenseProblem><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB, p, status, kGemmTimeoutNs);
   return cudaGetLastError();
 }

@@ -58,6 +58,10 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
 // status word (api.cu). Returns NVFP4_OK or the gate's error code.
 int current_device_context(int* num_sms, int** status);
 
+// Host-side count of kernel launches issued by the library (every launch
+// site calls note_launch() just before it launches).
+void note_launch();
+
 // Tensor-map encoder from the driver (resolved once through the runtime).
 CUresult encode_tensor_map_2d(CUtensorMap* map, const void* base, uint64_t inner_bytes,
                               uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner,

@@ -452,6 +452,7 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
     attr_err = cudaFuncSetAttribute(moe_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   });
   if (attr_err != cudaSuccess) return attr_err;
+  note_launch();
   moe_route_kernel<<<1, kRouteThreads, route_smem, s>>>(a.topk_ids, P, a.E, R, I32(L.counts), I32(L.offsets),
                                                          I32(L.row_pair), I32(L.tile_expert), I32(L.tile_count),
                                                          U32(L.amax_x), U32(L.amax_h), status);
@@ -462,6 +463,7 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
     int64_t blocks = (a.T + 7) / 8;
     if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
     if (blocks < 1) blocks = 1;
+    note_launch();
     moe_token_pass_kernel<<<(int)blocks, 256, 0, s>>>(static_cast<const uint4*>(a.x), a.T, a.H, a.topk_ids,
                                                        a.topk, a.E, U32(L.amax_x), reinterpret_cast<float4*>(a.out));
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -469,6 +471,7 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
 
   const int qgrid = num_sms * 8;
   // 3. gather + quantize x per expert
+  note_launch();
   moe_quantize_rows_kernel<true><<<qgrid, 256, 0, s>>>(
       static_cast<const uint4*>(a.x), a.H, a.topk, I32(L.row_pair), I32(L.tile_expert), I32(L.tile_count),
       U32(L.amax_x), a.E, U32(L.xq_codes), ws + L.xq_scales, F32(L.xq_g), status);
@@ -497,11 +500,13 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
     if ((e = prepare_moe_kernel<GateUpProblem>()) != cudaSuccess) return e;
     int64_t max_tiles = (R / 128) * p.n_tiles;
     const int grid = (int)(max_tiles < num_sms ? max_tiles : num_sms);
+    note_launch();
     nvf4_gemm_kernel<GateUpProblem><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB, p, status, kMoeTimeoutNs);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
 
   // 5. quantize h per expert
+  note_launch();
   moe_quantize_rows_kernel<false><<<qgrid, 256, 0, s>>>(
       reinterpret_cast<const uint4*>(ws + L.h), a.I, a.topk, I32(L.row_pair), I32(L.tile_expert),
       I32(L.tile_count), U32(L.amax_h), a.E, U32(L.hq_codes), ws + L.hq_scales, F32(L.hq_g), status);
@@ -532,6 +537,7 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
     if ((e = prepare_moe_kernel<DownProblem>()) != cudaSuccess) return e;
     int64_t max_tiles = (R / 128) * p.n_tiles;
     const int grid = (int)(max_tiles < num_sms ? max_tiles : num_sms);
+    note_launch();
     nvf4_gemm_kernel<DownProblem><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB, p, status, kMoeTimeoutNs);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }

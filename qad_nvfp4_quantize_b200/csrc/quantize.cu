@@ -650,6 +650,7 @@ int amax_partial_count(int64_t n, int num_sms) {
 
 cudaError_t launch_amax_partial(const void* x, int64_t n, uint32_t* partial, int n_partial,
                                 cudaStream_t s) {
+  note_launch();
   amax_partial_kernel<<<n_partial, kAmaxThreads, 0, s>>>(static_cast<const uint4*>(x), n / 8, partial);
   return cudaGetLastError();
 }
@@ -669,6 +670,7 @@ static cudaError_t launch_stream(const void* x, int64_t M, int64_t K, const uint
   if (chunks >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
   static const int occ = resident_blocks(stream_pass_kernel<Op>, kQThreads, 0);
   const int grid = grid_for(chunks, kQThreads / 32 * kUnroll, num_sms * (occ > 0 ? occ : 1));
+  note_launch();
   stream_pass_kernel<Op><<<grid, kQThreads, 0, s>>>(static_cast<const uint4*>(x), M, K, partial, n_partial, g_static,
                                                      op, g_out, status);
   return cudaGetLastError();
@@ -691,6 +693,7 @@ static cudaError_t launch_fused(const void* x, int64_t M, int64_t K, uint32_t* w
   uint64_t timeout_ns = kFusedTimeoutNs;
   void* args[] = {(void*)&xv, (void*)&M, (void*)&K, (void*)&partial, (void*)&bar, (void*)&op, (void*)&g_out,
                   (void*)&status, (void*)&timeout_ns};
+  note_launch();
   const cudaError_t e = cudaLaunchCooperativeKernel((const void*)fused_dynamic_kernel<Op>, dim3(num_sms),
                                                     dim3(kFusedThreads), args, kFusedSmem, s);
   if (e == cudaErrorCooperativeLaunchTooLarge) {
@@ -741,6 +744,7 @@ cudaError_t launch_fake_quant_fused(const void* x, int64_t M, int64_t K, bool fo
 cudaError_t launch_convert(const float* in, int64_t n, uint8_t* out, bool e4m3, int num_sms,
                            cudaStream_t s) {
   const int grid = grid_for(n, 256, num_sms * 8);
+  note_launch();
   if (e4m3)
     convert_e4m3_kernel<<<grid, 256, 0, s>>>(in, n, out);
   else
@@ -749,6 +753,7 @@ cudaError_t launch_convert(const float* in, int64_t n, uint8_t* out, bool e4m3, 
 }
 
 cudaError_t launch_selftest_timeout(uint64_t timeout_ns, int* status, cudaStream_t s) {
+  note_launch();
   selftest_timeout_kernel<<<1, 32, 0, s>>>(timeout_ns, status);
   return cudaGetLastError();
 }
