@@ -41,29 +41,39 @@ struct DenseProblem {
   // Columns [h*128, h*128+128) of the accumulator, 32 at a time.
   __device__ static constexpr uint32_t tmem_col(int h, int j) { return (uint32_t)(h * 128 + 32 * j); }
 
-  __device__ __forceinline__ void store(const TileJob& job, int q, int h, int lane,
-                                        const uint32_t (&acc)[4][32]) const {
-    const int row = job.m0 + q * 32 + lane;
-    if (row >= M) return;
+  // Epilogue of one warp (rows q*32.., columns h*128..): scale by ga*gb, round
+  // to BF16, and write 32 x 16 boxes through the warp's shared staging box with
+  // TMA stores (rows >= M and columns >= N are clipped by the tensor map). The
+  // staging box uses the 32-byte swizzle, so the 32 row writes of a warp fall
+  // on distinct shared-memory banks.
+  __device__ __forceinline__ void store(const TileJob& job, int q, int h, int lane, const uint32_t (&acc)[4][32],
+                                        uint8_t* stg, const CUtensorMap* tmC) const {
+    const int row0 = job.m0 + q * 32;
+    if (row0 >= M) return;
     const float alpha = __fmul_rn(*ga, *gb);
-    __nv_bfloat16* crow = C + (size_t)row * N;
+    const uint32_t sbase = smem_u32(stg);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = job.n0 + h * 128 + 32 * j;
+    for (int c0 = 0; c0 < 128; c0 += kEpiCols) {
+      const int n = job.n0 + h * 128 + c0;
+      if (n >= N) break;
+      if (lane == 0) bulk_wait_read_all();  // the previous box has left shared memory
+      __syncwarp();
 #pragma unroll
-      for (int c = 0; c < 32; c += 8) {
-        if (n + c < N) {
-          uint4 w;
-          w.x = f32x2_to_bf16x2(__fmul_rn(__uint_as_float(acc[j][c + 0]), alpha),
-                                __fmul_rn(__uint_as_float(acc[j][c + 1]), alpha));
-          w.y = f32x2_to_bf16x2(__fmul_rn(__uint_as_float(acc[j][c + 2]), alpha),
-                                __fmul_rn(__uint_as_float(acc[j][c + 3]), alpha));
-          w.z = f32x2_to_bf16x2(__fmul_rn(__uint_as_float(acc[j][c + 4]), alpha),
-                                __fmul_rn(__uint_as_float(acc[j][c + 5]), alpha));
-          w.w = f32x2_to_bf16x2(__fmul_rn(__uint_as_float(acc[j][c + 6]), alpha),
-                                __fmul_rn(__uint_as_float(acc[j][c + 7]), alpha));
-          *reinterpret_cast<uint4*>(crow + n + c) = w;
-        }
+      for (int ch = 0; ch < kEpiCols / 8; ++ch) {
+        const uint32_t* a = &acc[(c0 + ch * 8) / 32][(c0 + ch * 8) % 32];
+        uint4 w;
+        w.x = f32x2_to_bf16x2(__fmul_rn(__uint_as_float(a[0]), alpha), __fmul_rn(__uint_as_float(a[1]), alpha));
+        w.y = f32x2_to_bf16x2(__fmul_rn(__uint_as_float(a[2]), alpha), __fmul_rn(__uint_as_float(a[3]), alpha));
+        w.z = f32x2_to_bf16x2(__fmul_rn(__uint_as_float(a[4]), alpha), __fmul_rn(__uint_as_float(a[5]), alpha));
+        w.w = f32x2_to_bf16x2(__fmul_rn(__uint_as_float(a[6]), alpha), __fmul_rn(__uint_as_float(a[7]), alpha));
+        // 32-byte swizzle: 16-byte chunk index XOR bit 2 of the row
+        st_shared_v4(sbase + lane * (kEpiCols * 2) + ((ch ^ ((lane >> 2) & 1)) << 4), w);
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(tmC, stg, n, row0);
+        bulk_commit_group();
       }
     }
   }
@@ -106,6 +116,19 @@ CUresult encode_tensor_map_2d(CUtensorMap* map, const void* base, uint64_t inner
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
 }
 
+// Row-major BF16 [rows][cols] output written in 32-row x kEpiCols-column boxes
+// from a 32-byte-swizzled staging box. cols * 2 must be a multiple of 16.
+CUresult encode_store_map_bf16(CUtensorMap* map, void* base, uint64_t cols, uint64_t rows) {
+  EncodeTiledFn fn = get_encoder();
+  if (!fn) return CUDA_ERROR_NOT_FOUND;
+  const cuuint64_t dims[2] = {cols, rows};
+  const cuuint64_t strides[1] = {cols * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)kEpiCols, 32};
+  const cuuint32_t elem[2] = {1, 1};
+  return fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, base, dims, strides, box, elem, CU_TENSOR_MAP_INTERLEAVE_NONE,
+            CU_TENSOR_MAP_SWIZZLE_32B, CU_TENSOR_MAP_L2_PROMOTION_NONE, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+}
+
 template <class Prob>
 static cudaError_t prepare_kernel() {
   static std::once_flag once;
@@ -142,10 +165,12 @@ cudaError_t launch_gemm(const uint8_t* Aq, const uint8_t* As, const float* ga, c
   p.C = static_cast<__nv_bfloat16*>(C);
   cudaError_t e = prepare_kernel<DenseProblem>();
   if (e != cudaSuccess) return e;
+  CUtensorMap tmC;
+  if (encode_store_map_bf16(&tmC, C, (uint64_t)N, (uint64_t)M) != CUDA_SUCCESS) return cudaErrorInvalidValue;
   const int tiles = p.m_tiles * p.n_tiles;
   const int grid = tiles < num_sms ? tiles : num_sms;
   note_launch();
-  nvf4_gemm_kernel<DenseProblem><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB, p, status, kGemmTimeoutNs);
+  nvf4_gemm_kernel<DenseProblem><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB, tmC, p, status, kGemmTimeoutNs);
   return cudaGetLastError();
 }
 

@@ -14,7 +14,10 @@
 //               block-scaled MMAs (kind::mxf4nvf4, M=128, N=256, K=64);
 //   warps 2..9  epilogue: drain the 128 x 256 FP32 accumulator from tensor
 //               memory into registers, release it to the MMA warp, then scale,
-//               round and store (policy-specific).
+//               round and store (policy-specific; the dense store stages
+//               32 x 16 boxes in shared memory and writes them with TMA, so C
+//               leaves as whole 32-byte rows instead of 16-byte pieces of 32
+//               rows that would compete with the operand loads).
 // Tensor memory: columns [0,256) accumulator; from column 256 each pipeline
 // stage owns 48 columns of scales -- 16 for A (4 per MMA) then 32 for B (8 per
 // MMA) -- so the scale copy of one stage never overwrites columns that MMAs of
@@ -39,6 +42,8 @@ constexpr uint32_t kSFAtom = 512;              // 128 rows x 4 scales
 constexpr uint32_t kSFABytes = 4 * kSFAtom;
 constexpr uint32_t kSFBBytes = 8 * kSFAtom;
 constexpr int kGemmThreads = 320;
+constexpr int kEpiCols = 16;                   // output columns per TMA store box
+constexpr uint32_t kEpiBytes = 32 * kEpiCols * 2;  // one epilogue warp's BF16 staging box
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemSF = 256;         // first scale column
 constexpr uint32_t kTmemSFStage = 48;     // scale columns per stage
@@ -49,7 +54,8 @@ constexpr uint32_t kSmemA = 0;
 constexpr uint32_t kSmemB = kSmemA + kStages * kABytes;
 constexpr uint32_t kSmemSFA = kSmemB + kStages * kBBytes;
 constexpr uint32_t kSmemSFB = kSmemSFA + kStages * kSFABytes;
-constexpr uint32_t kSmemBar = kSmemSFB + kStages * kSFBBytes;
+constexpr uint32_t kSmemEpi = kSmemSFB + kStages * kSFBBytes;  // 8 warps x kEpiBytes
+constexpr uint32_t kSmemBar = kSmemEpi + 8 * kEpiBytes;
 constexpr uint32_t kNumBars = 2 * kStages + 3;   // full, empty, acc_full, acc_empty, drain
 constexpr uint32_t kSmemMisc = kSmemBar + kNumBars * 8;
 constexpr uint32_t kGemmSmemBytes = kSmemMisc + 16 + 1024;  // + alignment slack
@@ -75,7 +81,8 @@ struct TileJob {
 template <class Prob>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     nvf4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
-                     const Prob prob, int* status, uint64_t timeout_ns) {
+                     const __grid_constant__ CUtensorMap tmC, const Prob prob, int* status,
+                     uint64_t timeout_ns) {
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemBar);
@@ -250,9 +257,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty);
       const TileJob job = prob.job(t);
-      prob.store(job, q, h, lane, acc);
+      prob.store(job, q, h, lane, acc, smem + kSmemEpi + (warp - 2) * kEpiBytes, &tmC);
       acc_phase ^= 1;
     }
+    if (lane == 0) bulk_wait_all();  // TMA stores of C complete before the CTA exits
   }
 
   tc_fence_before();

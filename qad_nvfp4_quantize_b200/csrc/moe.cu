@@ -322,7 +322,7 @@ struct GateUpProblem {
   }
 
   __device__ __forceinline__ void store(const TileJob& job, int q, int hh, int lane,
-                                        const uint32_t (&acc)[4][32]) const {
+                                        const uint32_t (&acc)[4][32], uint8_t*, const CUtensorMap*) const {
     const int row = job.m0 + q * 32 + lane;
     const float alpha = __fmul_rn(ga[job.expert], gb[job.expert]);
     __nv_bfloat16* hrow = h + (size_t)row * I + job.n0 + hh * 64;
@@ -398,7 +398,7 @@ struct DownProblem {
   __device__ static constexpr uint32_t tmem_col(int h, int j) { return (uint32_t)(h * 128 + 32 * j); }
 
   __device__ __forceinline__ void store(const TileJob& job, int q, int hh, int lane,
-                                        const uint32_t (&acc)[4][32]) const {
+                                        const uint32_t (&acc)[4][32], uint8_t*, const CUtensorMap*) const {
     const int row = job.m0 + q * 32 + lane;
     const int32_t pair = row_pair[row];
     if (pair < 0) return;
@@ -501,7 +501,8 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
     int64_t max_tiles = (R / 128) * p.n_tiles;
     const int grid = (int)(max_tiles < num_sms ? max_tiles : num_sms);
     note_launch();
-    nvf4_gemm_kernel<GateUpProblem><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB, p, status, kMoeTimeoutNs);
+    nvf4_gemm_kernel<GateUpProblem><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB, tmA /* output map unused: direct stores */, p, status,
+                                                                                 kMoeTimeoutNs);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
 
@@ -538,7 +539,8 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
     int64_t max_tiles = (R / 128) * p.n_tiles;
     const int grid = (int)(max_tiles < num_sms ? max_tiles : num_sms);
     note_launch();
-    nvf4_gemm_kernel<DownProblem><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB, p, status, kMoeTimeoutNs);
+    nvf4_gemm_kernel<DownProblem><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB, tmA /* output map unused: direct stores */, p, status,
+                                                                                 kMoeTimeoutNs);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;

@@ -34,6 +34,20 @@ __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   return v;
 }
 
+// Lane-wise magnitude maximum of two BF16 pairs: |result| = max(|a|, |b|) per
+// half (the sign bits hold the XOR of the inputs' signs and are masked off by
+// every user); NaN in either input gives NaN.
+__device__ __forceinline__ uint32_t bmax2(uint32_t a, uint32_t b) {
+  uint32_t m;
+  asm("max.NaN.xorsign.abs.bf16x2 %0, %1, %2;" : "=r"(m) : "r"(a), "r"(b));
+  return m;
+}
+
+// Larger of the two 16-bit magnitudes (bits & 0x7FFF) of a BF16 pair.
+__device__ __forceinline__ uint32_t mag_max_halves(uint32_t m2) {
+  return max(m2 & 0x7FFFu, (m2 >> 16) & 0x7FFFu);
+}
+
 // ----------------------------------------------------------------------------
 // amax, pass 1: per-CTA maximum of |x| as a BF16 magnitude (bits & 0x7FFF).
 // Magnitudes of finite BF16 values order like their bit patterns; anything
@@ -64,7 +78,7 @@ __global__ void __launch_bounds__(kAmaxThreads, 8) amax_partial_kernel(const uin
     m2 = __vmaxu2(m2, v.z & 0x7FFF7FFFu);
     m2 = __vmaxu2(m2, v.w & 0x7FFF7FFFu);
   }
-  uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+  uint32_t m = mag_max_halves(m2);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFull, m, o));
   __shared__ uint32_t red[kAmaxThreads / 32];
@@ -135,12 +149,13 @@ struct Chunk {
   int64_t vec;        // 16-byte vector index of the block's first 8 elements
 };
 
-__device__ __forceinline__ Chunk chunk_at(int64_t ch, int32_t cpr, int64_t K, int lane) {
+__device__ __forceinline__ Chunk chunk_at(int64_t ch, int32_t cpr, uint64_t cpr_magic, int64_t K, int lane) {
   Chunk c;
-  const uint32_t chu = (uint32_t)ch;  // the launcher keeps chunk counts below 2^31
-  const uint32_t r = chu / (uint32_t)cpr;
-  c.row = r;
-  c.col = (int32_t)(chu - r * (uint32_t)cpr) * 512 + lane * 16;
+  // ch / cpr by multiplication with cpr_magic = ceil(2^64 / cpr) (exact for
+  // ch * cpr < 2^64; division by an invariant integer, Granlund & Montgomery 1994)
+  const uint64_t r = cpr == 1 ? (uint64_t)ch : __umul64hi((uint64_t)ch, cpr_magic);
+  c.row = (int64_t)r;
+  c.col = (int32_t)((uint64_t)ch - r * (uint64_t)cpr) * 512 + lane * 16;
   c.valid = c.col < K;
   c.vec = (c.row * K + c.col) >> 3;
   return c;
@@ -172,23 +187,49 @@ __device__ __forceinline__ f32x2 sub2(f32x2 a, f32x2 b) {
 __device__ __forceinline__ f32x2 bf16x2_unpack(uint32_t w) {
   return pack2(__uint_as_float(w << 16), __uint_as_float(w & 0xFFFF0000u));
 }
-// FP32 pair -> one byte of two E2M1 codes (low element in the low nibble).
-__device__ __forceinline__ uint32_t e2m1x2(f32x2 v) {
-  float lo, hi;
-  unpack2(v, lo, hi);
-  uint16_t out;
-  asm("{\n\t.reg .b8 q;\n\tcvt.rn.satfinite.e2m1x2.f32 q, %2, %1;\n\tcvt.u16.u8 %0, q;\n\t}"
-      : "=h"(out) : "f"(lo), "f"(hi));
-  return out & 0xFFu;
+// Four FP32 pairs -> one word of eight E2M1 codes (element 2j in the low
+// nibble of byte j). cvt.e2m1x2 puts its first source in the high nibble.
+__device__ __forceinline__ uint32_t e2m1_pack4(f32x2 v0, f32x2 v1, f32x2 v2, f32x2 v3) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 q0, q1, q2, q3;\n\t.reg .f32 a0, a1, a2, a3, a4, a5, a6, a7;\n\t"
+      "mov.b64 {a0, a1}, %1;\n\tmov.b64 {a2, a3}, %2;\n\tmov.b64 {a4, a5}, %3;\n\tmov.b64 {a6, a7}, %4;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q0, a1, a0;\n\tcvt.rn.satfinite.e2m1x2.f32 q1, a3, a2;\n\t"
+      "cvt.rn.satfinite.e2m1x2.f32 q2, a5, a4;\n\tcvt.rn.satfinite.e2m1x2.f32 q3, a7, a6;\n\t"
+      "mov.b32 %0, {q0, q1, q2, q3};\n\t}"
+      : "=r"(out)
+      : "l"(v0), "l"(v1), "l"(v2), "l"(v3));
+  return out;
 }
-// Byte of two E2M1 codes -> their two values as FP32 (exact, through f16x2).
-__device__ __forceinline__ f32x2 e2m1x2_value(uint32_t byte) {
+
+// Byte of two E2M1 codes (low bits of `byte`) -> their values as an FP32 pair
+// (exact, through the hardware E2M1 -> f16x2 conversion; low nibble -> low
+// half). The byte is narrowed with cvt.u8 on purpose: unpacking a 32-bit word
+// into four 8-bit registers with one vector mov did not yield bytes 2 and 3.
+__device__ __forceinline__ f32x2 e2m1_byte_value(uint32_t byte) {
   float lo, hi;
-  asm("{\n\t.reg .b8 t;\n\t.reg .b32 h2;\n\t.reg .b16 a, b;\n\t"
-      "cvt.u8.u32 t, %2;\n\tcvt.rn.f16x2.e2m1x2 h2, t;\n\t"
-      "mov.b32 {a, b}, h2;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
-      : "=f"(lo), "=f"(hi) : "r"(byte));
+  asm("{\n\t.reg .b8 t;\n\t.reg .b32 h;\n\t.reg .b16 a, b;\n\t"
+      "cvt.u8.u32 t, %2;\n\tcvt.rn.f16x2.e2m1x2 h, t;\n\t"
+      "mov.b32 {a, b}, h;\n\tcvt.f32.f16 %0, a;\n\tcvt.f32.f16 %1, b;\n\t}"
+      : "=f"(lo), "=f"(hi)
+      : "r"(byte));
   return pack2(lo, hi);
+}
+
+// One word of eight E2M1 codes -> their values as four FP32 pairs.
+__device__ __forceinline__ void e2m1_unpack4(uint32_t w, f32x2* v) {
+#pragma unroll
+  for (int j = 0; j < 4; ++j) v[j] = e2m1_byte_value(w >> (8 * j));
+}
+
+// Value of an E4M3 scale code (exact, through the hardware E4M3 -> f16x2
+// conversion; the code sits in both bytes so either half holds it).
+__device__ __forceinline__ float scale_value(uint32_t code) {
+  float v;
+  asm("{\n\t.reg .b16 t, a, b;\n\t.reg .b32 h;\n\tcvt.u16.u32 t, %1;\n\t"
+      "cvt.rn.f16x2.e4m3x2 h, t;\n\tmov.b32 {a, b}, h;\n\tcvt.f32.f16 %0, a;\n\t}"
+      : "=f"(v)
+      : "r"(code * 0x101u));
+  return v;
 }
 
 // A lane's 16-element block as 8 raw BF16 words.
@@ -206,12 +247,12 @@ __device__ __forceinline__ void load_raw16(const uint4* x, int64_t vec, bool val
   r.w[4] = b.x; r.w[5] = b.y; r.w[6] = b.z; r.w[7] = b.w;
 }
 
-// max |x| of the block (BF16 magnitudes order like their bit patterns).
+// max |x| of the block as an FP32 value.
 __device__ __forceinline__ float block_absmax(const Raw16& r) {
-  uint32_t m2 = 0;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) m2 = __vmaxu2(m2, r.w[i] & 0x7FFF7FFFu);
-  return __uint_as_float(max(m2 & 0xFFFFu, m2 >> 16) << 16);
+  uint32_t m = bmax2(bmax2(bmax2(r.w[0], r.w[1]), bmax2(r.w[2], r.w[3])),
+                     bmax2(bmax2(r.w[4], r.w[5]), bmax2(r.w[6], r.w[7])));
+  m = bmax2(m, __byte_perm(m, 0, 0x1032));  // both halves now hold the maximum
+  return __uint_as_float((m & 0x7FFFu) << 16);
 }
 
 // One 16-element block: scale code, packed codes (two 32-bit words, element
@@ -227,29 +268,34 @@ struct Block {
 template <bool kDeq, bool kErr>
 __device__ __forceinline__ void quantize_block(const Raw16& raw, float bmax, float g, float mt, Block& b) {
   b.sc = block_scale_code(bmax, g, mt);
-  const float d = __fmul_rn(g, e4m3_value(b.sc));
+  const float d = __fmul_rn(g, scale_value(b.sc));
   const float r = __frcp_rn(d);
   const f32x2 rr = pack2(r, r);
-  uint32_t bytes[8];
+  f32x2 sv[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) bytes[i] = e2m1x2(mul2(bf16x2_unpack(raw.w[i]), rr));
-  b.q0 = bytes[0] | (bytes[1] << 8) | (bytes[2] << 16) | (bytes[3] << 24);
-  b.q1 = bytes[4] | (bytes[5] << 8) | (bytes[6] << 16) | (bytes[7] << 24);
-  if (kErr) {
-    // Scalar products here: with a packed multiply feeding the packed
-    // subtraction below, the compiler was seen to fuse the two into one
-    // fused multiply-add (one rounding of x - d*q where the method rounds
-    // d*q first), which flips near-tie four_over_six choices.
+  for (int i = 0; i < 8; ++i) sv[i] = mul2(bf16x2_unpack(raw.w[i]), rr);
+  b.q0 = e2m1_pack4(sv[0], sv[1], sv[2], sv[3]);
+  b.q1 = e2m1_pack4(sv[4], sv[5], sv[6], sv[7]);
+  if (kDeq || kErr) {
+    f32x2 v[8];
+    e2m1_unpack4(b.q0, v);
+    e2m1_unpack4(b.q1, v + 4);
+    if (kErr) {
+      // Scalar products here: with a packed multiply feeding the packed
+      // subtraction below, the compiler was seen to fuse the two into one
+      // fused multiply-add (one rounding of x - d*q where the method rounds
+      // d*q first), which flips near-tie four_over_six choices.
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float lo, hi;
-      unpack2(e2m1x2_value(bytes[i]), lo, hi);
-      b.deq[i] = pack2(__fmul_rn(d, lo), __fmul_rn(d, hi));
+      for (int i = 0; i < 8; ++i) {
+        float lo, hi;
+        unpack2(v[i], lo, hi);
+        b.deq[i] = pack2(__fmul_rn(d, lo), __fmul_rn(d, hi));
+      }
+    } else {
+      const f32x2 dd = pack2(d, d);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) b.deq[i] = mul2(dd, v[i]);
     }
-  } else if (kDeq) {
-    const f32x2 dd = pack2(d, d);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) b.deq[i] = mul2(dd, e2m1x2_value(bytes[i]));
   }
   if (kErr) {
     float acc = 0.0f;
@@ -265,15 +311,6 @@ __device__ __forceinline__ void quantize_block(const Raw16& raw, float bmax, flo
   } else {
     b.err = 0.0f;
   }
-}
-
-// Gather the scale codes of the 4 blocks of a 64-element group onto the
-// group's first lane (lanes 4c .. 4c+3 hold blocks 4c .. 4c+3).
-__device__ __forceinline__ uint32_t gather_group_scales(uint32_t sc) {
-  const uint32_t s1 = __shfl_down_sync(kFull, sc, 1);
-  const uint32_t s2 = __shfl_down_sync(kFull, sc, 2);
-  const uint32_t s3 = __shfl_down_sync(kFull, sc, 3);
-  return sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
 }
 
 // Zero the scale bytes of the padding rows [M, ceil128(M)).
@@ -315,11 +352,10 @@ struct QuantOp {
         q1 = b4.q1;
       }
     }
-    const uint32_t group = gather_group_scales(sc);
+    (void)lane;
     if (c.valid) {
       codes[c.vec >> 1] = make_uint2(q0, q1);
-      if ((lane & 3) == 0)
-        *reinterpret_cast<uint32_t*>(scales + scale_offset(c.row, c.col >> 4, K >> 6)) = group;
+      scales[scale_offset(c.row, c.col >> 4, K >> 6)] = (uint8_t)sc;  // 4 lanes fill one 4-byte group
       if (kFos && choice) choice[c.vec >> 1] = (uint8_t)pick4;
     }
   }
@@ -382,12 +418,16 @@ struct FrozenFakeOp {
   __device__ __forceinline__ void operator()(const Raw16& v, const Chunk& c, float g, int lane) const {
     (void)lane;
     const uint32_t sc = c.valid ? scales_frozen[scale_offset(c.row, c.col >> 4, K >> 6)] : 1u;
-    const float d = __fmul_rn(g, e4m3_value(sc));
+    const float d = __fmul_rn(g, scale_value(sc));
     const float r = __frcp_rn(d);
     const f32x2 rr = pack2(r, r), dd = pack2(d, d);
-    f32x2 out[8];
+    f32x2 sv[8], out[8];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) out[i] = mul2(dd, e2m1x2_value(e2m1x2(mul2(bf16x2_unpack(v.w[i]), rr))));
+    for (int i = 0; i < 8; ++i) sv[i] = mul2(bf16x2_unpack(v.w[i]), rr);
+    e2m1_unpack4(e2m1_pack4(sv[0], sv[1], sv[2], sv[3]), out);
+    e2m1_unpack4(e2m1_pack4(sv[4], sv[5], sv[6], sv[7]), out + 4);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) out[i] = mul2(dd, out[i]);
     FakeOp<false>::store_bf16x16(y, c, out);
   }
   __device__ __forceinline__ void finish() const {}
@@ -401,7 +441,8 @@ template <class Op>
 __global__ void __launch_bounds__(kQThreads) stream_pass_kernel(const uint4* __restrict__ x, int64_t M, int64_t K,
                                                                  const uint32_t* __restrict__ partial, int n_partial,
                                                                  const float* __restrict__ g_static, Op op,
-                                                                 float* __restrict__ g_out, int* status) {
+                                                                 float* __restrict__ g_out, int* status,
+                                                                 uint64_t cpr_magic) {
   bool bad;
   const float g = resolve_global_scale(partial, n_partial, g_static, &bad);
   if (blockIdx.x == 0 && threadIdx.x == 0) {
@@ -420,7 +461,7 @@ __global__ void __launch_bounds__(kQThreads) stream_pass_kernel(const uint4* __r
     Chunk cc[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      cc[u] = chunk_at(ch0 + u * nwarps, cpr, K, lane);
+      cc[u] = chunk_at(ch0 + u * nwarps, cpr, cpr_magic, K, lane);
       load_raw16(x, cc[u].vec, cc[u].valid && ch0 + u * nwarps < n_chunks, vv[u]);
     }
 #pragma unroll
@@ -486,7 +527,7 @@ template <class Op>
 __global__ void __launch_bounds__(kFusedThreads, 1) fused_dynamic_kernel(const uint4* __restrict__ x, int64_t M,
                                                                            int64_t K, uint32_t* partial, uint32_t* bar,
                                                                            Op op, float* g_out, int* status,
-                                                                           uint64_t timeout_ns) {
+                                                                           uint64_t timeout_ns, uint64_t cpr_magic) {
   extern __shared__ uint4 keep[];
   __shared__ uint32_t red[kFusedWarps];
   __shared__ float s_g;
@@ -509,7 +550,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_dynamic_kernel(const u
       const int64_t ch = base + u * kFusedWarps;
       a[u] = b[u] = make_uint4(0, 0, 0, 0);
       if (ch < hi) {
-        const Chunk c = chunk_at(ch, cpr, K, lane);
+        const Chunk c = chunk_at(ch, cpr, cpr_magic, K, lane);
         if (c.valid) {
           a[u] = ld_stream(x + c.vec);
           b[u] = ld_stream(x + c.vec + 1);
@@ -518,14 +559,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_dynamic_kernel(const u
     }
 #pragma unroll
     for (int u = 0; u < kFusedUnroll; ++u) {
-      m2 = __vmaxu2(m2, a[u].x & 0x7FFF7FFFu);
-      m2 = __vmaxu2(m2, a[u].y & 0x7FFF7FFFu);
-      m2 = __vmaxu2(m2, a[u].z & 0x7FFF7FFFu);
-      m2 = __vmaxu2(m2, a[u].w & 0x7FFF7FFFu);
-      m2 = __vmaxu2(m2, b[u].x & 0x7FFF7FFFu);
-      m2 = __vmaxu2(m2, b[u].y & 0x7FFF7FFFu);
-      m2 = __vmaxu2(m2, b[u].z & 0x7FFF7FFFu);
-      m2 = __vmaxu2(m2, b[u].w & 0x7FFF7FFFu);
+      m2 = bmax2(m2, bmax2(bmax2(bmax2(a[u].x, a[u].y), bmax2(a[u].z, a[u].w)),
+                           bmax2(bmax2(b[u].x, b[u].y), bmax2(b[u].z, b[u].w))));
       const int64_t k = base + u * kFusedWarps - lo;
       if (k < nkeep) {  // lane-contiguous halves: conflict-free 512-byte rows
         keep[k * 64 + lane] = a[u];
@@ -533,7 +568,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_dynamic_kernel(const u
       }
     }
   }
-  uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+  uint32_t m = mag_max_halves(m2);
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFull, m, o));
   if (lane == 0) red[warp] = m;
@@ -580,7 +615,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_dynamic_kernel(const u
     for (int u = 0; u < kFusedUnroll; ++u) {
       const int64_t ch = top - u * kFusedWarps;
       uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
-      cc[u] = chunk_at(ch >= lo ? ch : lo, cpr, K, lane);
+      cc[u] = chunk_at(ch >= lo ? ch : lo, cpr, cpr_magic, K, lane);
       if (ch >= lo && cc[u].valid) {
         const int64_t k = ch - lo;
         if (k < nkeep) {
@@ -636,6 +671,13 @@ __global__ void selftest_timeout_kernel(uint64_t timeout_ns, int* status) {
 // ----------------------------------------------------------------------------
 // Host launchers.
 // ----------------------------------------------------------------------------
+// ceil(2^64 / cpr) for the row division of chunk indices (cpr = chunks per
+// row); unused when cpr == 1.
+static uint64_t chunk_magic(int64_t K) {
+  const uint64_t cpr = (uint64_t)((K + 511) / 512);
+  return cpr > 1 ? ~uint64_t(0) / cpr + 1 : 0;
+}
+
 static int grid_for(int64_t work_items, int per_block, int max_blocks) {
   int64_t b = (work_items + per_block - 1) / per_block;
   if (b < 1) b = 1;
@@ -672,7 +714,7 @@ static cudaError_t launch_stream(const void* x, int64_t M, int64_t K, const uint
   const int grid = grid_for(chunks, kQThreads / 32 * kUnroll, num_sms * (occ > 0 ? occ : 1));
   note_launch();
   stream_pass_kernel<Op><<<grid, kQThreads, 0, s>>>(static_cast<const uint4*>(x), M, K, partial, n_partial, g_static,
-                                                     op, g_out, status);
+                                                     op, g_out, status, chunk_magic(K));
   return cudaGetLastError();
 }
 
@@ -691,8 +733,9 @@ static cudaError_t launch_fused(const void* x, int64_t M, int64_t K, uint32_t* w
   uint32_t* partial = ws;
   uint32_t* bar = ws + kMaxPartials;
   uint64_t timeout_ns = kFusedTimeoutNs;
+  uint64_t magic = chunk_magic(K);
   void* args[] = {(void*)&xv, (void*)&M, (void*)&K, (void*)&partial, (void*)&bar, (void*)&op, (void*)&g_out,
-                  (void*)&status, (void*)&timeout_ns};
+                  (void*)&status, (void*)&timeout_ns, (void*)&magic};
   note_launch();
   const cudaError_t e = cudaLaunchCooperativeKernel((const void*)fused_dynamic_kernel<Op>, dim3(num_sms),
                                                     dim3(kFusedThreads), args, kFusedSmem, s);

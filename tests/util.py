@@ -44,14 +44,15 @@ def tiled(scales: np.ndarray) -> np.ndarray:
 
 
 def assert_quantized_equal(gpu, ref, rows, K, check_choice=False):
+    assert to_np(gpu.g)[0] == np.float32(ref["g"]), ("global scale", to_np(gpu.g)[0], ref["g"])
     codes = to_np(gpu.codes)
     mism = np.nonzero(codes != ref["codes"])
     assert mism[0].size == 0, f"{mism[0].size} code bytes differ, first at {mism[0][0]},{mism[1][0]}: " \
-                              f"gpu {codes[mism][0]:#x} oracle {ref['codes'][mism][0]:#x}"
+                              f"gpu {codes[mism][0]:#x} oracle {ref['codes'][mism][0]:#x}; first scale bytes " \
+                              f"gpu {to_np(gpu.scales)[:8].tolist()} oracle {ref['scales'][:8].tolist()}"
     sc = to_np(gpu.scales)[: ref["scales"].size]
     bad = np.nonzero(sc != ref["scales"])[0]
     assert bad.size == 0, f"{bad.size} scale bytes differ, first at byte {bad[0]}"
-    assert to_np(gpu.g)[0] == np.float32(ref["g"]), (to_np(gpu.g)[0], ref["g"])
     if check_choice:
         assert np.array_equal(to_np(gpu.choice), ref["choice"])
 
