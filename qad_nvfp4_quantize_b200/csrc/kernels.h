@@ -9,6 +9,13 @@ namespace nvfp4 {
 
 constexpr int kMaxPartials = 1024;  // amax pass-1 partial slots in a workspace
 
+// ceil(2^64 / cpr) for the row division of 512-element chunk indices (cpr =
+// chunks per row of K elements); unused (0) when cpr == 1.
+inline uint64_t chunk_magic(int64_t K) {
+  const uint64_t cpr = (uint64_t)((K + 511) / 512);
+  return cpr > 1 ? ~uint64_t(0) / cpr + 1 : 0;
+}
+
 int amax_partial_count(int64_t n, int num_sms);
 cudaError_t launch_amax_partial(const void* x, int64_t n, uint32_t* partial, int n_partial,
                                 cudaStream_t s);

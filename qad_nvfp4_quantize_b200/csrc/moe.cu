@@ -23,6 +23,7 @@
 //                and adds into out[token] in FP32 (vector atomics).
 #include <mutex>
 
+#include "block_math.cuh"
 #include "gemm_kernel.cuh"
 #include "kernels.h"
 
@@ -36,17 +37,14 @@ int64_t align256(int64_t v) { return (v + 255) & ~int64_t(255); }
 
 int64_t scale_bytes_(int64_t rows, int64_t K) { return ((rows + 127) / 128) * (K / 64) * 512; }
 
-// Byte offset of (row, block column c) in the tiled scale layout.
-__device__ __forceinline__ int64_t sf_offset(int64_t row, int64_t c, int64_t kgroups) {
-  return (((row >> 7) * kgroups + (c >> 2)) << 9) + ((row & 31) << 4) + (((row >> 5) & 3) << 2) + (c & 3);
-}
-
 }  // namespace
+
+constexpr int kRouteCtasMax = 128;  // routing CTAs (each owns a contiguous pair range)
 
 // Workspace layout (all regions 256-byte aligned).
 struct MoeLayout {
   int64_t R, P;
-  int64_t counts, offsets, cursor, row_pair, tile_expert, tile_count, amax_x, amax_h;
+  int64_t counts, offsets, cursor, row_pair, tile_expert, tile_count, amax_x, amax_h, cta_count, cta_base;
   int64_t xq_codes, xq_scales, xq_g, h, hq_codes, hq_scales, hq_g, total;
 };
 
@@ -73,6 +71,8 @@ static MoeLayout moe_layout(int64_t T, int64_t H, int64_t I, int E, int topk) {
   L.tile_count = take(4);
   L.amax_x = take(4 * (int64_t)E);
   L.amax_h = take(4 * (int64_t)E);
+  L.cta_count = take(4 * (int64_t)kRouteCtasMax * E);
+  L.cta_base = take(4 * (int64_t)kRouteCtasMax * E);
   L.xq_codes = take(L.R * H / 2);
   L.xq_scales = take(scale_bytes_(L.R, H));
   L.xq_g = take(4 * (int64_t)E);
@@ -85,86 +85,137 @@ static MoeLayout moe_layout(int64_t T, int64_t H, int64_t I, int E, int topk) {
 }
 
 // ----------------------------------------------------------------------------
-// 1. Routing: one CTA of 1024 threads (32 warps). Warp w owns the contiguous
-// pair range [w*P/32, (w+1)*P/32); per-warp histograms give each warp its base
-// position inside every expert segment, and inside a warp pairs are ranked
-// with __match_any_sync, so the sort is stable (increasing pair index within
-// an expert, as a counting sort).
+// 1. Routing: a stable counting sort of the P = T*topk pairs by expert, in
+// three launches. G routing CTAs each own the contiguous pair range
+// [c*P/G, (c+1)*P/G).
+//   count  per-CTA expert histograms -> cta_count[c][e]
+//   scan   one CTA: per expert, exclusive prefix over CTAs -> cta_base[c][e],
+//          totals -> counts, 128-padded segment offsets, m-tile -> expert
+//          table, pad rows of row_pair = -1, per-expert amax slots zeroed
+//   place  each CTA ranks its pairs again: per-warp histograms give each
+//          warp its base inside every expert segment, and within a warp pairs
+//          are ranked with __match_any_sync, so the order inside an expert is
+//          increasing pair index (stable).
 // ----------------------------------------------------------------------------
-constexpr int kRouteThreads = 1024;
+constexpr int kRouteThreads = 256;
 constexpr int kRouteWarps = kRouteThreads / 32;
 
-__global__ void __launch_bounds__(kRouteThreads, 1) moe_route_kernel(
-    const int32_t* __restrict__ topk_ids, int64_t P, int E, int64_t R, int32_t* __restrict__ counts,
-    int32_t* __restrict__ offsets, int32_t* __restrict__ row_pair, int32_t* __restrict__ tile_expert,
-    int32_t* __restrict__ tile_count, uint32_t* __restrict__ amax_x, uint32_t* __restrict__ amax_h,
-    int* status) {
-  extern __shared__ int32_t sh[];
-  int32_t* wcount = sh;                           // [kRouteWarps][E]
-  int32_t* seg = sh + kRouteWarps * E;            // [E+1] padded offsets
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < kRouteWarps * E; i += blockDim.x) wcount[i] = 0;
-  for (int64_t i = threadIdx.x; i < R; i += blockDim.x) row_pair[i] = -1;
-  __syncthreads();
+__device__ __forceinline__ void route_range(int64_t P, int G, int c, int64_t& lo, int64_t& hi) {
+  lo = P * c / G;
+  hi = P * (c + 1) / G;
+}
 
-  const int64_t lo = P * warp / kRouteWarps, hi = P * (warp + 1) / kRouteWarps;
+__global__ void __launch_bounds__(kRouteThreads) moe_route_count_kernel(const int32_t* __restrict__ topk_ids,
+                                                                         int64_t P, int E,
+                                                                         int32_t* __restrict__ cta_count,
+                                                                         int* status) {
+  extern __shared__ int32_t hist[];  // [E]
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  int64_t lo, hi;
+  route_range(P, gridDim.x, blockIdx.x, lo, hi);
   bool bad = false;
-  for (int64_t p = lo + lane; p < hi; p += 32) {
+  for (int64_t p = lo + threadIdx.x; p < hi; p += blockDim.x) {
     const int e = topk_ids[p];
     if (e < 0 || e >= E) {
       bad = true;
       continue;
     }
-    atomicAdd(&wcount[warp * E + e], 1);
+    atomicAdd(&hist[e], 1);
   }
   if (bad) record_status(status, NVFP4_ERR_INVALID_ARG);
   __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cta_count[(int64_t)blockIdx.x * E + e] = hist[e];
+}
 
-  // per expert: total count, padded segment size; exclusive scan over experts
-  // (thread e handles expert e; E <= 1024) and per-warp bases.
+constexpr int kScanThreads = 1024;
+
+__global__ void __launch_bounds__(kScanThreads, 1) moe_route_scan_kernel(
+    const int32_t* __restrict__ cta_count, int G, int E, int32_t* __restrict__ cta_base,
+    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ row_pair,
+    int32_t* __restrict__ tile_expert, int32_t* __restrict__ tile_count, uint32_t* __restrict__ amax_x,
+    uint32_t* __restrict__ amax_h) {
+  __shared__ int32_t seg[kScanThreads + 1];   // padded segment sizes, then offsets
+  __shared__ int32_t wsum[kScanThreads / 32];
+  const int e = threadIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int32_t total = 0;
-  if (threadIdx.x < E) {
-    const int e = threadIdx.x;
-    for (int w = 0; w < kRouteWarps; ++w) {
-      const int32_t c = wcount[w * E + e];
-      wcount[w * E + e] = total;  // exclusive prefix over warps
-      total += c;
+  if (e < E) {
+    for (int c = 0; c < G; ++c) {
+      const int32_t v = cta_count[(int64_t)c * E + e];
+      cta_base[(int64_t)c * E + e] = total;
+      total += v;
     }
     counts[e] = total;
-    seg[e] = (total + 127) & ~127;
-  }
-  __syncthreads();
-  if (threadIdx.x == 0) {
-    int32_t run = 0;
-    for (int e = 0; e < E; ++e) {
-      const int32_t sz = seg[e];
-      seg[e] = run;
-      run += sz;
-    }
-    seg[E] = run;
-    *tile_count = run / 128;
-  }
-  __syncthreads();
-  for (int e = threadIdx.x; e <= E; e += blockDim.x) offsets[e] = seg[e];
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
     amax_x[e] = 0u;
     amax_h[e] = 0u;
-    const int32_t t0 = seg[e] / 128, t1 = seg[e + 1] / 128;
-    for (int t = t0; t < t1; ++t) tile_expert[t] = e;
   }
-  // placement, in pair order within each warp's range
-  for (int64_t base = lo; base < hi; base += 32) {
+  const int32_t padded = e < E ? (total + 127) & ~127 : 0;
+  // exclusive scan of padded sizes over experts (thread e = expert e)
+  int32_t incl = padded;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += v;
+  }
+  if (lane == 31) wsum[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    int32_t w = wsum[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int32_t v = __shfl_up_sync(0xFFFFFFFFu, w, o);
+      if (lane >= o) w += v;
+    }
+    wsum[lane] = w;  // inclusive over warps
+  }
+  __syncthreads();
+  const int32_t excl = incl - padded + (warp > 0 ? wsum[warp - 1] : 0);
+  if (e < E) {
+    offsets[e] = excl;
+    for (int32_t t = excl / 128; t < (excl + padded) / 128; ++t) tile_expert[t] = e;
+    for (int32_t r = excl + total; r < excl + padded; ++r) row_pair[r] = -1;  // pad rows
+  }
+  if (e == E - 1) {
+    offsets[E] = excl + padded;
+    *tile_count = (excl + padded) / 128;
+  }
+}
+
+__global__ void __launch_bounds__(kRouteThreads) moe_route_place_kernel(const int32_t* __restrict__ topk_ids,
+                                                                         int64_t P, int E,
+                                                                         const int32_t* __restrict__ cta_base,
+                                                                         const int32_t* __restrict__ offsets,
+                                                                         int32_t* __restrict__ row_pair) {
+  extern __shared__ int32_t wcount[];  // [kRouteWarps][E]
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (int i = threadIdx.x; i < kRouteWarps * E; i += blockDim.x) wcount[i] = 0;
+  __syncthreads();
+  int64_t lo, hi;
+  route_range(P, gridDim.x, blockIdx.x, lo, hi);
+  const int64_t wlo = lo + (hi - lo) * warp / kRouteWarps, whi = lo + (hi - lo) * (warp + 1) / kRouteWarps;
+  for (int64_t p = wlo + lane; p < whi; p += 32) {
+    const int e = topk_ids[p];
+    if (e >= 0 && e < E) atomicAdd(&wcount[warp * E + e], 1);
+  }
+  __syncthreads();
+  // per expert: segment offset + this CTA's base + exclusive prefix over warps
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    int32_t run = offsets[e] + cta_base[(int64_t)blockIdx.x * E + e];
+    for (int w = 0; w < kRouteWarps; ++w) {
+      const int32_t c = wcount[w * E + e];
+      wcount[w * E + e] = run;
+      run += c;
+    }
+  }
+  __syncthreads();
+  for (int64_t base = wlo; base < whi; base += 32) {
     const int64_t p = base + lane;
-    const bool valid = p < hi;
-    int e = valid ? topk_ids[p] : -1;
+    int e = p < whi ? topk_ids[p] : -1;
     if (e >= E) e = -1;
     const unsigned same = __match_any_sync(kFullMask, e);
     const int rank = __popc(same & ((1u << lane) - 1u));
     const int leader = __ffs(same) - 1;
-    if (e >= 0) {
-      const int32_t pos = seg[e] + wcount[warp * E + e] + rank;
-      row_pair[pos] = (int32_t)p;
-    }
+    if (e >= 0) row_pair[wcount[warp * E + e] + rank] = (int32_t)p;
     __syncwarp();
     if (e >= 0 && lane == leader) wcount[warp * E + e] += __popc(same);
     __syncwarp();
@@ -205,74 +256,70 @@ __global__ void __launch_bounds__(256) moe_token_pass_kernel(const uint4* __rest
 
 // ----------------------------------------------------------------------------
 // 3 / 5. Row-gathered quantization with a per-expert dynamic global scale.
-// A warp quantizes 256 consecutive elements of one padded row (lane = 8
-// elements, lane pair = one 16-element block). Source row of padded row p:
-// kGather ? x[row_pair[p] / topk] : src[p]; pad rows get zero codes and scales.
-// amax_bits[e] is the BF16 magnitude (kGather) or FP32 bits (h) of the amax.
+// A warp's unit is a 512-element chunk of one padded row, one 16-element
+// block per lane (block_math.cuh). Each trip takes kRowUnroll chunks: first
+// their row lookups, then all their (gathered) loads, then the arithmetic, so
+// several chunks' loads are in flight together. Source row of padded row p:
+// kGather ? x[row_pair[p] / topk] : src[p]; pad rows get zero codes and
+// scales. amax_bits[e] is the BF16 magnitude (kGather) or the FP32 bits (h)
+// of expert e's amax; every CTA turns them into global scales in shared
+// memory once.
 // ----------------------------------------------------------------------------
+constexpr int kRowThreads = 256;
+constexpr int kRowUnroll = 4;
+
 template <bool kGather>
-__global__ void __launch_bounds__(256) moe_quantize_rows_kernel(
+__global__ void __launch_bounds__(kRowThreads) moe_quantize_rows_kernel(
     const uint4* __restrict__ src, int64_t K, int topk, const int32_t* __restrict__ row_pair,
     const int32_t* __restrict__ tile_expert, const int32_t* __restrict__ tile_count,
-    const uint32_t* __restrict__ amax_bits, int E, uint32_t* __restrict__ codes, uint8_t* __restrict__ scales,
-    float* __restrict__ g_out, int* status) {
-  const int lane = threadIdx.x & 31;
-  const int64_t rows = (int64_t)(*tile_count) * 128;
-  const int64_t chunks_per_row = (K + 255) / 256;
-  const int64_t kgroups = K / 64;
-  const int64_t n_chunks = rows * chunks_per_row;
-  if (blockIdx.x == 0) {
-    for (int e = threadIdx.x; e < E; e += blockDim.x) {
-      const uint32_t a = amax_bits[e];
-      const float amax = kGather ? __uint_as_float(a << 16) : __uint_as_float(a);
+    const uint32_t* __restrict__ amax_bits, int E, uint2* __restrict__ codes, uint8_t* __restrict__ scales,
+    float* __restrict__ g_out, int* status, uint64_t cpr_magic) {
+  extern __shared__ float g_s[];  // [E]
+  for (int e = threadIdx.x; e < E; e += blockDim.x) {
+    const uint32_t a = amax_bits[e];
+    const float amax = kGather ? __uint_as_float(a << 16) : __uint_as_float(a);
+    const float g = global_scale_from_amax(amax);
+    g_s[e] = g;
+    if (blockIdx.x == 0) {
+      g_out[e] = g;
       if (kGather ? a >= 0x7F80u : !(amax <= 3.0e38f)) record_status(status, NVFP4_ERR_NONFINITE_INPUT);
-      g_out[e] = global_scale_from_amax(amax);
     }
   }
-  const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t ch = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); ch < n_chunks; ch += nw) {
-    const int64_t p = ch / chunks_per_row;
-    const int64_t col0 = (ch - p * chunks_per_row) * 256;
-    const int32_t pair = row_pair[p];
-    const int e = tile_expert[p >> 7];
-    const uint32_t a = amax_bits[e];
-    const float g = global_scale_from_amax(kGather ? __uint_as_float(a << 16) : __uint_as_float(a));
-    const int64_t e0 = col0 + lane * 8;  // element within the row
-    const bool in_row = e0 < K;          // K % 64 == 0: whole 64-element groups
-    const bool active = pair >= 0 && in_row;
-    float v[8];
-    {
-      uint4 w = make_uint4(0, 0, 0, 0);
-      if (active) {
-        const int64_t srow = kGather ? (int64_t)(pair / topk) : p;
-        w = src[(srow * K + e0) >> 3];
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t rows = (int64_t)(*tile_count) * 128;
+  const int32_t cpr = (int32_t)((K + 511) >> 9);
+  const int64_t n_chunks = rows * cpr;
+  const int64_t kgroups = K >> 6;
+  const int64_t warp = (int64_t)blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * (kRowThreads / 32);
+  for (int64_t ch0 = warp; ch0 < n_chunks; ch0 += kRowUnroll * nwarps) {
+    Chunk cc[kRowUnroll];
+    int32_t pr[kRowUnroll], ex[kRowUnroll];
+#pragma unroll
+    for (int u = 0; u < kRowUnroll; ++u) {
+      const int64_t ch = ch0 + u * nwarps;
+      cc[u] = chunk_at(ch < n_chunks ? ch : 0, cpr, cpr_magic, K, lane);
+      pr[u] = ch < n_chunks ? row_pair[cc[u].row] : -1;
+      ex[u] = ch < n_chunks ? tile_expert[cc[u].row >> 7] : 0;
+    }
+    Raw16 vv[kRowUnroll];
+#pragma unroll
+    for (int u = 0; u < kRowUnroll; ++u) {
+      const int64_t srow = kGather ? (int64_t)(pr[u] / topk) : cc[u].row;
+      load_raw16(src, (srow * K + cc[u].col) >> 3, pr[u] >= 0 && cc[u].valid, vv[u]);
+    }
+#pragma unroll
+    for (int u = 0; u < kRowUnroll; ++u) {
+      if (ch0 + u * nwarps >= n_chunks) break;  // warp-uniform
+      Block b;
+      quantize_block<false, false>(vv[u], block_absmax(vv[u]), g_s[ex[u]], 6.0f, b);
+      if (pr[u] < 0) b.sc = b.q0 = b.q1 = 0u;  // pad row
+      if (cc[u].valid) {
+        codes[(cc[u].row * K + cc[u].col) >> 4] = make_uint2(b.q0, b.q1);
+        scales[scale_offset(cc[u].row, cc[u].col >> 4, kgroups)] = (uint8_t)b.sc;
       }
-      bf16x2_to_f32(w.x, v[0], v[1]);
-      bf16x2_to_f32(w.y, v[2], v[3]);
-      bf16x2_to_f32(w.z, v[4], v[5]);
-      bf16x2_to_f32(w.w, v[6], v[7]);
     }
-    float m = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(v[i]));
-    const float bmax = fmaxf(m, __shfl_xor_sync(kFullMask, m, 1));  // all lanes, uniform
-    uint32_t q = 0, sc = 0;
-    if (active) {
-      sc = block_scale_code(bmax, g, 6.0f);
-      const float d = __fmul_rn(g, e4m3_value(sc));
-      const float r = __frcp_rn(d);
-      float sv[8];
-#pragma unroll
-      for (int i = 0; i < 8; ++i) sv[i] = __fmul_rn(v[i], r);
-      q = e2m1_pack8(sv);
-    }
-    const uint32_t s1 = __shfl_down_sync(kFullMask, sc, 2);
-    const uint32_t s2 = __shfl_down_sync(kFullMask, sc, 4);
-    const uint32_t s3 = __shfl_down_sync(kFullMask, sc, 6);
-    if (!in_row) continue;
-    codes[(p * K + e0) >> 3] = q;
-    if ((lane & 7) == 0)
-      *reinterpret_cast<uint32_t*>(scales + sf_offset(p, e0 >> 4, kgroups)) = sc | (s1 << 8) | (s2 << 16) | (s3 << 24);
   }
 }
 
@@ -444,19 +491,24 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
   const int64_t P = L.P, R = L.R;
   cudaError_t e;
 
-  // 1. route
-  const size_t route_smem = (size_t)(kRouteWarps * a.E + a.E + 1) * sizeof(int32_t);
-  static std::once_flag once;
-  static cudaError_t attr_err = cudaSuccess;
-  std::call_once(once, [] {
-    attr_err = cudaFuncSetAttribute(moe_route_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-  });
-  if (attr_err != cudaSuccess) return attr_err;
-  note_launch();
-  moe_route_kernel<<<1, kRouteThreads, route_smem, s>>>(a.topk_ids, P, a.E, R, I32(L.counts), I32(L.offsets),
-                                                         I32(L.row_pair), I32(L.tile_expert), I32(L.tile_count),
-                                                         U32(L.amax_x), U32(L.amax_h), status);
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  // 1. route: count, scan, place
+  {
+    int64_t G64 = (P + 511) / 512;
+    const int G = (int)(G64 < 1 ? 1 : (G64 > kRouteCtasMax ? kRouteCtasMax : G64));
+    note_launch();
+    moe_route_count_kernel<<<G, kRouteThreads, (size_t)a.E * sizeof(int32_t), s>>>(a.topk_ids, P, a.E,
+                                                                                    I32(L.cta_count), status);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    note_launch();
+    moe_route_scan_kernel<<<1, kScanThreads, 0, s>>>(I32(L.cta_count), G, a.E, I32(L.cta_base), I32(L.counts),
+                                                      I32(L.offsets), I32(L.row_pair), I32(L.tile_expert),
+                                                      I32(L.tile_count), U32(L.amax_x), U32(L.amax_h));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    note_launch();
+    moe_route_place_kernel<<<G, kRouteThreads, (size_t)kRouteWarps * a.E * sizeof(int32_t), s>>>(
+        a.topk_ids, P, a.E, I32(L.cta_base), I32(L.offsets), I32(L.row_pair));
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
 
   // 2. token pass
   {
@@ -469,12 +521,14 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
 
-  const int qgrid = num_sms * 8;
+  const int qgrid = num_sms * 4;
+  const size_t qsmem = (size_t)a.E * sizeof(float);
   // 3. gather + quantize x per expert
   note_launch();
-  moe_quantize_rows_kernel<true><<<qgrid, 256, 0, s>>>(
+  moe_quantize_rows_kernel<true><<<qgrid, kRowThreads, qsmem, s>>>(
       static_cast<const uint4*>(a.x), a.H, a.topk, I32(L.row_pair), I32(L.tile_expert), I32(L.tile_count),
-      U32(L.amax_x), a.E, U32(L.xq_codes), ws + L.xq_scales, F32(L.xq_g), status);
+      U32(L.amax_x), a.E, reinterpret_cast<uint2*>(ws + L.xq_codes), ws + L.xq_scales, F32(L.xq_g), status,
+      chunk_magic(a.H));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   // 4. gate_up grouped GEMM
@@ -508,9 +562,10 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
 
   // 5. quantize h per expert
   note_launch();
-  moe_quantize_rows_kernel<false><<<qgrid, 256, 0, s>>>(
+  moe_quantize_rows_kernel<false><<<qgrid, kRowThreads, qsmem, s>>>(
       reinterpret_cast<const uint4*>(ws + L.h), a.I, a.topk, I32(L.row_pair), I32(L.tile_expert),
-      I32(L.tile_count), U32(L.amax_h), a.E, U32(L.hq_codes), ws + L.hq_scales, F32(L.hq_g), status);
+      I32(L.tile_count), U32(L.amax_h), a.E, reinterpret_cast<uint2*>(ws + L.hq_codes), ws + L.hq_scales,
+      F32(L.hq_g), status, chunk_magic(a.I));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   // 6. down grouped GEMM + weighted FP32 combine
