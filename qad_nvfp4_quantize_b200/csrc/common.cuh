@@ -205,6 +205,13 @@ NVFP4_DEVINL void tma_store_2d(const CUtensorMap* map, const void* smem_src, int
                ::"l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(smem_src))
                : "memory");
 }
+// out[i] += shared[i] for `bytes` / 4 FP32 values (each an atomic add in the
+// memory system), from a 16-byte-aligned shared address to a 16-byte-aligned
+// global address; bytes a multiple of 16. Bulk-group completion.
+NVFP4_DEVINL void bulk_reduce_add_f32(float* dst, uint32_t smem_src, uint32_t bytes) {
+  asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], %2;"
+               ::"l"(dst), "r"(smem_src), "r"(bytes) : "memory");
+}
 NVFP4_DEVINL void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until the bulk stores issued by this thread have finished reading shared memory.
 NVFP4_DEVINL void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }

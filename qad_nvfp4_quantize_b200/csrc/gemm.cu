@@ -10,6 +10,8 @@
 namespace nvfp4 {
 
 struct DenseProblem {
+  static constexpr int kPipeStages = 4;
+  static constexpr uint32_t kEpiWarpBytes = kEpiBytes;
   int M, N, K;
   int m_tiles, n_tiles;
   int kgroups;
@@ -135,7 +137,7 @@ static cudaError_t prepare_kernel() {
   static cudaError_t err = cudaSuccess;
   std::call_once(once, [] {
     err = cudaFuncSetAttribute(nvf4_gemm_kernel<Prob>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)kGemmSmemBytes);
+                               (int)gemm_smem_bytes<Prob>());
   });
   return err;
 }
@@ -170,7 +172,7 @@ cudaError_t launch_gemm(const uint8_t* Aq, const uint8_t* As, const float* ga, c
   const int tiles = p.m_tiles * p.n_tiles;
   const int grid = tiles < num_sms ? tiles : num_sms;
   note_launch();
-  nvf4_gemm_kernel<DenseProblem><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB, tmC, p, status, kGemmTimeoutNs);
+  nvf4_gemm_kernel<DenseProblem><<<grid, kGemmThreads, gemm_smem_bytes<DenseProblem>(), s>>>(tmA, tmB, tmC, p, status, kGemmTimeoutNs);
   return cudaGetLastError();
 }
 

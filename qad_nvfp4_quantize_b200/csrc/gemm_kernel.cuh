@@ -34,7 +34,6 @@ namespace nvfp4 {
 constexpr int kBM = 128;
 constexpr int kBN = 256;
 constexpr int kBK = 256;                       // K elements per stage
-constexpr int kStages = 4;
 constexpr uint32_t kABytes = kBM * kBK / 2;    // 16 KB of codes
 constexpr uint32_t kBHalfBytes = 128 * kBK / 2;
 constexpr uint32_t kBBytes = kBN * kBK / 2;    // 32 KB
@@ -42,23 +41,37 @@ constexpr uint32_t kSFAtom = 512;              // 128 rows x 4 scales
 constexpr uint32_t kSFABytes = 4 * kSFAtom;
 constexpr uint32_t kSFBBytes = 8 * kSFAtom;
 constexpr int kGemmThreads = 320;
-constexpr int kEpiCols = 16;                   // output columns per TMA store box
+constexpr int kEpiCols = 16;                   // dense output columns per TMA store box
 constexpr uint32_t kEpiBytes = 32 * kEpiCols * 2;  // one epilogue warp's BF16 staging box
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kTmemSF = 256;         // first scale column
 constexpr uint32_t kTmemSFStage = 48;     // scale columns per stage
 constexpr uint32_t kTmemSFBOff = 16;      // B scales after A scales inside a stage
-static_assert(kTmemSF + kStages * kTmemSFStage <= kTmemCols, "tensor memory budget");
 
-constexpr uint32_t kSmemA = 0;
-constexpr uint32_t kSmemB = kSmemA + kStages * kABytes;
-constexpr uint32_t kSmemSFA = kSmemB + kStages * kBBytes;
-constexpr uint32_t kSmemSFB = kSmemSFA + kStages * kSFABytes;
-constexpr uint32_t kSmemEpi = kSmemSFB + kStages * kSFBBytes;  // 8 warps x kEpiBytes
-constexpr uint32_t kSmemBar = kSmemEpi + 8 * kEpiBytes;
-constexpr uint32_t kNumBars = 2 * kStages + 3;   // full, empty, acc_full, acc_empty, drain
-constexpr uint32_t kSmemMisc = kSmemBar + kNumBars * 8;
-constexpr uint32_t kGemmSmemBytes = kSmemMisc + 16 + 1024;  // + alignment slack
+// Shared-memory layout of one CTA for a problem with `kStagesT` pipeline
+// stages and `kEpiWarpBytesT` bytes of epilogue staging per epilogue warp.
+template <int kStagesT, uint32_t kEpiWarpBytesT>
+struct GemmSmem {
+  static constexpr int kStages = kStagesT;
+  static constexpr uint32_t kA = 0;
+  static constexpr uint32_t kB = kA + kStages * kABytes;
+  static constexpr uint32_t kSFA = kB + kStages * kBBytes;
+  static constexpr uint32_t kSFB = kSFA + kStages * kSFABytes;
+  static constexpr uint32_t kEpi = kSFB + kStages * kSFBBytes;  // 8 warps x kEpiWarpBytesT
+  static constexpr uint32_t kEpiWarp = kEpiWarpBytesT;
+  static constexpr uint32_t kBar = kEpi + 8 * kEpiWarpBytesT;
+  static constexpr uint32_t kNumBars = 2 * kStages + 3;   // full, empty, acc_full, acc_empty, drain
+  static constexpr uint32_t kMisc = kBar + kNumBars * 8;
+  static constexpr uint32_t kBytes = kMisc + 16 + 1024;  // + alignment slack
+  static_assert(kTmemSF + kStages * kTmemSFStage <= kTmemCols, "tensor memory budget");
+  static_assert(kBytes <= 232448, "shared memory budget");
+};
+
+// Dynamic shared memory of nvf4_gemm_kernel<Prob>.
+template <class Prob>
+constexpr uint32_t gemm_smem_bytes() {
+  return GemmSmem<Prob::kPipeStages, Prob::kEpiWarpBytes>::kBytes;
+}
 
 // Instruction descriptor of kind::mxf4nvf4: A and B E2M1 (format 1), K-major,
 // UE4M3 scales (scale format 0), N >> 3 in bits [17,23), M >> 4 in [24,29).
@@ -83,16 +96,18 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     nvf4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const Prob prob, int* status,
                      uint64_t timeout_ns) {
+  using Lay = GemmSmem<Prob::kPipeStages, Prob::kEpiWarpBytes>;
+  constexpr int kStages = Lay::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + kSmemBar);
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + Lay::kBar);
   uint64_t* full = bars;
   uint64_t* empty = bars + kStages;
   uint64_t* acc_full = bars + 2 * kStages;
   uint64_t* acc_empty = acc_full + 1;
   uint64_t* drain = acc_full + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + kSmemMisc);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kSmemMisc + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + Lay::kMisc);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + Lay::kMisc + 4);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -142,14 +157,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         const uint32_t tx = kABytes + kBBytes + sf_bytes * (job.sfb1 ? 3u : 2u);
         mbar_arrive_expect_tx_elect(&full[stage], tx);
         armed = (armed & ~(0x101u << stage)) | (1u << stage) | (phase << (8 + stage));
-        uint8_t* sA = smem + kSmemA + stage * kABytes;
-        uint8_t* sB = smem + kSmemB + stage * kBBytes;
+        uint8_t* sA = smem + Lay::kA + stage * kABytes;
+        uint8_t* sB = smem + Lay::kB + stage * kBBytes;
         tma_load_2d_elect(sA, &tmA, kt * (kBK / 2), job.a_row, &full[stage]);
         tma_load_2d_elect(sB, &tmB, kt * (kBK / 2), job.b_row0, &full[stage]);
         tma_load_2d_elect(sB + kBHalfBytes, &tmB, kt * (kBK / 2), job.b_row1, &full[stage]);
-        bulk_load_elect(smem + kSmemSFA + stage * kSFABytes, job.sfa + (size_t)kt * kSFABytes, sf_bytes,
+        bulk_load_elect(smem + Lay::kSFA + stage * kSFABytes, job.sfa + (size_t)kt * kSFABytes, sf_bytes,
                         &full[stage]);
-        uint8_t* sSFB = smem + kSmemSFB + stage * kSFBBytes;
+        uint8_t* sSFB = smem + Lay::kSFB + stage * kSFBBytes;
         bulk_load_elect(sSFB, job.sfb0 + (size_t)kt * kSFABytes, sf_bytes, &full[stage]);
         if (job.sfb1) bulk_load_elect(sSFB + kSFABytes, job.sfb1 + (size_t)kt * kSFABytes, sf_bytes, &full[stage]);
         if (++stage == kStages) {
@@ -190,10 +205,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         }
         tc_fence_after();
         const int nkb = min(4, kgroups - 4 * kt);
-        const uint32_t sA = smem_u32(smem + kSmemA + stage * kABytes);
-        const uint32_t sB = smem_u32(smem + kSmemB + stage * kBBytes);
-        const uint32_t sSFA = smem_u32(smem + kSmemSFA + stage * kSFABytes);
-        const uint32_t sSFB = smem_u32(smem + kSmemSFB + stage * kSFBBytes);
+        const uint32_t sA = smem_u32(smem + Lay::kA + stage * kABytes);
+        const uint32_t sB = smem_u32(smem + Lay::kB + stage * kBBytes);
+        const uint32_t sSFA = smem_u32(smem + Lay::kSFA + stage * kSFABytes);
+        const uint32_t sSFB = smem_u32(smem + Lay::kSFB + stage * kSFBBytes);
         const uint64_t adesc = smem_desc(sA, 16, 1024, 2);
         const uint64_t bdesc = smem_desc(sB, 16, 1024, 2);
         const uint32_t tsfa = tmem + kTmemSF + stage * kTmemSFStage;
@@ -257,10 +272,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(acc_empty);
       const TileJob job = prob.job(t);
-      prob.store(job, q, h, lane, acc, smem + kSmemEpi + (warp - 2) * kEpiBytes, &tmC);
+      prob.store(job, q, h, lane, acc, smem + Lay::kEpi + (warp - 2) * Lay::kEpiWarp, &tmC);
       acc_phase ^= 1;
     }
-    if (lane == 0) bulk_wait_all();  // TMA stores of C complete before the CTA exits
+    bulk_wait_all();  // bulk stores / reductions issued by this lane complete before the CTA exits
   }
 
   tc_fence_before();

@@ -329,6 +329,8 @@ __global__ void __launch_bounds__(kRowThreads) moe_quantize_rows_kernel(
 // expert are adjacent (its weight tiles are re-read from L2).
 // ----------------------------------------------------------------------------
 struct GateUpProblem {
+  static constexpr int kPipeStages = 4;
+  static constexpr uint32_t kEpiWarpBytes = 0;  // direct stores
   int K;             // H
   int I;
   int n_tiles;       // I / 128
@@ -404,8 +406,18 @@ struct GateUpProblem {
 
 // ----------------------------------------------------------------------------
 // 6. down grouped GEMM problem: out[token] += w * (g_h * g_w2) * acc.
+// The rows of a tile belong to different tokens, so the sum over a token's
+// experts is a reduction into out. Each epilogue lane stages 32 FP32 values
+// of its row (128 bytes, rows 144 bytes apart so the 32 lanes' writes fall on
+// distinct banks) and adds them into out with one bulk reduction
+// (cp.reduce.async.bulk .add.f32: element-wise atomic adds done by the memory
+// system), 1024 per tile instead of 8192 vector atomics.
 // ----------------------------------------------------------------------------
+constexpr uint32_t kDownRowStride = 144;  // staged row pitch (128 bytes of data)
+
 struct DownProblem {
+  static constexpr int kPipeStages = 3;    // K = I is short: 3 stages cover 1.5 tiles
+  static constexpr uint32_t kEpiWarpBytes = 32 * kDownRowStride;
   int K;             // I
   int H;
   int n_tiles;       // ceil(H / 256)
@@ -445,25 +457,31 @@ struct DownProblem {
   __device__ static constexpr uint32_t tmem_col(int h, int j) { return (uint32_t)(h * 128 + 32 * j); }
 
   __device__ __forceinline__ void store(const TileJob& job, int q, int hh, int lane,
-                                        const uint32_t (&acc)[4][32], uint8_t*, const CUtensorMap*) const {
+                                        const uint32_t (&acc)[4][32], uint8_t* stg, const CUtensorMap*) const {
     const int row = job.m0 + q * 32 + lane;
     const int32_t pair = row_pair[row];
-    if (pair < 0) return;
     const float alpha = __fmul_rn(ga[job.expert], gb[job.expert]);
-    const float w = topk_w[pair];
-    float* orow = out + (size_t)(pair / topk) * H;
+    const float w = pair >= 0 ? topk_w[pair] : 0.0f;
+    float* orow = out + (size_t)(pair >= 0 ? pair / topk : 0) * H;
+    const uint32_t srow = smem_u32(stg) + lane * kDownRowStride;
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int n = job.n0 + hh * 128 + 32 * j;
       if (n >= H) break;
+      bulk_wait_read_all();  // this lane's previous row segment has left shared memory
 #pragma unroll
       for (int c = 0; c < 32; c += 4) {
-        float4 v;
-        v.x = __fmul_rn(__fmul_rn(__uint_as_float(acc[j][c + 0]), alpha), w);
-        v.y = __fmul_rn(__fmul_rn(__uint_as_float(acc[j][c + 1]), alpha), w);
-        v.z = __fmul_rn(__fmul_rn(__uint_as_float(acc[j][c + 2]), alpha), w);
-        v.w = __fmul_rn(__fmul_rn(__uint_as_float(acc[j][c + 3]), alpha), w);
-        atomicAdd(reinterpret_cast<float4*>(orow + n + c), v);
+        uint4 v;
+        v.x = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(acc[j][c + 0]), alpha), w));
+        v.y = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(acc[j][c + 1]), alpha), w));
+        v.z = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(acc[j][c + 2]), alpha), w));
+        v.w = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(acc[j][c + 3]), alpha), w));
+        st_shared_v4(srow + c * 4, v);
+      }
+      fence_proxy_async_smem();
+      if (pair >= 0) {
+        bulk_reduce_add_f32(orow + n, srow, 128);
+        bulk_commit_group();
       }
     }
   }
@@ -475,7 +493,7 @@ static cudaError_t prepare_moe_kernel() {
   static cudaError_t err = cudaSuccess;
   std::call_once(once, [] {
     err = cudaFuncSetAttribute(nvf4_gemm_kernel<Prob>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               (int)kGemmSmemBytes);
+                               (int)gemm_smem_bytes<Prob>());
   });
   return err;
 }
@@ -555,8 +573,8 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
     int64_t max_tiles = (R / 128) * p.n_tiles;
     const int grid = (int)(max_tiles < num_sms ? max_tiles : num_sms);
     note_launch();
-    nvf4_gemm_kernel<GateUpProblem><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB, tmA /* output map unused: direct stores */, p, status,
-                                                                                 kMoeTimeoutNs);
+    nvf4_gemm_kernel<GateUpProblem><<<grid, kGemmThreads, gemm_smem_bytes<GateUpProblem>(), s>>>(
+        tmA, tmB, tmA /* output map unused: direct stores */, p, status, kMoeTimeoutNs);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
 
@@ -594,8 +612,8 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
     int64_t max_tiles = (R / 128) * p.n_tiles;
     const int grid = (int)(max_tiles < num_sms ? max_tiles : num_sms);
     note_launch();
-    nvf4_gemm_kernel<DownProblem><<<grid, kGemmThreads, kGemmSmemBytes, s>>>(tmA, tmB, tmA /* output map unused: direct stores */, p, status,
-                                                                                 kMoeTimeoutNs);
+    nvf4_gemm_kernel<DownProblem><<<grid, kGemmThreads, gemm_smem_bytes<DownProblem>(), s>>>(
+        tmA, tmB, tmA /* output map unused: bulk reductions */, p, status, kMoeTimeoutNs);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;

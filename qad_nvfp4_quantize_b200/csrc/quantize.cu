@@ -284,33 +284,34 @@ constexpr int kFusedThreads = 1024;
 constexpr int kFusedWarps = kFusedThreads / 32;
 constexpr int kKeepChunks = 200;                       // 1 KB of BF16 per chunk
 constexpr int kFusedSmem = kKeepChunks * 1024;
-constexpr int kFusedUnroll = 2;
+constexpr int kFusedUnroll = 2;                        // phase 2: chunks per trip
+constexpr int kLoadUnroll = 4;                         // phase 1: chunk loads in flight per warp
 
-// Grid-wide barrier on bar[0] (arrivals) and bar[1] (generation). Returns
-// false if the wait ran out (the status is recorded by the caller).
-__device__ __forceinline__ bool grid_barrier(uint32_t* bar, uint64_t timeout_ns) {
+// Grid-wide barrier on a 64-bit arrival counter that only grows: CTA arrival
+// number `old` belongs to the barrier generation old / gridDim.x, which
+// releases when the counter reaches the next multiple of gridDim.x. Every
+// launch that uses a workspace has the same grid (one CTA per SM), so the
+// counter stays a multiple of it between launches. Returns false if the wait
+// ran out (the status is recorded by the caller).
+__device__ __forceinline__ bool grid_barrier(unsigned long long* ctr, uint64_t timeout_ns) {
   __shared__ int s_ok;
   __syncthreads();
   if (threadIdx.x == 0) {
-    volatile uint32_t* vgen = bar + 1;
-    const uint32_t gen = *vgen;
-    __threadfence();
     int ok = 1;
-    if (atomicAdd(bar, 1u) == gridDim.x - 1) {
-      atomicExch(bar, 0u);
-      __threadfence();
-      atomicAdd(bar + 1, 1u);
-    } else {
-      const uint64_t t0 = globaltimer_ns();
-      while (*vgen == gen) {
-        if (globaltimer_ns() - t0 > timeout_ns) {
-          ok = 0;
-          break;
-        }
-        __nanosleep(64);
+    __threadfence();  // this CTA's partial maximum before its arrival
+    const unsigned long long old = atomicAdd(ctr, 1ull);
+    const unsigned long long target = (old / gridDim.x + 1) * gridDim.x;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+      unsigned long long now;
+      asm volatile("ld.acquire.gpu.global.u64 %0, [%1];" : "=l"(now) : "l"(ctr) : "memory");
+      if ((long long)(now - target) >= 0) break;
+      if (globaltimer_ns() - t0 > timeout_ns) {
+        ok = 0;
+        break;
       }
+      __nanosleep(32);
     }
-    __threadfence();
     s_ok = ok;
   }
   __syncthreads();
@@ -337,10 +338,10 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_dynamic_kernel(const u
 
   // ---- phase 1: magnitude maximum, keep the first nkeep chunks
   uint32_t m2 = 0;
-  for (int64_t base = lo + warp; base < hi; base += kFusedUnroll * kFusedWarps) {
-    uint4 a[kFusedUnroll], b[kFusedUnroll];
+  for (int64_t base = lo + warp; base < hi; base += kLoadUnroll * kFusedWarps) {
+    uint4 a[kLoadUnroll], b[kLoadUnroll];
 #pragma unroll
-    for (int u = 0; u < kFusedUnroll; ++u) {
+    for (int u = 0; u < kLoadUnroll; ++u) {
       const int64_t ch = base + u * kFusedWarps;
       a[u] = b[u] = make_uint4(0, 0, 0, 0);
       if (ch < hi) {
@@ -352,7 +353,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_dynamic_kernel(const u
       }
     }
 #pragma unroll
-    for (int u = 0; u < kFusedUnroll; ++u) {
+    for (int u = 0; u < kLoadUnroll; ++u) {
       m2 = bmax2(m2, bmax2(bmax2(bmax2(a[u].x, a[u].y), bmax2(a[u].z, a[u].w)),
                            bmax2(bmax2(b[u].x, b[u].y), bmax2(b[u].z, b[u].w))));
       const int64_t k = base + u * kFusedWarps - lo;
@@ -374,7 +375,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_dynamic_kernel(const u
   }
 
   // ---- grid-wide maximum -> global scale
-  if (!grid_barrier(bar, timeout_ns) && threadIdx.x == 0) record_status(status, NVFP4_ERR_TIMEOUT);
+  if (!grid_barrier(reinterpret_cast<unsigned long long*>(bar), timeout_ns) && threadIdx.x == 0) record_status(status, NVFP4_ERR_TIMEOUT);
   if (threadIdx.x < 32) {
     uint32_t mm = 0;
     for (int base = 0; base < (int)gridDim.x; base += 8 * 32) {
