@@ -47,6 +47,12 @@ R9  MoE: routing is input; pairs are stably sorted by expert; each expert's
     rows are quantized with that expert's own dynamic g; h = SiLU(gate) * up
     (gate = first I columns of gate_up) rounded to BF16; h is quantized per
     expert; the weighted combine is a plain sum.
+R10 MSE calibration ([NEMO-QAD] Table 1 "MSE"; "Quantization scale handling
+    during QAD": MSE reaches its scales by a search that minimises the
+    quantization error): for each block, every positive finite E4M3 code
+    (1..126, i.e. 2^-9 .. 448) is a candidate scale under the same g; the
+    block keeps the candidate with the lowest FP32 squared error computed as
+    in R6; ties keep the lowest code.
 """
 from __future__ import annotations
 
@@ -55,6 +61,7 @@ import numpy as np
 BLOCK = 16                 # elements per block scale [QF-NVFP4, level 1]
 E2M1_MAX = 6.0             # largest E2M1 magnitude
 E4M3_MAX = 448.0           # largest finite E4M3 value
+E4M3_MAX_CODE = 126        # its code (0x7F is NaN)
 GLOBAL_DIVISOR = np.float32(6.0 * 448.0)   # R2: 2688
 
 
@@ -237,6 +244,8 @@ def quantize(x: np.ndarray, mode: str = "max", g: np.float32 | None = None):
     [QF-NVFP4] dynamic activations use the same rule).
     mode "four_over_six": per block keep the M=6 or M=4 scale, whichever
     gives the lower block error ([NEMO-QAD] Table 1, four_over_six).
+    mode "mse": per block keep, of all 126 positive finite E4M3 scales, the
+    one with the lowest block error (R10; [NEMO-QAD] Table 1, MSE).
     g: a static global scale; None computes it from the tensor (dynamic).
     """
     x = np.asarray(x, dtype=np.float32)
@@ -253,6 +262,18 @@ def quantize(x: np.ndarray, mode: str = "max", g: np.float32 | None = None):
     if mode == "max":
         return dict(codes=q6.reshape(rows, K), scales=s6, g=g,
                     choice=np.zeros_like(s6), err=e6)
+    if mode == "mse":
+        best_s = np.ones(s6.shape, np.uint8)
+        best_q, best_e = _encode_blocks(blocks, g, best_s)
+        for c in range(2, E4M3_MAX_CODE + 1):                   # R10: increasing code
+            sc = np.full(s6.shape, c, np.uint8)
+            q, e = _encode_blocks(blocks, g, sc)
+            better = e < best_e                                  # ties keep the lower code
+            best_q = np.where(better[..., None], q, best_q)
+            best_s = np.where(better, sc, best_s).astype(np.uint8)
+            best_e = np.where(better, e, best_e)
+        return dict(codes=best_q.reshape(rows, K), scales=best_s, g=g,
+                    choice=np.zeros_like(s6), err=best_e)
     if mode != "four_over_six":
         raise ValueError(f"unknown mode {mode!r}")
     s4 = block_scale_codes(bmax, g, 4.0)

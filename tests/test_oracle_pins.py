@@ -290,6 +290,81 @@ def test_four_over_six_brute_force_over_all_scales():
             assert best <= out["err"][r, b]
 
 
+# --------------------------------------------------------- MSE calibration ---
+
+def _lib_e4m3_scales():
+    """(code, value) of every positive finite E4M3 code, decoded by ml_dtypes."""
+    codes = np.arange(1, 127, dtype=np.uint8)
+    return codes, codes.view(ml_dtypes.float8_e4m3fn).astype(np.float32)
+
+
+def _mse_blocks(seed):
+    rng = np.random.default_rng(seed)
+    rows = []
+    for kind in range(8):
+        base = rng.standard_normal(16).astype(np.float32) * 0.02
+        if kind == 1:
+            base[rng.integers(16)] *= 20
+        if kind == 2:
+            base = rng.uniform(-1, 1, 16).astype(np.float32)
+        if kind == 3:
+            base = np.sign(base) * np.abs(base) ** 3
+        if kind == 4:
+            base[:] = 0.01
+        if kind == 5:
+            base = rng.standard_t(3, 16).astype(np.float32)
+        if kind == 6:
+            base[:] = 0.0
+        if kind == 7:
+            base = rng.standard_t(2, 16).astype(np.float32) * 1e-3
+        rows.append(base)
+    x = torch.from_numpy(np.stack(rows).reshape(4, 32)).to(torch.bfloat16).float().numpy()
+    x[0, 0] = 1.0                                       # sets the tensor amax
+    return x
+
+
+def test_mse_matches_brute_force_over_all_scales():
+    # R10: the kept scale is the lowest code reaching the smallest block error
+    # over all 126 scales; errors by library conversions, summed in index order
+    codes, values = _lib_e4m3_scales()
+    for seed in (3, 4):
+        x = _mse_blocks(seed)
+        out = o.quantize(x, "mse")
+        g = out["g"]
+        for r in range(x.shape[0]):
+            for b in range(2):
+                xb = x[r, 16 * b:16 * b + 16]
+                errs = np.array([_lib_block_error(xb, g, v) for v in values], np.float32)
+                best = int(np.argmin(errs))                 # first minimum = lowest code
+                assert out["err"][r, b] == errs[best], (seed, r, b)
+                assert out["scales"][r, b] == codes[best], (seed, r, b)
+                s = values[best]
+                want = [lib_e2m1(np.float32(v) * (np.float32(1.0) / (np.float32(g) * s))) for v in xb]
+                assert list(out["codes"][r, 16 * b:16 * b + 16]) == want
+
+
+def test_mse_never_worse_than_max_or_four_over_six():
+    rng = np.random.default_rng(12)
+    x = torch.from_numpy((rng.standard_t(3, (24, 256)) * 0.05).astype(np.float32)).to(torch.bfloat16).float().numpy()
+    e_max = o.quantize(x, "max")["err"]
+    e_fos = o.quantize(x, "four_over_six")["err"]
+    e_mse = o.quantize(x, "mse")["err"]
+    assert np.all(e_fos <= e_max)
+    assert np.all(e_mse <= e_fos)
+    assert np.any(e_mse < e_fos)                            # the wider search does find better scales
+
+
+def test_mse_finds_exact_representation():
+    # a block that is exactly g*s*q for one scale s is reproduced with error 0
+    g = np.float32(2.0 ** -8)
+    s = np.float32(12.0)                                # E4M3 code 0x52 = 82
+    q = np.array([0, .5, 1, 1.5, 2, 3, 4, 6, -0.5, -1, -1.5, -2, -3, -4, -6, 0], np.float32)
+    x = (g * s * q).astype(np.float32)[None, :]
+    out = o.quantize(x, "mse", g=g)
+    assert out["err"][0, 0] == 0.0
+    assert np.array_equal(o.dequantize(out["codes"], out["scales"], g), x)
+
+
 # -------------------------------------------------------------------- GEMM ---
 
 def test_gemm_reference_brute_force_tiny():
