@@ -68,7 +68,12 @@ typedef enum {
 
 typedef enum {
   NVFP4_MODE_MAX = 0,           /* every block targets the E2M1 maximum 6 */
-  NVFP4_MODE_FOUR_OVER_SIX = 1  /* per block, target 6 or 4, lower block MSE */
+  NVFP4_MODE_FOUR_OVER_SIX = 1, /* per block, target 6 or 4, lower block MSE */
+  NVFP4_MODE_MSE = 2            /* per block, the E4M3 scale (of all 126) with the
+                                   lowest block squared error, ties to the lowest
+                                   code: MSE calibration, Table 1 of "Developing
+                                   Nemotron 3.5 Lightning NVFP4 with QAD using
+                                   NVIDIA Model Optimizer". nvfp4_quantize only. */
 } nvfp4_mode;
 
 /* Library version (major*10000 + minor*100 + patch). Host only. */
@@ -98,8 +103,12 @@ size_t nvfp4_quantize_workspace_bytes(int64_t M, int64_t K);
  *   g = amax/2688 (or *g_in when given: a static, calibrated global scale);
  *   per block of 16, s = E4M3(bmax / (Mt * g)) floored at 2^-9, Mt = 6
  *   (mode MAX) or the better of 6 and 4 by block squared error (mode
- *   FOUR_OVER_SIX, tie -> 6); codes = E2M1(x * (1 / (g * s))); every
- *   rounding is to nearest even and saturating (E2M1 at +-6, E4M3 at 448).
+ *   FOUR_OVER_SIX, tie -> 6), or (mode MSE, Table 1 "MSE" of "Developing
+ *   Nemotron 3.5 Lightning NVFP4 with QAD using NVIDIA Model Optimizer")
+ *   the E4M3 scale, of all 126 positive finite ones, with the lowest block
+ *   squared error (ties -> lowest code); codes = E2M1(x * (1 / (g * s)));
+ *   every rounding is to nearest even and saturating (E2M1 at +-6, E4M3 at
+ *   448).
  *   Dynamic activations use g_in = NULL ("the A4 side: dynamic activations");
  *   static weights pass a precomputed g_in or let the call compute it.
  * x           [M][K] BF16, device.
@@ -108,7 +117,7 @@ size_t nvfp4_quantize_workspace_bytes(int64_t M, int64_t K);
  * scales      out nvfp4_scale_bytes(M, K) bytes (tiled layout, padding zeroed).
  * g_out       out device FP32 scalar: the global scale used.
  * fos_choice  nullable out [M][K/16] bytes: 1 where the block kept the M=4
- *             scale, else 0 (always 0 in mode MAX).
+ *             scale, else 0 (always 0 in modes MAX and MSE).
  * workspace   >= nvfp4_quantize_workspace_bytes(M, K) bytes when g_in is
  *             NULL (zero-filled before its first use, see above); may be
  *             NULL when g_in is given. Calls that share one workspace must

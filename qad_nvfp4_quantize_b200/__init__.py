@@ -24,8 +24,9 @@ __all__ = [
 
 MODE_MAX = 0
 MODE_FOUR_OVER_SIX = 1
-_MODES = {"max": MODE_MAX, "four_over_six": MODE_FOUR_OVER_SIX, MODE_MAX: MODE_MAX,
-          MODE_FOUR_OVER_SIX: MODE_FOUR_OVER_SIX}
+MODE_MSE = 2
+_MODES = {"max": MODE_MAX, "four_over_six": MODE_FOUR_OVER_SIX, "mse": MODE_MSE, MODE_MAX: MODE_MAX,
+          MODE_FOUR_OVER_SIX: MODE_FOUR_OVER_SIX, MODE_MSE: MODE_MSE}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
 library_path = os.path.join(_HERE, "libnvfp4.so")

@@ -119,7 +119,8 @@ size_t nvfp4_quantize_workspace_bytes(int64_t M, int64_t K) {
 nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t K, nvfp4_mode mode, const float* g_in,
                             uint8_t* codes, uint8_t* scales, float* g_out, uint8_t* fos_choice,
                             void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
-  if (M < 0 || K <= 0 || K % 64 || (mode != NVFP4_MODE_MAX && mode != NVFP4_MODE_FOUR_OVER_SIX))
+  if (M < 0 || K <= 0 || K % 64 ||
+      (mode != NVFP4_MODE_MAX && mode != NVFP4_MODE_FOUR_OVER_SIX && mode != NVFP4_MODE_MSE))
     return NVFP4_ERR_INVALID_ARG;
   if (M > 0 && (!x || !codes || !scales || !aligned16(x) || !aligned16(codes) || !aligned16(scales)))
     return NVFP4_ERR_INVALID_ARG;
@@ -129,18 +130,18 @@ nvfp4_status nvfp4_quantize(const void* x, int64_t M, int64_t K, nvfp4_mode mode
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   const uint32_t* partial = nullptr;
   int np = 0;
-  const bool fos = mode == NVFP4_MODE_FOUR_OVER_SIX;
+  const int m = (int)mode;
   if (!g_in) {
     if (!workspace || workspace_bytes < nvfp4_quantize_workspace_bytes(M, K) || !aligned16(workspace))
       return NVFP4_ERR_WORKSPACE;
     // one launch: amax, grid barrier and quantization with X kept on chip
-    const cudaError_t e = nvfp4::launch_quantize_fused(x, M, K, fos, static_cast<uint32_t*>(workspace), codes,
+    const cudaError_t e = nvfp4::launch_quantize_fused(x, M, K, m, static_cast<uint32_t*>(workspace), codes,
                                                        scales, g_out, fos_choice, d->status, d->num_sms, s);
     if (e != cudaErrorNotSupported) return launched(e);
     st = run_amax(x, M * K, workspace, workspace_bytes, d->num_sms, s, &partial, &np);
     if (st != NVFP4_OK) return st;
   }
-  return launched(nvfp4::launch_quantize(x, M, K, fos, partial, np, g_in, codes, scales, g_out, fos_choice,
+  return launched(nvfp4::launch_quantize(x, M, K, m, partial, np, g_in, codes, scales, g_out, fos_choice,
                                          d->status, d->num_sms, s));
 }
 

@@ -146,15 +146,20 @@ struct Block {
   float err;
 };
 
+// The block's 16 values as FP32 pairs (exact).
+__device__ __forceinline__ void unpack_block(const Raw16& raw, f32x2 (&xs)[8]) {
+#pragma unroll
+  for (int i = 0; i < 8; ++i) xs[i] = bf16x2_unpack(raw.w[i]);
+}
+
+// Codes of a block under step d = g*s and its reciprocal r = RN(1/d), and on
+// request the dequantized values and the squared error (sequential FP32 sum).
 template <bool kDeq, bool kErr>
-__device__ __forceinline__ void quantize_block(const Raw16& raw, float bmax, float g, float mt, Block& b) {
-  b.sc = block_scale_code(bmax, g, mt);
-  const float d = __fmul_rn(g, scale_value(b.sc));
-  const float r = __frcp_rn(d);
+__device__ __forceinline__ void encode_block(const f32x2 (&xs)[8], float d, float r, Block& b) {
   const f32x2 rr = pack2(r, r);
   f32x2 sv[8];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) sv[i] = mul2(bf16x2_unpack(raw.w[i]), rr);
+  for (int i = 0; i < 8; ++i) sv[i] = mul2(xs[i], rr);
   b.q0 = e2m1_pack4(sv[0], sv[1], sv[2], sv[3]);
   b.q1 = e2m1_pack4(sv[4], sv[5], sv[6], sv[7]);
   if (kDeq || kErr) {
@@ -182,7 +187,7 @@ __device__ __forceinline__ void quantize_block(const Raw16& raw, float bmax, flo
     float acc = 0.0f;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-      const f32x2 df = sub2(bf16x2_unpack(raw.w[i]), b.deq[i]);
+      const f32x2 df = sub2(xs[i], b.deq[i]);
       float lo, hi;
       unpack2(mul2(df, df), lo, hi);
       acc = __fadd_rn(acc, lo);  // element order: 2i, then 2i+1
@@ -192,6 +197,21 @@ __device__ __forceinline__ void quantize_block(const Raw16& raw, float bmax, flo
   } else {
     b.err = 0.0f;
   }
+}
+
+// Block scale for target magnitude mt (6 or 4), then the codes under it.
+template <bool kDeq, bool kErr>
+__device__ __forceinline__ void quantize_block(const f32x2 (&xs)[8], float bmax, float g, float mt, Block& b) {
+  b.sc = block_scale_code(bmax, g, mt);
+  const float d = __fmul_rn(g, scale_value(b.sc));
+  encode_block<kDeq, kErr>(xs, d, __frcp_rn(d), b);
+}
+
+template <bool kDeq, bool kErr>
+__device__ __forceinline__ void quantize_block(const Raw16& raw, float bmax, float g, float mt, Block& b) {
+  f32x2 xs[8];
+  unpack_block(raw, xs);
+  quantize_block<kDeq, kErr>(xs, bmax, g, mt, b);
 }
 
 // A warp's unit of work: 512 consecutive elements of one row ("chunk"), one

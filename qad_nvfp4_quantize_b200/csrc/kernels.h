@@ -19,7 +19,8 @@ inline uint64_t chunk_magic(int64_t K) {
 int amax_partial_count(int64_t n, int num_sms);
 cudaError_t launch_amax_partial(const void* x, int64_t n, uint32_t* partial, int n_partial,
                                 cudaStream_t s);
-cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, bool fos, const uint32_t* partial,
+// mode: 0 max, 1 four_over_six, 2 MSE calibration (nvfp4_mode values).
+cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, int mode, const uint32_t* partial,
                             int n_partial, const float* g_static, uint8_t* codes, uint8_t* scales,
                             float* g_out, uint8_t* choice, int* status, int num_sms, cudaStream_t s);
 cudaError_t launch_fake_quant(const void* x, int64_t M, int64_t K, bool fos, const uint32_t* partial,
@@ -29,7 +30,7 @@ cudaError_t launch_fake_quant(const void* x, int64_t M, int64_t K, bool fos, con
 // quantization). ws: kMaxPartials partial slots followed by two barrier
 // words that must be zero before the first use. Returns
 // cudaErrorNotSupported when the cooperative launch is not possible.
-cudaError_t launch_quantize_fused(const void* x, int64_t M, int64_t K, bool fos, uint32_t* ws, uint8_t* codes,
+cudaError_t launch_quantize_fused(const void* x, int64_t M, int64_t K, int mode, uint32_t* ws, uint8_t* codes,
                                   uint8_t* scales, float* g_out, uint8_t* choice, int* status, int num_sms,
                                   cudaStream_t s);
 cudaError_t launch_fake_quant_fused(const void* x, int64_t M, int64_t K, bool fos, uint32_t* ws, void* y,

@@ -82,7 +82,7 @@ extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t M, int64_t
     if (np < 1) np = 1;
     if (nvfp4::launch_amax_partial(x, n, partial, np, s) != cudaSuccess) return NVFP4_ERR_CUDA;
   }
-  return nvfp4::launch_quantize(x, M, K, mode == NVFP4_MODE_FOUR_OVER_SIX, partial, np, g_in, codes, scales,
+  return nvfp4::launch_quantize(x, M, K, (int)mode, partial, np, g_in, codes, scales,
                                 g_out, fos_choice, status, num_sms, s) == cudaSuccess
              ? NVFP4_OK
              : NVFP4_ERR_CUDA;

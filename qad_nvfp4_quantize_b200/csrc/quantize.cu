@@ -133,12 +133,14 @@ struct QuantOp {
 
   __device__ __forceinline__ void operator()(const Raw16& v, const Chunk& c, float g, int lane) const {
     const float bmax = block_absmax(v);
+    f32x2 xs[8];
+    unpack_block(v, xs);
     Block b6;
-    quantize_block<false, kFos>(v, bmax, g, 6.0f, b6);
+    quantize_block<false, kFos>(xs, bmax, g, 6.0f, b6);
     uint32_t sc = b6.sc, q0 = b6.q0, q1 = b6.q1, pick4 = 0;
     if (kFos) {
       Block b4;
-      quantize_block<false, true>(v, bmax, g, 4.0f, b4);
+      quantize_block<false, true>(xs, bmax, g, 4.0f, b4);
       pick4 = b4.err < b6.err;  // tie keeps M = 6
       if (pick4) {
         sc = b4.sc;
@@ -153,6 +155,8 @@ struct QuantOp {
       if (kFos && choice) choice[c.vec >> 1] = (uint8_t)pick4;
     }
   }
+
+  __device__ __forceinline__ void prepare(float) const {}
 
   // Work independent of the values: zero padding-row scales; a max-mode call
   // that asked for a choice map gets zeros.
@@ -176,11 +180,13 @@ struct FakeOp {
   __device__ __forceinline__ void operator()(const Raw16& v, const Chunk& c, float g, int lane) const {
     (void)lane;
     const float bmax = block_absmax(v);
+    f32x2 xs[8];
+    unpack_block(v, xs);
     Block b6;
-    quantize_block<true, kFos>(v, bmax, g, 6.0f, b6);
+    quantize_block<true, kFos>(xs, bmax, g, 6.0f, b6);
     if (kFos) {
       Block b4;
-      quantize_block<true, true>(v, bmax, g, 4.0f, b4);
+      quantize_block<true, true>(xs, bmax, g, 4.0f, b4);
       if (b4.err < b6.err) {
         store_bf16x16(y, c, b4.deq);
         return;
@@ -188,6 +194,7 @@ struct FakeOp {
     }
     store_bf16x16(y, c, b6.deq);
   }
+  __device__ __forceinline__ void prepare(float) const {}
   __device__ __forceinline__ void finish() const {}
 
   __device__ static __forceinline__ uint32_t to_bf16x2(f32x2 v) {
@@ -224,7 +231,73 @@ struct FrozenFakeOp {
     for (int i = 0; i < 8; ++i) out[i] = mul2(dd, out[i]);
     FakeOp<false>::store_bf16x16(y, c, out);
   }
+  __device__ __forceinline__ void prepare(float) const {}
   __device__ __forceinline__ void finish() const {}
+};
+
+// MSE calibration ("Developing Nemotron 3.5 Lightning NVFP4 with QAD using
+// NVIDIA Model Optimizer", Table 1 "MSE"): every positive finite E4M3 code is
+// a candidate block scale; the block keeps the lowest squared error, ties to
+// the lowest code. Candidates run from code 126 down; the block's largest
+// element alone costs (bmax - RN(6d))^2 once 6d < bmax (its code saturates at
+// 6), which grows as d shrinks, so the search stops at the first candidate
+// whose bound exceeds the best error (it cannot win or tie). d and 1/d per
+// code are tabulated once per CTA.
+struct MseOp {
+  uint2* codes;
+  uint8_t* scales;
+  uint8_t* choice;
+  int64_t M, K;
+
+  __device__ static __forceinline__ float* table() {
+    __shared__ float t[2 * 128];  // d[c], then RN(1/d[c])
+    return t;
+  }
+
+  __device__ __forceinline__ void prepare(float g) const {
+    float* t = table();
+    for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+      const float d = __fmul_rn(g, scale_value(c >= 1 && c <= 126 ? (uint32_t)c : 1u));
+      t[c] = d;
+      t[128 + c] = __frcp_rn(d);
+    }
+    __syncthreads();
+  }
+
+  __device__ __forceinline__ void operator()(const Raw16& v, const Chunk& c, float g, int lane) const {
+    (void)g;
+    (void)lane;
+    const float* t = table();
+    const float bmax = block_absmax(v);
+    f32x2 xs[8];
+    unpack_block(v, xs);
+    Block b;
+    encode_block<false, true>(xs, t[126], t[128 + 126], b);
+    uint32_t best_sc = 126, q0 = b.q0, q1 = b.q1;
+    float best = b.err;
+    for (int code = 125; code >= 1; --code) {
+      const float d = t[code];
+      const float dm = __fmul_rn(d, 6.0f);
+      if (dm < bmax) {
+        const float df = __fsub_rn(bmax, dm);
+        if (__fmul_rn(df, df) > best) break;
+      }
+      encode_block<false, true>(xs, d, t[128 + code], b);
+      if (b.err <= best) {  // ties move to the lower code
+        best = b.err;
+        best_sc = (uint32_t)code;
+        q0 = b.q0;
+        q1 = b.q1;
+      }
+    }
+    if (c.valid) {
+      codes[c.vec >> 1] = make_uint2(q0, q1);
+      scales[scale_offset(c.row, c.col >> 4, K >> 6)] = (uint8_t)best_sc;
+      if (choice) choice[c.vec >> 1] = 0;
+    }
+  }
+
+  __device__ __forceinline__ void finish() const { zero_pad_scale_rows(scales, M, K >> 6); }
 };
 
 // ----------------------------------------------------------------------------
@@ -239,6 +312,7 @@ __global__ void __launch_bounds__(kQThreads) stream_pass_kernel(const uint4* __r
                                                                  uint64_t cpr_magic) {
   bool bad;
   const float g = resolve_global_scale(partial, n_partial, g_static, &bad);
+  op.prepare(g);
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     if (g_out) *g_out = g;
     if (bad) record_status(status, NVFP4_ERR_NONFINITE_INPUT);
@@ -397,6 +471,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_dynamic_kernel(const u
   }
   __syncthreads();
   const float g = s_g;
+  op.prepare(g);
   if (blockIdx.x == 0 && threadIdx.x == 0) {
     if (g_out) *g_out = g;
     if (s_bad) record_status(status, NVFP4_ERR_NONFINITE_INPUT);
@@ -534,11 +609,14 @@ static cudaError_t launch_fused(const void* x, int64_t M, int64_t K, uint32_t* w
   return e;
 }
 
-cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, bool fos, const uint32_t* partial,
+cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, int mode, const uint32_t* partial,
                             int n_partial, const float* g_static, uint8_t* codes, uint8_t* scales,
                             float* g_out, uint8_t* choice, int* status, int num_sms, cudaStream_t s) {
   uint2* c = reinterpret_cast<uint2*>(codes);
-  if (fos)
+  if (mode == 2)
+    return launch_stream(x, M, K, partial, n_partial, g_static, MseOp{c, scales, choice, M, K}, g_out, status,
+                         num_sms, s);
+  if (mode == 1)
     return launch_stream(x, M, K, partial, n_partial, g_static, QuantOp<true>{c, scales, choice, M, K}, g_out, status,
                          num_sms, s);
   return launch_stream(x, M, K, partial, n_partial, g_static, QuantOp<false>{c, scales, choice, M, K}, g_out, status,
@@ -557,11 +635,12 @@ cudaError_t launch_fake_quant(const void* x, int64_t M, int64_t K, bool fos, con
   return launch_stream(x, M, K, partial, n_partial, g_static, FakeOp<false>{yv, M, K}, nullptr, status, num_sms, s);
 }
 
-cudaError_t launch_quantize_fused(const void* x, int64_t M, int64_t K, bool fos, uint32_t* ws, uint8_t* codes,
+cudaError_t launch_quantize_fused(const void* x, int64_t M, int64_t K, int mode, uint32_t* ws, uint8_t* codes,
                                   uint8_t* scales, float* g_out, uint8_t* choice, int* status, int num_sms,
                                   cudaStream_t s) {
   uint2* c = reinterpret_cast<uint2*>(codes);
-  if (fos) return launch_fused(x, M, K, ws, QuantOp<true>{c, scales, choice, M, K}, g_out, status, num_sms, s);
+  if (mode == 2) return launch_fused(x, M, K, ws, MseOp{c, scales, choice, M, K}, g_out, status, num_sms, s);
+  if (mode == 1) return launch_fused(x, M, K, ws, QuantOp<true>{c, scales, choice, M, K}, g_out, status, num_sms, s);
   return launch_fused(x, M, K, ws, QuantOp<false>{c, scales, choice, M, K}, g_out, status, num_sms, s);
 }
 

@@ -198,3 +198,43 @@ def test_bounded_wait_reports_timeout(nv):
     x = torch.ones((128, 64), dtype=torch.bfloat16, device="cuda")
     nv.quantize(x)                      # the context is still usable
     assert nv.device_status(clear=True) == 0
+
+
+@pytest.mark.parametrize("M,K", [(3, 64), (130, 320), (64, 1024)])
+def test_mse_calibration_matches_oracle(nv, M, K):
+    rng = np.random.default_rng(M + K)
+    x = (rng.standard_t(3, (M, K)) * 0.05).astype(np.float32)
+    x[0, :16] = 0.0                                             # all-tie block: lowest code
+    x[1 % M, 16:32] = rng.choice([-6, -1, 0, 0.5, 3, 6], 16) * 0.01  # exact on some scale grid
+    x[2 % M, 40] = 3.0                                          # outlier sets the amax
+    xt = inputs.to_bf16(x)
+    for g in (None, torch.tensor([np.float32(0.05)])):
+        q = nv.quantize(xt.cuda(), "mse", g=None if g is None else g.cuda(), want_choice=True)
+        ref = oracle_quantized(bf16_np(xt), "mse", None if g is None else np.float32(0.05))
+        assert_quantized_equal(q, ref, M, K)
+        assert not to_np(q.choice).any()
+
+
+def test_mse_calibration_full_weight_sampled_rows(nv):
+    # W 14336 x 4096 with 0.1% outliers: quantize on the GPU, check sampled rows
+    # against the oracle run with the GPU's global scale
+    d = inputs.four_over_six_linear(0, M=16)
+    w = d["w"]
+    q = nv.quantize(w.cuda(), "mse")
+    g = np.float32(to_np(q.g)[0])
+    wf = bf16_np(w)
+    assert g == o.global_scale(wf)[0]
+    rows = np.array([0, 1, 127, 128, 5000, 9999, 14335])
+    ref = o.quantize(wf[rows], "mse", g)
+    codes = o.unpack_codes(to_np(q.codes)[rows])
+    scales = o.scales_from_tiled(to_np(q.scales), w.shape[0], w.shape[1])[rows]
+    assert np.array_equal(scales, ref["scales"])
+    assert np.array_equal(codes, ref["codes"])
+
+
+def test_mse_rejected_outside_quantize(nv):
+    x = torch.zeros((4, 64), dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(nv.NVFP4Error):
+        nv.fake_quant(x, "mse")
+    with pytest.raises(nv.NVFP4Error):
+        nv.quantize_noalloc(x, "mse")
