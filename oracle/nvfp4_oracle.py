@@ -47,6 +47,12 @@ R9  MoE: routing is input; pairs are stably sorted by expert; each expert's
     rows are quantized with that expert's own dynamic g; h = SiLU(gate) * up
     (gate = first I columns of gate_up) rounded to BF16; h is quantized per
     expert; the weighted combine is a plain sum.
+R11 QAD backward through the simulated quantization ([NEMO-QAD] Figure 2:
+    "gradient back to the FP weights through the loss"; the estimator is not
+    named): a straight-through estimator clipped to the quantizer's range --
+    dL/dx = dL/dy where |x * r| <= 6 for the block's r = RN(1/(g*s)) (FP32
+    product), else 0. Rounding is passed straight through; saturation is not.
+    The scales are those of the forward: recomputed (dynamic) or frozen.
 R10 MSE calibration ([NEMO-QAD] Table 1 "MSE"; "Quantization scale handling
     during QAD": MSE reaches its scales by a search that minimises the
     quantization error): for each block, every positive finite E4M3 code
@@ -315,6 +321,30 @@ def fake_quant(x: np.ndarray, mode: str = "max", g_frozen=None, scales_frozen=No
         q, _ = _encode_blocks(x.reshape(rows, K // BLOCK, BLOCK), g, scales)
         codes = q.reshape(rows, K)
     return bf16_round(dequantize(codes, scales, g))
+
+
+def fake_quant_backward(x: np.ndarray, grad_y: np.ndarray, mode: str = "max", g_frozen=None,
+                        scales_frozen=None) -> np.ndarray:
+    """Gradient of the QAD fake-quant w.r.t. x (R11): grad_y where the
+    element is inside its block's quantizer range |x * RN(1/(g*s))| <= 6, else
+    0. Scales as in ``fake_quant`` (dynamic: from x with ``mode``; frozen:
+    given). Returns FP32 arrays holding the (BF16) gradient values."""
+    x = np.asarray(x, dtype=np.float32)
+    gy = np.asarray(grad_y, dtype=np.float32)
+    rows, K = x.shape
+    if (g_frozen is None) != (scales_frozen is None):
+        raise ValueError("frozen mode needs both g and the block scales")
+    if g_frozen is None:
+        qz = quantize(x, mode)
+        scales, g = qz["scales"], qz["g"]
+    else:
+        g = np.float32(g_frozen)
+        scales = np.asarray(scales_frozen, dtype=np.uint8).reshape(rows, K // BLOCK)
+    d = np.float32(g) * e4m3_decode(scales).astype(np.float32)          # R4
+    r = np.float32(1.0) / d
+    v = x.reshape(rows, K // BLOCK, BLOCK) * r[..., None]               # FP32 products
+    inside = (np.abs(v) <= np.float32(E2M1_MAX)).reshape(rows, K)
+    return np.where(inside, gy, np.float32(0.0)).astype(np.float32)
 
 
 # ----------------------------------------------------------------------------

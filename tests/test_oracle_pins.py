@@ -478,3 +478,49 @@ def test_moe_single_expert_is_the_dense_mlp():
     y = gh * gw2 * (ha @ w2a.T)
     assert np.allclose(ref["stages"][0]["gate_up"], gu, rtol=1e-12, atol=1e-15)
     assert np.allclose(ref["out"], y, rtol=1e-9, atol=1e-12)
+
+
+# ------------------------------------------------------- QAD backward (STE) ---
+
+def test_ste_backward_closed_form_block():
+    # frozen g = 1, s = 1 (E4M3 code 0x38): the range is |x| <= 6
+    x = np.zeros((1, 16), np.float32)
+    x[0, :8] = [0.5, 6.0, 6.5, -7.0, 5.9375, -6.0, 100.0, -0.0]
+    gy = np.arange(1, 17, dtype=np.float32)[None, :]
+    gx = o.fake_quant_backward(x, gy, g_frozen=np.float32(1.0), scales_frozen=np.array([[0x38]], np.uint8))
+    want = gy.copy()
+    want[0, [2, 3, 6]] = 0.0
+    assert np.array_equal(gx, want)
+
+
+def test_ste_backward_matches_autograd_of_clamp():
+    # the clipped STE passes the gradient exactly where clamp(x * r, -6, 6)
+    # has derivative 1 (rounding passed straight through): torch autograd
+    rng = np.random.default_rng(31)
+    x = torch.from_numpy((rng.standard_t(3, (8, 64)) * 0.3).astype(np.float32)).to(torch.bfloat16).float().numpy()
+    gy = rng.standard_normal((8, 64)).astype(np.float32)
+    # frozen scales calibrated on a narrower tensor, so some elements saturate
+    q = o.quantize(x * np.float32(0.5), "max")
+    g, sc = q["g"], q["scales"]
+    gx = o.fake_quant_backward(x, gy, g_frozen=g, scales_frozen=sc)
+    d = torch.from_numpy((np.float32(g) * ml_dtypes_values(sc)).astype(np.float32))
+    r = (1.0 / d).repeat_interleave(16, dim=1)
+    v = (torch.from_numpy(x) * r).requires_grad_(True)     # FP32 products x * r
+    torch.clamp(v, -6.0, 6.0).backward(torch.from_numpy(gy))
+    assert np.array_equal(gx, v.grad.numpy())
+    assert (gx == 0).any() and (gx != 0).any()
+
+
+def ml_dtypes_values(codes):
+    return np.asarray(codes, np.uint8).view(ml_dtypes.float8_e4m3fn).astype(np.float32)
+
+
+def test_ste_backward_dynamic_passes_unsaturated():
+    # dynamic max scales: every element whose forward code is below the E2M1
+    # maximum gets its gradient back unchanged
+    rng = np.random.default_rng(32)
+    x = torch.from_numpy((rng.standard_normal((4, 128))).astype(np.float32)).to(torch.bfloat16).float().numpy()
+    gy = np.ones_like(x)
+    gx = o.fake_quant_backward(x, gy, "max")
+    codes = o.quantize(x, "max")["codes"] & 7
+    assert np.all(gx[codes < 7] == 1.0)
