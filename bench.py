@@ -334,6 +334,15 @@ def measure_rows(nv, peaks, flush_buf, stream, iters=10):
     alg = x.numel() * 4.0
     rows["fake_quant_dynamic"] = {"workload": "X 16384x4096 BF16 -> BF16", "ms": t * 1e3, "GB/s": alg / t / 1e9,
                                   "frac_hbm": alg / t / 1e9 / hbm, "algorithmic_bytes": alg}
+    gy = torch.randn_like(x)
+    gx = torch.empty_like(x)
+    tot, _ = time_loop(lambda ev: nv.fake_quant_backward(x, gy, "max", out=gx), iters, 2, flush_buf, stream)
+    t = statistics.median(tot) * 1e-3
+    alg = x.numel() * 6.0
+    rows["qad_backward_ste_dynamic"] = {"workload": "X 16384x4096 BF16 and dL/dy BF16 -> dL/dx BF16 (clipped STE, "
+                                                    "dynamic max scales)", "ms": t * 1e3, "GB/s": alg / t / 1e9,
+                                        "frac_hbm": alg / t / 1e9 / hbm, "algorithmic_bytes": alg}
+    del gy, gx
     xq = nv.quantize(x)
     tot, _ = time_loop(lambda ev: nv.quantize(x, out=xq), iters, 2, flush_buf, stream)
     t = statistics.median(tot) * 1e-3
@@ -347,6 +356,24 @@ def measure_rows(nv, peaks, flush_buf, stream, iters=10):
     fl = 2.0 * x.shape[0] * w.shape[0] * x.shape[1]
     rows["gemm_fos_16384x14336x4096"] = {"ms": t * 1e3, "TFLOP/s": fl / t / 1e12, "frac_fp4_peak": fl / t / 1e12 / fp4_peak}
     del w, x, y, xq, wq, C
+    torch.cuda.empty_cache()
+
+    # NVFP4 KV cache: K and V of 32768 tokens x 8 heads x 128, four_over_six on
+    # write, BF16 on read (dequantize is the per-step read side)
+    kv = torch.randn((2 * 32768, 1024), device="cuda").to(torch.bfloat16)
+    kvq = nv.quantize(kv, "four_over_six")
+    kvy = torch.empty_like(kv)
+    tot, _ = time_loop(lambda ev: nv.dequantize(kvq, out=kvy), iters, 2, flush_buf, stream)
+    t = statistics.median(tot) * 1e-3
+    alg = kv.numel() * (0.5 + 1 / 16 + 2)
+    rows["kv_cache_dequantize"] = {"workload": "K,V 2x32768x1024 NVFP4 -> BF16", "ms": t * 1e3, "GB/s": alg / t / 1e9,
+                                   "frac_hbm": alg / t / 1e9 / hbm, "algorithmic_bytes": alg}
+    tot, _ = time_loop(lambda ev: nv.quantize(kv, "four_over_six", out=kvq), iters, 2, flush_buf, stream)
+    t = statistics.median(tot) * 1e-3
+    alg = kv.numel() * (2 + 0.5 + 1 / 16)
+    rows["kv_cache_quantize_fos"] = {"workload": "K,V 2x32768x1024 BF16 -> NVFP4 four_over_six", "ms": t * 1e3,
+                                     "GB/s": alg / t / 1e9, "frac_hbm": alg / t / 1e9 / hbm, "algorithmic_bytes": alg}
+    del kv, kvq, kvy
     torch.cuda.empty_cache()
 
     # lm_head decode: X 128x2048, W 151936x2048 (HBM-bound weight streaming)

@@ -171,6 +171,42 @@ nvfp4_status nvfp4_gemm(const uint8_t* Aq, const uint8_t* As, const float* ga,
                         nvfp4_stream_t stream);
 
 /*
+ * nvfp4_dequantize -- y = BF16(g * s * q) for every element of an NVFP4
+ *   tensor: the read side of an NVFP4 KV cache ("Developing Nemotron 3.5
+ *   Lightning NVFP4 with QAD using NVIDIA Model Optimizer", Table 1
+ *   "four_over_six + NVFP4 KV": K and V stored in NVFP4, QK^T in BF16).
+ *   Products d = g*s then d*q in FP32, rounded once to BF16 (nearest even),
+ *   so nvfp4_dequantize of nvfp4_quantize's output equals nvfp4_fake_quant.
+ * codes   [M][K/2] bytes (element 2j in the low nibble), device, 16-aligned.
+ * scales  tiled block scales (nvfp4_scale_bytes(M, K) bytes), device.
+ * g       device FP32 scalar.
+ * y       out [M][K] BF16, device, 16-byte aligned.
+ * Errors: NVFP4_ERR_INVALID_ARG for K % 64 != 0 or bad pointers.
+ */
+nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t M,
+                              int64_t K, void* y, nvfp4_stream_t stream);
+
+/*
+ * nvfp4_fake_quant_backward -- gradient of the QAD fake-quant w.r.t. x
+ *   ("Developing Nemotron 3.5 Lightning NVFP4 with QAD using NVIDIA Model
+ *   Optimizer", Figure 2: the gradient returns to the FP weights through
+ *   the simulated quantization; the page does not name the estimator).
+ *   Clipped straight-through estimator: grad_x = grad_y where
+ *   |x * RN(1/(g*s))| <= 6 (FP32 product) for the element's block scale s,
+ *   else 0. The scales are those nvfp4_fake_quant would use for the same
+ *   arguments: recomputed from x (dynamic, static g), or frozen g*, s*.
+ * x, grad_y   [M][K] BF16, device, 16-byte aligned.
+ * mode        MAX or FOUR_OVER_SIX (used when the scales are recomputed).
+ * g_frozen, scales_frozen, workspace: as for nvfp4_fake_quant.
+ * grad_x      out [M][K] BF16 (distinct from x and grad_y).
+ * Errors: NVFP4_ERR_INVALID_ARG for bad sizes, pointers, aliasing or mode.
+ */
+nvfp4_status nvfp4_fake_quant_backward(const void* x, const void* grad_y, int64_t M, int64_t K,
+                                       nvfp4_mode mode, const float* g_frozen,
+                                       const uint8_t* scales_frozen, void* grad_x, void* workspace,
+                                       size_t workspace_bytes, nvfp4_stream_t stream);
+
+/*
  * Routed-expert (MoE) layer in NVFP4 W4A4 -- the layer the pages quantize
  * first ("2. PTQ": routed experts are 99.2% of the quantized tensors; the
  * Qwen3.8-Flash-Next page quantizes only the fused gate_up_proj/down_proj of

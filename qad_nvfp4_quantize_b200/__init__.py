@@ -17,7 +17,7 @@ import torch
 
 __all__ = [
     "MODE_MAX", "MODE_FOUR_OVER_SIX", "NVFP4Error", "Quantized", "lib", "library_path",
-    "check_device", "scale_bytes", "quantize", "fake_quant", "gemm", "moe_grouped_gemm",
+    "check_device", "scale_bytes", "quantize", "fake_quant", "fake_quant_backward", "dequantize", "gemm", "moe_grouped_gemm",
     "moe_workspace_layout", "convert_e2m1", "convert_e4m3", "device_status", "selftest_timeout",
     "quantize_workspace_bytes", "moe_workspace_bytes", "quantize_experts", "quantize_noalloc",
 ]
@@ -60,6 +60,8 @@ _SIGS = {
     "nvfp4_quantize_workspace_bytes": (SZ, [I64, I64]),
     "nvfp4_quantize": (I32, [P, I64, I64, I32, P, P, P, P, P, P, SZ, P]),
     "nvfp4_fake_quant": (I32, [P, I64, I64, I32, P, P, P, P, SZ, P]),
+    "nvfp4_fake_quant_backward": (I32, [P, P, I64, I64, I32, P, P, P, P, SZ, P]),
+    "nvfp4_dequantize": (I32, [P, P, P, I64, I64, P, P]),
     "nvfp4_quantize_noalloc": (I32, [P, I64, I64, I32, P, P, P, P, P, P]),
     "nvfp4_gemm": (I32, [P, P, P, P, P, P, I64, I64, I64, P, P]),
     "nvfp4_moe_workspace_bytes": (SZ, [I64, I64, I64, I32, I32]),
@@ -222,6 +224,38 @@ def fake_quant(x: torch.Tensor, mode="max", g: Optional[torch.Tensor] = None,
                                 ws_bytes, _stream(dev))
     _check(st, "nvfp4_fake_quant")
     return y
+
+
+def dequantize(q: Quantized, out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """BF16 values g*s*q of an NVFP4 tensor (nvfp4_dequantize)."""
+    dev = q.codes.device
+    y = torch.empty((q.rows, q.K), dtype=torch.bfloat16, device=dev) if out is None else out
+    _check(lib().nvfp4_dequantize(_ptr(q.codes), _ptr(q.scales), _ptr(q.g), q.rows, q.K, _ptr(y), _stream(dev)),
+           "nvfp4_dequantize")
+    return y
+
+
+def fake_quant_backward(x: torch.Tensor, grad_y: torch.Tensor, mode="max", g: Optional[torch.Tensor] = None,
+                        scales: Optional[torch.Tensor] = None,
+                        out: Optional[torch.Tensor] = None) -> torch.Tensor:
+    """Gradient of fake_quant w.r.t. x, clipped straight-through
+    (nvfp4_fake_quant_backward); scales as fake_quant with the same arguments."""
+    x = _cuda(x, "x", torch.bfloat16)
+    grad_y = _cuda(grad_y, "grad_y", torch.bfloat16)
+    if grad_y.shape != x.shape:
+        raise ValueError("grad_y must have x's shape")
+    M, K = x.shape
+    dev = x.device
+    gx = torch.empty_like(x) if out is None else out
+    ws = None
+    ws_bytes = 0
+    if g is None:
+        ws_bytes = quantize_workspace_bytes(M, K)
+        ws = _workspace(dev, ws_bytes)
+    st = lib().nvfp4_fake_quant_backward(_ptr(x), _ptr(grad_y), M, K, _MODES[mode], _ptr(g), _ptr(scales),
+                                         _ptr(gx), _ptr(ws), ws_bytes, _stream(dev))
+    _check(st, "nvfp4_fake_quant_backward")
+    return gx
 
 
 def gemm(a: Quantized, b: Quantized, out: Optional[torch.Tensor] = None) -> torch.Tensor:

@@ -205,6 +205,46 @@ nvfp4_status nvfp4_convert_e4m3(const float* in, int64_t n, uint8_t* out, nvfp4_
   return launched(nvfp4::launch_convert(in, n, out, true, d->num_sms, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t M, int64_t K,
+                              void* y, nvfp4_stream_t stream) {
+  if (M < 0 || K <= 0 || K % 64) return NVFP4_ERR_INVALID_ARG;
+  if (M > 0 && (!codes || !scales || !g || !y || !aligned16(codes) || !aligned16(y))) return NVFP4_ERR_INVALID_ARG;
+  DeviceInfo* d;
+  nvfp4_status st = current_device(&d);
+  if (st != NVFP4_OK) return st;
+  if (M == 0) return NVFP4_OK;
+  return launched(nvfp4::launch_dequantize(codes, scales, g, M, K, y, d->num_sms, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvfp4_status nvfp4_fake_quant_backward(const void* x, const void* grad_y, int64_t M, int64_t K, nvfp4_mode mode,
+                                       const float* g_frozen, const uint8_t* scales_frozen, void* grad_x,
+                                       void* workspace, size_t workspace_bytes, nvfp4_stream_t stream) {
+  if (M < 0 || K <= 0 || K % 64 || (mode != NVFP4_MODE_MAX && mode != NVFP4_MODE_FOUR_OVER_SIX))
+    return NVFP4_ERR_INVALID_ARG;
+  if (scales_frozen && !g_frozen) return NVFP4_ERR_INVALID_ARG;
+  if (M > 0 && (!x || !grad_y || !grad_x || !aligned16(x) || !aligned16(grad_y) || !aligned16(grad_x) ||
+                grad_x == x || grad_x == grad_y))
+    return NVFP4_ERR_INVALID_ARG;
+  DeviceInfo* d;
+  nvfp4_status st = current_device(&d);
+  if (st != NVFP4_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const uint32_t* partial = nullptr;
+  int np = 0;
+  const bool fos = mode == NVFP4_MODE_FOUR_OVER_SIX;
+  if (!g_frozen) {
+    if (!workspace || workspace_bytes < nvfp4_quantize_workspace_bytes(M, K) || !aligned16(workspace))
+      return NVFP4_ERR_WORKSPACE;
+    const cudaError_t e = nvfp4::launch_fake_quant_bwd_fused(x, grad_y, M, K, fos, static_cast<uint32_t*>(workspace),
+                                                             grad_x, d->status, d->num_sms, s);
+    if (e != cudaErrorNotSupported) return launched(e);
+    st = run_amax(x, M * K, workspace, workspace_bytes, d->num_sms, s, &partial, &np);
+    if (st != NVFP4_OK) return st;
+  }
+  return launched(nvfp4::launch_fake_quant_bwd(x, grad_y, M, K, fos, partial, np, g_frozen, scales_frozen, grad_x,
+                                               d->status, d->num_sms, s));
+}
+
 nvfp4_status nvfp4_get_device_status(nvfp4_stream_t stream, int clear, nvfp4_status* out) {
   if (!out) return NVFP4_ERR_INVALID_ARG;
   DeviceInfo* d;

@@ -35,6 +35,15 @@ cudaError_t launch_quantize_fused(const void* x, int64_t M, int64_t K, int mode,
                                   cudaStream_t s);
 cudaError_t launch_fake_quant_fused(const void* x, int64_t M, int64_t K, bool fos, uint32_t* ws, void* y,
                                     int* status, int num_sms, cudaStream_t s);
+// y = BF16(g * s * q) from codes and tiled scales.
+cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t M, int64_t K,
+                              void* y, int num_sms, cudaStream_t s);
+// QAD backward (clipped straight-through estimator); scales as the forward.
+cudaError_t launch_fake_quant_bwd(const void* x, const void* gy, int64_t M, int64_t K, bool fos,
+                                  const uint32_t* partial, int n_partial, const float* g_static,
+                                  const uint8_t* scales_frozen, void* gx, int* status, int num_sms, cudaStream_t s);
+cudaError_t launch_fake_quant_bwd_fused(const void* x, const void* gy, int64_t M, int64_t K, bool fos, uint32_t* ws,
+                                        void* gx, int* status, int num_sms, cudaStream_t s);
 cudaError_t launch_convert(const float* in, int64_t n, uint8_t* out, bool e4m3, int num_sms,
                            cudaStream_t s);
 cudaError_t launch_selftest_timeout(uint64_t timeout_ns, int* status, cudaStream_t s);

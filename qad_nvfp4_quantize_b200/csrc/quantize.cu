@@ -235,6 +235,73 @@ struct FrozenFakeOp {
   __device__ __forceinline__ void finish() const {}
 };
 
+// QAD backward through the simulated quantization ("Developing Nemotron 3.5
+// Lightning NVFP4 with QAD using NVIDIA Model Optimizer", Figure 2: the
+// gradient returns to the FP weights through the fake-quant): a
+// straight-through estimator clipped to the quantizer's range, grad_x =
+// grad_y where |x * r| <= 6 for the block's forward r = RN(1/(g*s)), else 0.
+__device__ __forceinline__ uint32_t ste_word(uint32_t gy, f32x2 xr) {
+  float lo, hi;
+  unpack2(xr, lo, hi);
+  return gy & ((fabsf(lo) <= 6.0f ? 0x0000FFFFu : 0u) | (fabsf(hi) <= 6.0f ? 0xFFFF0000u : 0u));
+}
+
+__device__ __forceinline__ void ste_store(const uint4* gy, uint4* gx, const Chunk& c, const f32x2 (&xs)[8],
+                                          float r) {
+  if (!c.valid) return;
+  const uint4 a = ld_stream(gy + c.vec), b = ld_stream(gy + c.vec + 1);
+  const f32x2 rr = pack2(r, r);
+  gx[c.vec] = make_uint4(ste_word(a.x, mul2(xs[0], rr)), ste_word(a.y, mul2(xs[1], rr)),
+                         ste_word(a.z, mul2(xs[2], rr)), ste_word(a.w, mul2(xs[3], rr)));
+  gx[c.vec + 1] = make_uint4(ste_word(b.x, mul2(xs[4], rr)), ste_word(b.y, mul2(xs[5], rr)),
+                             ste_word(b.z, mul2(xs[6], rr)), ste_word(b.w, mul2(xs[7], rr)));
+}
+
+// Backward with the forward's scales recomputed from x (max or four_over_six).
+template <bool kFos>
+struct SteOp {
+  const uint4* gy;
+  uint4* gx;
+  int64_t M, K;
+
+  __device__ __forceinline__ void prepare(float) const {}
+  __device__ __forceinline__ void operator()(const Raw16& v, const Chunk& c, float g, int lane) const {
+    (void)lane;
+    const float bmax = block_absmax(v);
+    f32x2 xs[8];
+    unpack_block(v, xs);
+    uint32_t sc;
+    if (kFos) {
+      Block b6, b4;
+      quantize_block<false, true>(xs, bmax, g, 6.0f, b6);
+      quantize_block<false, true>(xs, bmax, g, 4.0f, b4);
+      sc = b4.err < b6.err ? b4.sc : b6.sc;
+    } else {
+      sc = block_scale_code(bmax, g, 6.0f);
+    }
+    ste_store(gy, gx, c, xs, __frcp_rn(__fmul_rn(g, scale_value(sc))));
+  }
+  __device__ __forceinline__ void finish() const {}
+};
+
+// Backward with frozen block scales s* (tiled layout) and frozen g*.
+struct FrozenSteOp {
+  const uint4* gy;
+  uint4* gx;
+  const uint8_t* scales_frozen;
+  int64_t M, K;
+
+  __device__ __forceinline__ void prepare(float) const {}
+  __device__ __forceinline__ void operator()(const Raw16& v, const Chunk& c, float g, int lane) const {
+    (void)lane;
+    const uint32_t sc = c.valid ? scales_frozen[scale_offset(c.row, c.col >> 4, K >> 6)] : 1u;
+    f32x2 xs[8];
+    unpack_block(v, xs);
+    ste_store(gy, gx, c, xs, __frcp_rn(__fmul_rn(g, scale_value(sc))));
+  }
+  __device__ __forceinline__ void finish() const {}
+};
+
 // MSE calibration ("Developing Nemotron 3.5 Lightning NVFP4 with QAD using
 // NVIDIA Model Optimizer", Table 1 "MSE"): every positive finite E4M3 code is
 // a candidate block scale; the block keeps the lowest squared error, ties to
@@ -665,6 +732,86 @@ cudaError_t launch_convert(const float* in, int64_t n, uint8_t* out, bool e4m3, 
 cudaError_t launch_selftest_timeout(uint64_t timeout_ns, int* status, cudaStream_t s) {
   note_launch();
   selftest_timeout_kernel<<<1, 32, 0, s>>>(timeout_ns, status);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fake_quant_bwd(const void* x, const void* gy, int64_t M, int64_t K, bool fos,
+                                  const uint32_t* partial, int n_partial, const float* g_static,
+                                  const uint8_t* scales_frozen, void* gx, int* status, int num_sms, cudaStream_t s) {
+  const uint4* gyv = static_cast<const uint4*>(gy);
+  uint4* gxv = static_cast<uint4*>(gx);
+  if (scales_frozen)
+    return launch_stream(x, M, K, partial, n_partial, g_static, FrozenSteOp{gyv, gxv, scales_frozen, M, K}, nullptr,
+                         status, num_sms, s);
+  if (fos)
+    return launch_stream(x, M, K, partial, n_partial, g_static, SteOp<true>{gyv, gxv, M, K}, nullptr, status,
+                         num_sms, s);
+  return launch_stream(x, M, K, partial, n_partial, g_static, SteOp<false>{gyv, gxv, M, K}, nullptr, status, num_sms,
+                       s);
+}
+
+cudaError_t launch_fake_quant_bwd_fused(const void* x, const void* gy, int64_t M, int64_t K, bool fos, uint32_t* ws,
+                                        void* gx, int* status, int num_sms, cudaStream_t s) {
+  const uint4* gyv = static_cast<const uint4*>(gy);
+  uint4* gxv = static_cast<uint4*>(gx);
+  if (fos) return launch_fused(x, M, K, ws, SteOp<true>{gyv, gxv, M, K}, nullptr, status, num_sms, s);
+  return launch_fused(x, M, K, ws, SteOp<false>{gyv, gxv, M, K}, nullptr, status, num_sms, s);
+}
+
+// ----------------------------------------------------------------------------
+// Dequantize: y = BF16(g * s * q) from stored codes and tiled scales -- the
+// read side of an NVFP4 KV cache ("Developing Nemotron 3.5 Lightning NVFP4
+// with QAD using NVIDIA Model Optimizer", Table 1 "four_over_six + NVFP4 KV":
+// K and V stored in NVFP4, QK^T kept in BF16). Same products as fake-quant
+// (d = g*s, then d*q, FP32), so dequantize(quantize(x)) == fake_quant(x).
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(kQThreads) dequantize_kernel(const uint2* __restrict__ codes,
+                                                                const uint8_t* __restrict__ scales,
+                                                                const float* __restrict__ g_ptr, int64_t M,
+                                                                int64_t K, uint64_t cpr_magic, uint4* __restrict__ y) {
+  const float g = *g_ptr;
+  const int32_t cpr = (int32_t)((K + 511) >> 9);
+  const int64_t n_chunks = M * cpr;
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (int64_t)blockIdx.x * (kQThreads / 32) + (threadIdx.x >> 5);
+  const int64_t nwarps = (int64_t)gridDim.x * (kQThreads / 32);
+  for (int64_t ch0 = warp; ch0 < n_chunks; ch0 += kUnroll * nwarps) {
+    Chunk cc[kUnroll];
+    uint2 q[kUnroll];
+    uint32_t sc[kUnroll];
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t ch = ch0 + u * nwarps;
+      cc[u] = chunk_at(ch < n_chunks ? ch : 0, cpr, cpr_magic, K, lane);
+      const bool ok = ch < n_chunks && cc[u].valid;
+      q[u] = ok ? codes[cc[u].vec >> 1] : make_uint2(0, 0);
+      sc[u] = ok ? scales[scale_offset(cc[u].row, cc[u].col >> 4, K >> 6)] : 1u;
+    }
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      if (ch0 + u * nwarps >= n_chunks) break;  // warp-uniform
+      const float d = __fmul_rn(g, scale_value(sc[u]));
+      const f32x2 dd = pack2(d, d);
+      f32x2 v[8];
+      e2m1_unpack4(q[u].x, v);
+      e2m1_unpack4(q[u].y, v + 4);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) v[i] = mul2(dd, v[i]);
+      FakeOp<false>::store_bf16x16(y, cc[u], v);
+    }
+  }
+}
+
+cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t M, int64_t K,
+                              void* y, int num_sms, cudaStream_t s) {
+  const int64_t chunks = M * ((K + 511) / 512);
+  if (chunks == 0) return cudaSuccess;
+  if (chunks >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
+  static const int occ = resident_blocks(dequantize_kernel, kQThreads, 0);
+  const int grid = grid_for(chunks, kQThreads / 32 * kUnroll, num_sms * (occ > 0 ? occ : 1));
+  note_launch();
+  dequantize_kernel<<<grid, kQThreads, 0, s>>>(reinterpret_cast<const uint2*>(codes), scales, g, M, K,
+                                               chunk_magic(K), static_cast<uint4*>(y));
   return cudaGetLastError();
 }
 

@@ -238,3 +238,50 @@ def test_mse_rejected_outside_quantize(nv):
         nv.fake_quant(x, "mse")
     with pytest.raises(nv.NVFP4Error):
         nv.quantize_noalloc(x, "mse")
+
+
+@pytest.mark.parametrize("mode", ["max", "four_over_six"])
+def test_ste_backward_dynamic_and_static(nv, mode):
+    rng = np.random.default_rng(41)
+    M, K = 130, 320
+    x = inputs.to_bf16((rng.standard_t(3, (M, K)) * 0.2).astype(np.float32))
+    gy = inputs.to_bf16(rng.standard_normal((M, K)).astype(np.float32))
+    gx = nv.fake_quant_backward(x.cuda(), gy.cuda(), mode)
+    ref = o.fake_quant_backward(bf16_np(x), bf16_np(gy), mode)
+    np.testing.assert_array_equal(bf16_np(gx), ref)
+    # static g: the scales are recomputed from x under the given g; with g
+    # below amax/2688 many blocks saturate at E4M3 448 and clip
+    g = np.float32(0.1 / 2688)
+    gx = nv.fake_quant_backward(x.cuda(), gy.cuda(), mode, g=torch.tensor([g]).cuda())
+    q = o.quantize(bf16_np(x), mode, g)
+    ref = o.fake_quant_backward(bf16_np(x), bf16_np(gy), g_frozen=g, scales_frozen=q["scales"])
+    np.testing.assert_array_equal(bf16_np(gx), ref)
+    assert (ref == 0).any()
+
+
+def test_ste_backward_frozen_scales(nv):
+    rng = np.random.default_rng(42)
+    M, K = 200, 512
+    w0 = inputs.to_bf16((rng.standard_normal((M, K)) * 0.02).astype(np.float32))
+    q0 = nv.quantize(w0.cuda(), "four_over_six")                # calibrated once (PTQ)
+    w1 = inputs.to_bf16((bf16_np(w0) * 1.3 + rng.standard_normal((M, K)) * 0.004).astype(np.float32))
+    gy = inputs.to_bf16(rng.standard_normal((M, K)).astype(np.float32))
+    gx = nv.fake_quant_backward(w1.cuda(), gy.cuda(), g=q0.g, scales=q0.scales)
+    sc = o.scales_from_tiled(to_np(q0.scales), M, K)
+    ref = o.fake_quant_backward(bf16_np(w1), bf16_np(gy), g_frozen=to_np(q0.g)[0], scales_frozen=sc)
+    np.testing.assert_array_equal(bf16_np(gx), ref)
+    assert (ref == 0).any() and (ref != 0).any()
+
+
+def test_kv_cache_round_trip(nv):
+    # K / V of 8 KV heads x 128 dims per token, NVFP4 (four_over_six) in the
+    # cache, BF16 on read: equals the oracle and the GPU fake-quant
+    rng = np.random.default_rng(52)
+    for T in (1, 300):
+        kv = inputs.to_bf16((rng.standard_normal((T, 1024)) * 0.7).astype(np.float32))
+        q = nv.quantize(kv.cuda(), "four_over_six")
+        y = nv.dequantize(q)
+        ref = o.fake_quant(bf16_np(kv), "four_over_six")
+        np.testing.assert_array_equal(bf16_np(y), ref)
+        np.testing.assert_array_equal(to_np(y.view(torch.int16)),
+                                      to_np(nv.fake_quant(kv.cuda(), "four_over_six").view(torch.int16)))

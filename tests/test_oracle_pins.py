@@ -524,3 +524,22 @@ def test_ste_backward_dynamic_passes_unsaturated():
     gx = o.fake_quant_backward(x, gy, "max")
     codes = o.quantize(x, "max")["codes"] & 7
     assert np.all(gx[codes < 7] == 1.0)
+
+
+# ------------------------------------------------------------- dequantize ---
+
+def test_dequantize_closed_form_and_round_trip():
+    # code 7 (6.0) x scale 448 (code 0x7E) x g = 1 -> 2688; code 0xF -> -2688;
+    # code 1 (0.5) x scale 2^-9 (code 1) x g = 0.5 -> 2^-11
+    codes = np.zeros((1, 16), np.uint8)
+    codes[0, :3] = [7, 0xF, 1]
+    v = o.dequantize(codes, np.array([[0x7E]], np.uint8), np.float32(1.0))
+    assert v[0, 0] == 2688.0 and v[0, 1] == -2688.0 and v[0, 2] == 0.5 * 448.0
+    v = o.dequantize(codes, np.array([[1]], np.uint8), np.float32(0.5))
+    assert v[0, 2] == np.float32(2.0 ** -11)
+    # storing K/V in NVFP4 and reading them back is the fake-quant forward
+    rng = np.random.default_rng(51)
+    x = torch.from_numpy(rng.standard_normal((8, 128)).astype(np.float32)).to(torch.bfloat16).float().numpy()
+    for mode in ("max", "four_over_six"):
+        q = o.quantize(x, mode)
+        assert np.array_equal(o.bf16_round(o.dequantize(q["codes"], q["scales"], q["g"])), o.fake_quant(x, mode))
