@@ -53,6 +53,14 @@ R11 QAD backward through the simulated quantization ([NEMO-QAD] Figure 2:
     dL/dx = dL/dy where |x * r| <= 6 for the block's r = RN(1/(g*s)) (FP32
     product), else 0. Rounding is passed straight through; saturation is not.
     The scales are those of the forward: recomputed (dynamic) or frozen.
+R12 Top-k logit KL ([P1] "QAD": "--logit_kl_topk 4096" restricts the KD loss
+    to the teacher's top-4096 vocabulary entries; the loss compares teacher
+    and student logits element-wise over the vocabulary): per row, the k
+    entries with the largest teacher logits (ties to the lower index) form
+    the set; teacher and student distributions are softmax over that set
+    (temperature 1, the pages give none); loss = KL(teacher || student) =
+    sum p_t (log p_t - log p_s); its gradient w.r.t. the student logits on
+    the set is p_s - p_t (0 elsewhere).
 R10 MSE calibration ([NEMO-QAD] Table 1 "MSE"; "Quantization scale handling
     during QAD": MSE reaches its scales by a search that minimises the
     quantization error): for each block, every positive finite E4M3 code
@@ -345,6 +353,38 @@ def fake_quant_backward(x: np.ndarray, grad_y: np.ndarray, mode: str = "max", g_
     v = x.reshape(rows, K // BLOCK, BLOCK) * r[..., None]               # FP32 products
     inside = (np.abs(v) <= np.float32(E2M1_MAX)).reshape(rows, K)
     return np.where(inside, gy, np.float32(0.0)).astype(np.float32)
+
+
+def topk_kl(teacher: np.ndarray, student: np.ndarray, k: int):
+    """Top-k logit KL distillation loss per row (R12), in FP64.
+
+    teacher, student: [rows, V] logits (BF16 values). Returns a dict with
+      loss  float64 [rows]      KL(p_t || p_s) over the teacher's top-k set
+      idx   int64 [rows, k]     the set, ascending vocabulary index
+      grad  float64 [rows, k]   d loss / d student logit at idx
+      lse_t, lse_s float64 [rows]  log-sum-exp of each side over the set
+    """
+    t = np.asarray(teacher, dtype=np.float64)
+    s = np.asarray(student, dtype=np.float64)
+    rows, V = t.shape
+    if not 1 <= k <= V:
+        raise ValueError("need 1 <= k <= V")
+    out = dict(loss=np.empty(rows), idx=np.empty((rows, k), np.int64), grad=np.empty((rows, k)),
+               lse_t=np.empty(rows), lse_s=np.empty(rows))
+    for r in range(rows):
+        order = np.argsort(-t[r], kind="stable")   # descending; equal logits keep index order
+        idx = np.sort(order[:k])
+        tt, ss = t[r, idx], s[r, idx]
+        mt, ms = tt.max(), ss.max()
+        lse_t = mt + np.log(np.sum(np.exp(tt - mt)))
+        lse_s = ms + np.log(np.sum(np.exp(ss - ms)))
+        lpt, lps = tt - lse_t, ss - lse_s
+        pt = np.exp(lpt)
+        out["loss"][r] = np.sum(pt * (lpt - lps))
+        out["idx"][r] = idx
+        out["grad"][r] = np.exp(lps) - pt
+        out["lse_t"][r], out["lse_s"][r] = lse_t, lse_s
+    return out
 
 
 # ----------------------------------------------------------------------------

@@ -86,3 +86,15 @@ def moe_experts(seed: int = 0, T: int = 8192, H: int = 2048, E: int = 256, topk:
 def bf16_to_f32(t: torch.Tensor) -> np.ndarray:
     """BF16 torch tensor -> FP32 numpy array with the same values."""
     return t.detach().to("cpu").to(torch.float32).numpy()
+
+
+def kd_logits(seed: int = 0, rows: int = 2048, V: int = 248320, k_peaked: int = 64):
+    """Teacher / student logits for the top-k KL loss ([P1] "QAD", vocabulary of
+    248,320 entries): teacher = N(0, 2) with k_peaked entries per row raised
+    by 8 (a peaked distribution), student = teacher + N(0, 0.5); both BF16."""
+    rt, rp, rs = _streams(seed, 3)
+    t = normal(rt, (rows, V), 2.0)
+    for r in range(rows):
+        t[r, rp.choice(V, size=k_peaked, replace=False)] += np.float32(8.0)
+    s = t + normal(rs, (rows, V), 0.5)
+    return dict(teacher=to_bf16(t), student=to_bf16(s))

@@ -543,3 +543,46 @@ def test_dequantize_closed_form_and_round_trip():
     for mode in ("max", "four_over_six"):
         q = o.quantize(x, mode)
         assert np.array_equal(o.bf16_round(o.dequantize(q["codes"], q["scales"], q["g"])), o.fake_quant(x, mode))
+
+
+# ------------------------------------------------------------- top-k KL ---
+
+def test_topk_kl_full_vocab_equals_library_kl():
+    from scipy.special import rel_entr, softmax
+    rng = np.random.default_rng(61)
+    t = rng.standard_normal((3, 50)) * 2
+    s = t + rng.standard_normal((3, 50)) * 0.5
+    out = o.topk_kl(t, s, 50)
+    want = rel_entr(softmax(t, axis=1), softmax(s, axis=1)).sum(axis=1)
+    assert np.allclose(out["loss"], want, rtol=1e-12, atol=1e-14)
+
+
+def test_topk_kl_set_ties_and_zero_loss():
+    t = np.array([[1.0, 3.0, 3.0, 2.0, 3.0]])
+    out = o.topk_kl(t, t, 2)
+    assert out["idx"].tolist() == [[1, 2]]                 # three 3s: the two lowest indices
+    assert out["loss"][0] == 0.0 and np.all(out["grad"] == 0.0)
+    out = o.topk_kl(t, t * 0.5, 4)
+    assert out["idx"].tolist() == [[1, 2, 3, 4]]
+
+
+def test_topk_kl_matches_renormalised_library_kl_and_gradient():
+    from scipy.special import rel_entr, softmax
+    rng = np.random.default_rng(62)
+    V, k = 40, 7
+    t = np.round(rng.standard_normal((4, V)) * 3) / 2       # many ties
+    s = rng.standard_normal((4, V))
+    out = o.topk_kl(t, s, k)
+    for r in range(4):
+        idx = out["idx"][r]
+        rest = np.setdiff1d(np.arange(V), idx)
+        assert t[r, idx].min() >= t[r, rest].max()          # brute-force set property
+        assert np.isclose(out["loss"][r], rel_entr(softmax(t[r, idx]), softmax(s[r, idx])).sum(), rtol=1e-12)
+        # gradient by central differences of the loss in each student logit
+        for j in range(k):
+            h = 1e-6
+            sp, sm = s.copy(), s.copy()
+            sp[r, idx[j]] += h
+            sm[r, idx[j]] -= h
+            fd = (o.topk_kl(t[r:r + 1], sp[r:r + 1], k)["loss"][0] - o.topk_kl(t[r:r + 1], sm[r:r + 1], k)["loss"][0]) / (2 * h)
+            assert abs(fd - out["grad"][r, j]) < 1e-7
