@@ -376,6 +376,24 @@ def measure_rows(nv, peaks, flush_buf, stream, iters=10):
     del kv, kvq, kvy
     torch.cuda.empty_cache()
 
+    # top-k logit KL: 2048 positions x 248,320-entry vocabulary, teacher top-4096
+    gen = torch.Generator(device="cuda").manual_seed(7)
+    R, V = 2048, 248320
+    tl = torch.randn((R, V), device="cuda", generator=gen) * 2.0
+    tl.scatter_add_(1, torch.randint(0, V, (R, 64), device="cuda", generator=gen),
+                    torch.full((R, 64), 8.0, device="cuda"))
+    sl = (tl + torch.randn((R, V), device="cuda", generator=gen) * 0.5).to(torch.bfloat16)
+    tl = tl.to(torch.bfloat16)
+    kl = torch.empty(R, dtype=torch.float32, device="cuda")
+    tot, _ = time_loop(lambda ev: nv.topk_kl(tl, sl, 4096, loss_out=kl), iters, 2, flush_buf, stream)
+    t = statistics.median(tot) * 1e-3
+    alg = 2.0 * R * V * 2
+    rows["kd_topk_kl"] = {"workload": "2048 x 248320 BF16 teacher/student logits, top-4096 KL per row",
+                          "ms": t * 1e3, "GB/s": alg / t / 1e9, "frac_hbm": alg / t / 1e9 / hbm,
+                          "algorithmic_bytes": alg}
+    del tl, sl, kl
+    torch.cuda.empty_cache()
+
     # lm_head decode: X 128x2048, W 151936x2048 (HBM-bound weight streaming)
     d = inputs.lm_head(0)
     w = d["w"].cuda()

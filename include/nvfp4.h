@@ -171,6 +171,26 @@ nvfp4_status nvfp4_gemm(const uint8_t* Aq, const uint8_t* As, const float* ga,
                         nvfp4_stream_t stream);
 
 /*
+ * nvfp4_topk_kl -- top-k logit KL distillation loss per row ("Model-Optimizer
+ *   in practice: recovering Qwen3.6-35B-A3B W4A4 NVFP4 accuracy with QAD",
+ *   section "QAD", --logit_kl_topk: the KD loss restricted to the teacher's
+ *   top-k vocabulary entries, no dense [rows x V] FP32 tensor). Per row: the
+ *   set is the k largest teacher logits (ties to the lower index); p_t, p_s
+ *   are softmax of teacher and student logits over the set (temperature 1);
+ *   loss = KL(p_t || p_s); gradient w.r.t. the student logits = p_s - p_t on
+ *   the set. FP32 arithmetic with exp/log.
+ * teacher, student  [rows][V] BF16, device, 16-byte aligned; V % 8 == 0.
+ * k         1 <= k <= V.
+ * loss      out FP32 [rows], device.
+ * idx       nullable out int32 [rows][k]: the set, ascending index.
+ * grad      nullable out FP32 [rows][k]: d loss / d student logit at idx
+ *           (needs idx).
+ * Errors: NVFP4_ERR_INVALID_ARG for bad sizes or pointers.
+ */
+nvfp4_status nvfp4_topk_kl(const void* teacher, const void* student, int64_t rows, int64_t V, int k,
+                           float* loss, int32_t* idx, float* grad, nvfp4_stream_t stream);
+
+/*
  * nvfp4_dequantize -- y = BF16(g * s * q) for every element of an NVFP4
  *   tensor: the read side of an NVFP4 KV cache ("Developing Nemotron 3.5
  *   Lightning NVFP4 with QAD using NVIDIA Model Optimizer", Table 1

@@ -17,7 +17,7 @@ import torch
 
 __all__ = [
     "MODE_MAX", "MODE_FOUR_OVER_SIX", "NVFP4Error", "Quantized", "lib", "library_path",
-    "check_device", "scale_bytes", "quantize", "fake_quant", "fake_quant_backward", "dequantize", "gemm", "moe_grouped_gemm",
+    "check_device", "scale_bytes", "quantize", "fake_quant", "fake_quant_backward", "dequantize", "topk_kl", "gemm", "moe_grouped_gemm",
     "moe_workspace_layout", "convert_e2m1", "convert_e4m3", "device_status", "selftest_timeout",
     "quantize_workspace_bytes", "moe_workspace_bytes", "quantize_experts", "quantize_noalloc",
 ]
@@ -62,6 +62,7 @@ _SIGS = {
     "nvfp4_fake_quant": (I32, [P, I64, I64, I32, P, P, P, P, SZ, P]),
     "nvfp4_fake_quant_backward": (I32, [P, P, I64, I64, I32, P, P, P, P, SZ, P]),
     "nvfp4_dequantize": (I32, [P, P, P, I64, I64, P, P]),
+    "nvfp4_topk_kl": (I32, [P, P, I64, I64, I32, P, P, P, P]),
     "nvfp4_quantize_noalloc": (I32, [P, I64, I64, I32, P, P, P, P, P, P]),
     "nvfp4_gemm": (I32, [P, P, P, P, P, P, I64, I64, I64, P, P]),
     "nvfp4_moe_workspace_bytes": (SZ, [I64, I64, I64, I32, I32]),
@@ -224,6 +225,24 @@ def fake_quant(x: torch.Tensor, mode="max", g: Optional[torch.Tensor] = None,
                                 ws_bytes, _stream(dev))
     _check(st, "nvfp4_fake_quant")
     return y
+
+
+def topk_kl(teacher: torch.Tensor, student: torch.Tensor, k: int, want_idx: bool = False,
+            want_grad: bool = False, loss_out: Optional[torch.Tensor] = None):
+    """Top-k logit KL distillation loss per row (nvfp4_topk_kl). Returns
+    (loss [rows] FP32, idx [rows, k] int32 or None, grad [rows, k] FP32 or None)."""
+    teacher = _cuda(teacher, "teacher", torch.bfloat16)
+    student = _cuda(student, "student", torch.bfloat16)
+    if teacher.shape != student.shape or teacher.dim() != 2:
+        raise ValueError("teacher and student must be equal [rows, V]")
+    rows, V = teacher.shape
+    dev = teacher.device
+    loss = torch.empty(rows, dtype=torch.float32, device=dev) if loss_out is None else loss_out
+    idx = torch.empty((rows, k), dtype=torch.int32, device=dev) if (want_idx or want_grad) else None
+    grad = torch.empty((rows, k), dtype=torch.float32, device=dev) if want_grad else None
+    _check(lib().nvfp4_topk_kl(_ptr(teacher), _ptr(student), rows, V, k, _ptr(loss), _ptr(idx), _ptr(grad),
+                               _stream(dev)), "nvfp4_topk_kl")
+    return loss, idx, grad
 
 
 def dequantize(q: Quantized, out: Optional[torch.Tensor] = None) -> torch.Tensor:

@@ -205,6 +205,18 @@ nvfp4_status nvfp4_convert_e4m3(const float* in, int64_t n, uint8_t* out, nvfp4_
   return launched(nvfp4::launch_convert(in, n, out, true, d->num_sms, reinterpret_cast<cudaStream_t>(stream)));
 }
 
+nvfp4_status nvfp4_topk_kl(const void* teacher, const void* student, int64_t rows, int64_t V, int k, float* loss,
+                           int32_t* idx, float* grad, nvfp4_stream_t stream) {
+  if (rows < 0 || V <= 0 || V % 8 || k < 1 || k > V || (grad && !idx)) return NVFP4_ERR_INVALID_ARG;
+  if (rows > 0 && (!teacher || !student || !loss || !aligned16(teacher) || !aligned16(student)))
+    return NVFP4_ERR_INVALID_ARG;
+  DeviceInfo* d;
+  nvfp4_status st = current_device(&d);
+  if (st != NVFP4_OK) return st;
+  return launched(nvfp4::launch_topk_kl(teacher, student, rows, V, k, loss, idx, grad, d->num_sms,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
 nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t M, int64_t K,
                               void* y, nvfp4_stream_t stream) {
   if (M < 0 || K <= 0 || K % 64) return NVFP4_ERR_INVALID_ARG;

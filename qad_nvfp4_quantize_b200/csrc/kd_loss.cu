@@ -1,0 +1,319 @@
+// Top-k logit KL distillation loss ("Model-Optimizer in practice: recovering
+// Qwen3.6-35B-A3B W4A4 NVFP4 accuracy with QAD", section "QAD":
+// --logit_kl_topk 4096 restricts the KD loss to the teacher's top-4096
+// vocabulary entries, so no dense [seq x vocab] FP32 tensor is formed).
+//
+// Per row: the set is the k entries with the largest teacher logits (ties to
+// the lower index); teacher and student distributions are softmax over the
+// set; loss = KL(p_t || p_s) = sum p_t (t - s) - lse_t + lse_s with
+// p_t = exp(t - lse_t); d loss / d s = p_s - p_t on the set.
+//
+// One CTA of 1024 threads per row (persistent over rows). The set is found
+// by a two-digit radix select on order-preserving 16-bit keys of the BF16
+// teacher logits (high byte, then low byte among the high-byte bin that holds
+// the k-th largest), which gives the threshold key T, the count above it, and
+// how many entries equal to T the set takes (the lowest indices). A third
+// pass walks the row in index order, ranks the entries equal to T with a
+// block scan, and accumulates the two log-sum-exps and sum p_t (t - s)
+// online (rescaled when the running maximum grows). Histograms use
+// warp-aggregated shared atomics (__match_any_sync), since logits concentrate
+// in few bins.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace nvfp4 {
+
+constexpr int kKdThreads = 1024;
+constexpr int kKdWarps = kKdThreads / 32;
+
+// BF16 bits -> key whose unsigned order is the value order (-0 maps to +0).
+__device__ __forceinline__ uint32_t kd_key(uint32_t b) {
+  b &= 0xFFFFu;
+  if (b == 0x8000u) b = 0u;
+  return (b & 0x8000u) ? (~b & 0xFFFFu) : (b | 0x8000u);
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+struct KdShared {
+  uint32_t hist[256];
+  uint32_t scan[kKdWarps];
+  uint32_t bin, above;      // find_bin result
+  uint32_t eq_base, sel_base;
+  float red[kKdWarps][5];
+};
+
+// Warp-aggregated histogram add: lanes with equal bins add once.
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool active, int lane) {
+  const uint32_t key = active ? bin : 0xFFFFFFFFu;
+  const unsigned peers = __match_any_sync(0xFFFFFFFFu, key);
+  if (active && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+}
+
+// Bin b where the count of entries in bins >= b first reaches `need` (need >=
+// 1 and at most the histogram total); also the count strictly above b. Called
+// by all threads; reads sh.hist, writes sh.bin / sh.above.
+__device__ __forceinline__ void find_bin(KdShared& sh, uint32_t need) {
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  uint32_t suf = 0, own = 0;
+  if (t < 256) {
+    own = sh.hist[t];
+    suf = own;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t v = __shfl_down_sync(0xFFFFFFFFu, suf, o);
+      if (lane + o < 32) suf += v;
+    }
+    if (lane == 0) sh.scan[warp] = suf;  // warp total
+  }
+  __syncthreads();
+  if (t < 256) {
+    for (int w = warp + 1; w < 8; ++w) suf += sh.scan[w];
+    if (suf >= need && suf - own < need) {
+      sh.bin = (uint32_t)t;
+      sh.above = suf - own;
+    }
+  }
+  __syncthreads();
+}
+
+// Block-wide exclusive scan of v (1024 threads); returns the exclusive prefix
+// and writes the block total to *total.
+__device__ __forceinline__ uint32_t block_scan(KdShared& sh, uint32_t v, uint32_t* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  uint32_t incl = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    if (lane >= o) incl += u;
+  }
+  if (lane == 31) sh.scan[warp] = incl;
+  __syncthreads();
+  if (warp == 0) {
+    uint32_t w = sh.scan[lane];
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, w, o);
+      if (lane >= o) w += u;
+    }
+    sh.scan[lane] = w;
+  }
+  __syncthreads();
+  const uint32_t excl = incl - v + (warp > 0 ? sh.scan[warp - 1] : 0u);
+  *total = sh.scan[kKdWarps - 1];
+  __syncthreads();  // sh.scan is reused by the next scan
+  return excl;
+}
+
+// Online log-sum-exp state with the teacher-weighted sum of (t - s).
+struct KdAcc {
+  float mt, zt, a, ms, zs;
+  __device__ __forceinline__ void init() {
+    mt = ms = -INFINITY;
+    zt = a = zs = 0.0f;
+  }
+  __device__ __forceinline__ void add(float t, float s) {
+    if (t > mt) {
+      const float c = mt == -INFINITY ? 0.0f : expf(mt - t);
+      zt = zt * c + 1.0f;
+      a = a * c + (t - s);
+      mt = t;
+    } else {
+      const float w = expf(t - mt);
+      zt += w;
+      a += w * (t - s);
+    }
+    if (s > ms) {
+      zs = zs * (ms == -INFINITY ? 0.0f : expf(ms - s)) + 1.0f;
+      ms = s;
+    } else {
+      zs += expf(s - ms);
+    }
+  }
+  __device__ __forceinline__ void merge(const KdAcc& o) {
+    if (o.mt != -INFINITY) {
+      const float m = fmaxf(mt, o.mt);
+      const float c1 = mt == -INFINITY ? 0.0f : expf(mt - m), c2 = expf(o.mt - m);
+      zt = zt * c1 + o.zt * c2;
+      a = a * c1 + o.a * c2;
+      mt = m;
+    }
+    if (o.ms != -INFINITY) {
+      const float m = fmaxf(ms, o.ms);
+      zs = zs * (ms == -INFINITY ? 0.0f : expf(ms - m)) + o.zs * expf(o.ms - m);
+      ms = m;
+    }
+  }
+};
+
+__global__ void __launch_bounds__(kKdThreads, 1) topk_kl_kernel(const uint4* __restrict__ teacher,
+                                                                 const uint4* __restrict__ student, int64_t rows,
+                                                                 int64_t V, int k, float* __restrict__ loss,
+                                                                 int32_t* __restrict__ idx_out,
+                                                                 float* __restrict__ grad_out) {
+  __shared__ KdShared sh;
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const int64_t nvec = V / 8;
+  const int64_t trips = (nvec + kKdThreads - 1) / kKdThreads;
+  for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
+    const uint4* trow = teacher + row * nvec;
+    const uint4* srow = student + row * nvec;
+
+    // ---- pass 1: histogram of the key's high byte
+    for (int i = t; i < 256; i += kKdThreads) sh.hist[i] = 0u;
+    __syncthreads();
+    for (int64_t it = 0; it < trips; ++it) {
+      const int64_t j = it * kKdThreads + t;
+      const bool act = j < nvec;
+      const uint4 v = act ? trow[j] : make_uint4(0, 0, 0, 0);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        hist_add(sh.hist, kd_key(w[e]) >> 8, act, lane);
+        hist_add(sh.hist, kd_key(w[e] >> 16) >> 8, act, lane);
+      }
+    }
+    __syncthreads();
+    find_bin(sh, (uint32_t)k);
+    const uint32_t b1 = sh.bin, above1 = sh.above;
+    __syncthreads();
+
+    // ---- pass 2: histogram of the low byte inside bin b1
+    for (int i = t; i < 256; i += kKdThreads) sh.hist[i] = 0u;
+    __syncthreads();
+    for (int64_t it = 0; it < trips; ++it) {
+      const int64_t j = it * kKdThreads + t;
+      const bool act = j < nvec;
+      const uint4 v = act ? trow[j] : make_uint4(0, 0, 0, 0);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t k0 = kd_key(w[e]), k1 = kd_key(w[e] >> 16);
+        hist_add(sh.hist, k0 & 0xFFu, act && (k0 >> 8) == b1, lane);
+        hist_add(sh.hist, k1 & 0xFFu, act && (k1 >> 8) == b1, lane);
+      }
+    }
+    __syncthreads();
+    find_bin(sh, (uint32_t)k - above1);
+    const uint32_t T = (b1 << 8) | sh.bin;
+    const uint32_t need_eq = (uint32_t)k - (above1 + sh.above);  // entries equal to T taken
+    if (t == 0) {
+      sh.eq_base = 0u;
+      sh.sel_base = 0u;
+    }
+    __syncthreads();
+
+    // ---- pass 3: select in index order, accumulate
+    KdAcc acc;
+    acc.init();
+    for (int64_t it = 0; it < trips; ++it) {
+      const int64_t j = it * kKdThreads + t;
+      const bool act = j < nvec;
+      const uint4 v = act ? trow[j] : make_uint4(0, 0, 0, 0);
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      uint32_t keys[8];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        keys[2 * e] = act ? kd_key(w[e]) : 0u;
+        keys[2 * e + 1] = act ? kd_key(w[e] >> 16) : 0u;
+      }
+      uint32_t n_eq = 0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) n_eq += keys[e] == T && act;
+      uint32_t tot_eq;
+      const uint32_t eq_rank0 = sh.eq_base + block_scan(sh, n_eq, &tot_eq);
+      uint32_t selmask = 0, r = eq_rank0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const bool eq = act && keys[e] == T;
+        const bool sel = act && (keys[e] > T || (eq && r < need_eq));
+        r += eq;
+        selmask |= (uint32_t)sel << e;
+      }
+      uint32_t tot_sel = 0, pos = 0;
+      if (idx_out) pos = sh.sel_base + block_scan(sh, (uint32_t)__popc(selmask), &tot_sel);
+      if (selmask) {
+        const uint4 sv = srow[j];
+        const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          if (!((selmask >> e) & 1u)) continue;
+          const float tv = (e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]);
+          const float svv = (e & 1) ? bf16_hi(sw[e >> 1]) : bf16_lo(sw[e >> 1]);
+          acc.add(tv, svv);
+          if (idx_out) idx_out[row * k + pos++] = (int32_t)(8 * j + e);
+        }
+      }
+      __syncthreads();  // everyone has read eq_base / sel_base
+      if (t == 0) {
+        sh.eq_base += tot_eq;
+        if (idx_out) sh.sel_base += tot_sel;
+      }
+      __syncthreads();
+    }
+
+    // ---- block reduction of the accumulators
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      KdAcc other;
+      other.mt = __shfl_xor_sync(0xFFFFFFFFu, acc.mt, o);
+      other.zt = __shfl_xor_sync(0xFFFFFFFFu, acc.zt, o);
+      other.a = __shfl_xor_sync(0xFFFFFFFFu, acc.a, o);
+      other.ms = __shfl_xor_sync(0xFFFFFFFFu, acc.ms, o);
+      other.zs = __shfl_xor_sync(0xFFFFFFFFu, acc.zs, o);
+      acc.merge(other);
+    }
+    if (lane == 0) {
+      sh.red[warp][0] = acc.mt;
+      sh.red[warp][1] = acc.zt;
+      sh.red[warp][2] = acc.a;
+      sh.red[warp][3] = acc.ms;
+      sh.red[warp][4] = acc.zs;
+    }
+    __syncthreads();
+    if (t == 0) {
+      KdAcc tot;
+      tot.init();
+      for (int w2 = 0; w2 < kKdWarps; ++w2) {
+        KdAcc o;
+        o.mt = sh.red[w2][0];
+        o.zt = sh.red[w2][1];
+        o.a = sh.red[w2][2];
+        o.ms = sh.red[w2][3];
+        o.zs = sh.red[w2][4];
+        tot.merge(o);
+      }
+      const float lse_t = tot.mt + logf(tot.zt), lse_s = tot.ms + logf(tot.zs);
+      loss[row] = tot.a / tot.zt - lse_t + lse_s;
+      sh.red[0][0] = lse_t;
+      sh.red[0][1] = lse_s;
+    }
+    __syncthreads();
+
+    // ---- optional pass 4: gradient p_s - p_t at the selected entries
+    if (grad_out && idx_out) {
+      const float lse_t = sh.red[0][0], lse_s = sh.red[0][1];
+      const uint16_t* t16 = reinterpret_cast<const uint16_t*>(trow);
+      const uint16_t* s16 = reinterpret_cast<const uint16_t*>(srow);
+      for (int i = t; i < k; i += kKdThreads) {
+        const int32_t v = idx_out[row * k + i];
+        const float tv = __uint_as_float((uint32_t)t16[v] << 16), svv = __uint_as_float((uint32_t)s16[v] << 16);
+        grad_out[row * k + i] = expf(svv - lse_s) - expf(tv - lse_t);
+      }
+    }
+    __syncthreads();
+  }
+}
+
+cudaError_t launch_topk_kl(const void* teacher, const void* student, int64_t rows, int64_t V, int k, float* loss,
+                           int32_t* idx, float* grad, int num_sms, cudaStream_t s) {
+  if (rows == 0) return cudaSuccess;
+  const int grid = (int)(rows < num_sms ? rows : num_sms);
+  note_launch();
+  topk_kl_kernel<<<grid, kKdThreads, 0, s>>>(static_cast<const uint4*>(teacher), static_cast<const uint4*>(student),
+                                             rows, V, k, loss, idx, grad);
+  return cudaGetLastError();
+}
+
+}  // namespace nvfp4
