@@ -15,9 +15,9 @@
 // how many entries equal to T the set takes (the lowest indices). A third
 // pass walks the row in index order, ranks the entries equal to T with a
 // block scan, and accumulates the two log-sum-exps and sum p_t (t - s)
-// online (rescaled when the running maximum grows). Histograms use
-// warp-aggregated shared atomics (__match_any_sync), since logits concentrate
-// in few bins.
+// online (rescaled when the running maximum grows). The histograms are
+// per warp (shared-memory atomics; logits concentrate in few bins, so warps
+// must not share counters). Loads run kKdUnroll trips ahead.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -25,6 +25,7 @@ namespace nvfp4 {
 
 constexpr int kKdThreads = 1024;
 constexpr int kKdWarps = kKdThreads / 32;
+constexpr int kKdUnroll = 4;  // 16-byte loads in flight per thread in the histogram passes
 
 // BF16 bits -> key whose unsigned order is the value order (-0 maps to +0).
 __device__ __forceinline__ uint32_t kd_key(uint32_t b) {
@@ -37,6 +38,7 @@ __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w 
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
 struct KdShared {
+  uint32_t whist[kKdWarps][256];  // per-warp histograms (no cross-warp contention)
   uint32_t hist[256];
   uint32_t scan[kKdWarps];
   uint32_t bin, above;      // find_bin result
@@ -44,11 +46,22 @@ struct KdShared {
   float red[kKdWarps][5];
 };
 
-// Warp-aggregated histogram add: lanes with equal bins add once.
-__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool active, int lane) {
-  const uint32_t key = active ? bin : 0xFFFFFFFFu;
-  const unsigned peers = __match_any_sync(0xFFFFFFFFu, key);
-  if (active && lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+// Histogram add into this warp's own histogram (lanes of one warp that hit
+// the same bin are serialised by the shared-memory atomic unit; no other
+// warp touches these counters).
+__device__ __forceinline__ void hist_add(uint32_t* hist, uint32_t bin, bool active) {
+  if (active) atomicAdd(&hist[bin], 1u);
+}
+
+// hist[b] = sum over warps of whist[w][b].
+__device__ __forceinline__ void reduce_hist(KdShared& sh) {
+  if (threadIdx.x < 256) {
+    uint32_t c = 0;
+#pragma unroll 8
+    for (int w = 0; w < kKdWarps; ++w) c += sh.whist[w][threadIdx.x];
+    sh.hist[threadIdx.x] = c;
+  }
+  __syncthreads();
 }
 
 // Bin b where the count of entries in bins >= b first reaches `need` (need >=
@@ -161,40 +174,56 @@ __global__ void __launch_bounds__(kKdThreads, 1) topk_kl_kernel(const uint4* __r
     const uint4* srow = student + row * nvec;
 
     // ---- pass 1: histogram of the key's high byte
-    for (int i = t; i < 256; i += kKdThreads) sh.hist[i] = 0u;
+    for (int i = t; i < kKdWarps * 256; i += kKdThreads) (&sh.whist[0][0])[i] = 0u;
     __syncthreads();
-    for (int64_t it = 0; it < trips; ++it) {
-      const int64_t j = it * kKdThreads + t;
-      const bool act = j < nvec;
-      const uint4 v = act ? trow[j] : make_uint4(0, 0, 0, 0);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    for (int64_t it = 0; it < trips; it += kKdUnroll) {
+      uint4 v[kKdUnroll];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        hist_add(sh.hist, kd_key(w[e]) >> 8, act, lane);
-        hist_add(sh.hist, kd_key(w[e] >> 16) >> 8, act, lane);
+      for (int u = 0; u < kKdUnroll; ++u) {
+        const int64_t j = (it + u) * kKdThreads + t;
+        v[u] = j < nvec ? trow[j] : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < kKdUnroll; ++u) {
+        const bool act = (it + u) * kKdThreads + t < nvec;
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          hist_add(sh.whist[warp], kd_key(w[e]) >> 8, act);
+          hist_add(sh.whist[warp], kd_key(w[e] >> 16) >> 8, act);
+        }
       }
     }
     __syncthreads();
+    reduce_hist(sh);
     find_bin(sh, (uint32_t)k);
     const uint32_t b1 = sh.bin, above1 = sh.above;
     __syncthreads();
 
     // ---- pass 2: histogram of the low byte inside bin b1
-    for (int i = t; i < 256; i += kKdThreads) sh.hist[i] = 0u;
+    for (int i = t; i < kKdWarps * 256; i += kKdThreads) (&sh.whist[0][0])[i] = 0u;
     __syncthreads();
-    for (int64_t it = 0; it < trips; ++it) {
-      const int64_t j = it * kKdThreads + t;
-      const bool act = j < nvec;
-      const uint4 v = act ? trow[j] : make_uint4(0, 0, 0, 0);
-      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    for (int64_t it = 0; it < trips; it += kKdUnroll) {
+      uint4 v[kKdUnroll];
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        const uint32_t k0 = kd_key(w[e]), k1 = kd_key(w[e] >> 16);
-        hist_add(sh.hist, k0 & 0xFFu, act && (k0 >> 8) == b1, lane);
-        hist_add(sh.hist, k1 & 0xFFu, act && (k1 >> 8) == b1, lane);
+      for (int u = 0; u < kKdUnroll; ++u) {
+        const int64_t j = (it + u) * kKdThreads + t;
+        v[u] = j < nvec ? trow[j] : make_uint4(0, 0, 0, 0);
+      }
+#pragma unroll
+      for (int u = 0; u < kKdUnroll; ++u) {
+        const bool act = (it + u) * kKdThreads + t < nvec;
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+        for (int e = 0; e < 4; ++e) {
+          const uint32_t k0 = kd_key(w[e]), k1 = kd_key(w[e] >> 16);
+          hist_add(sh.whist[warp], k0 & 0xFFu, act && (k0 >> 8) == b1);
+          hist_add(sh.whist[warp], k1 & 0xFFu, act && (k1 >> 8) == b1);
+        }
       }
     }
     __syncthreads();
+    reduce_hist(sh);
     find_bin(sh, (uint32_t)k - above1);
     const uint32_t T = (b1 << 8) | sh.bin;
     const uint32_t need_eq = (uint32_t)k - (above1 + sh.above);  // entries equal to T taken
@@ -207,10 +236,17 @@ __global__ void __launch_bounds__(kKdThreads, 1) topk_kl_kernel(const uint4* __r
     // ---- pass 3: select in index order, accumulate
     KdAcc acc;
     acc.init();
+    uint4 v_next = t < nvec ? trow[t] : make_uint4(0, 0, 0, 0);
+    uint4 s_next = t < nvec ? srow[t] : make_uint4(0, 0, 0, 0);
     for (int64_t it = 0; it < trips; ++it) {
       const int64_t j = it * kKdThreads + t;
       const bool act = j < nvec;
-      const uint4 v = act ? trow[j] : make_uint4(0, 0, 0, 0);
+      const uint4 v = v_next, sv = s_next;
+      {  // next tile's loads overlap this tile's scans
+        const int64_t jn = j + kKdThreads;
+        v_next = jn < nvec ? trow[jn] : make_uint4(0, 0, 0, 0);
+        s_next = jn < nvec ? srow[jn] : make_uint4(0, 0, 0, 0);
+      }
       const uint32_t w[4] = {v.x, v.y, v.z, v.w};
       uint32_t keys[8];
 #pragma unroll
@@ -221,8 +257,8 @@ __global__ void __launch_bounds__(kKdThreads, 1) topk_kl_kernel(const uint4* __r
       uint32_t n_eq = 0;
 #pragma unroll
       for (int e = 0; e < 8; ++e) n_eq += keys[e] == T && act;
-      uint32_t tot_eq;
-      const uint32_t eq_rank0 = sh.eq_base + block_scan(sh, n_eq, &tot_eq);
+      uint32_t tot_eq = 0, eq_rank0 = sh.eq_base;
+      if (__syncthreads_or(n_eq != 0)) eq_rank0 += block_scan(sh, n_eq, &tot_eq);
       uint32_t selmask = 0, r = eq_rank0;
 #pragma unroll
       for (int e = 0; e < 8; ++e) {
@@ -234,7 +270,6 @@ __global__ void __launch_bounds__(kKdThreads, 1) topk_kl_kernel(const uint4* __r
       uint32_t tot_sel = 0, pos = 0;
       if (idx_out) pos = sh.sel_base + block_scan(sh, (uint32_t)__popc(selmask), &tot_sel);
       if (selmask) {
-        const uint4 sv = srow[j];
         const uint32_t sw[4] = {sv.x, sv.y, sv.z, sv.w};
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
