@@ -8,7 +8,7 @@
 // set; loss = KL(p_t || p_s) = sum p_t (t - s) - lse_t + lse_s with
 // p_t = exp(t - lse_t); d loss / d s = p_s - p_t on the set.
 //
-// One CTA of 1024 threads per row (persistent over rows). The set is found
+// One CTA of 512 threads per row (persistent over rows, two CTAs per SM). The set is found
 // by a two-digit radix select on order-preserving 16-bit keys of the BF16
 // teacher logits (high byte, then low byte among the high-byte bin that holds
 // the k-th largest), which gives the threshold key T, the count above it, and
@@ -17,13 +17,22 @@
 // block scan, and accumulates the two log-sum-exps and sum p_t (t - s)
 // online (rescaled when the running maximum grows). The histograms are
 // per warp (shared-memory atomics; logits concentrate in few bins, so warps
-// must not share counters). Loads run kKdUnroll trips ahead.
+// must not share counters).
+//
+// Fast path (taken when it can be): a 1/16 sample of the row gives a key T0
+// just below the k-th largest; one pass compacts the entries with key >= T0
+// (each warp its own contiguous segment, so the candidates stay in index
+// order) into shared memory; the exact select, the tie ranking and the
+// accumulation then run on the candidates only, and the student logits are
+// read at the candidates alone. If the sample undershoots (fewer than k
+// candidates) or a segment overflows its capacity, the row takes the full
+// three-pass path.
 #include "common.cuh"
 #include "kernels.h"
 
 namespace nvfp4 {
 
-constexpr int kKdThreads = 1024;
+constexpr int kKdThreads = 512;  // two CTAs per SM: one row's selection overlaps another's streaming
 constexpr int kKdWarps = kKdThreads / 32;
 constexpr int kKdUnroll = 4;  // 16-byte loads in flight per thread in the histogram passes
 
@@ -35,7 +44,15 @@ __device__ __forceinline__ uint32_t kd_key(uint32_t b) {
 }
 
 __device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+// Inverse of kd_key (for -0 it gives +0, the same value).
+__device__ __forceinline__ float kd_value(uint32_t key) {
+  const uint32_t b = (key & 0x8000u) ? (key ^ 0x8000u) : (~key & 0xFFFFu);
+  return __uint_as_float(b << 16);
+}
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+constexpr int kSampleStride = 16;   // the sample reads every 16th 16-byte vector of a row
+constexpr int kCandPerWarp = 512;   // candidate capacity of one warp's row segment
 
 struct KdShared {
   uint32_t whist[kKdWarps][256];  // per-warp histograms (no cross-warp contention)
@@ -43,7 +60,13 @@ struct KdShared {
   uint32_t scan[kKdWarps];
   uint32_t bin, above;      // find_bin result
   uint32_t eq_base, sel_base;
+  uint32_t wcount[kKdWarps];  // candidates per warp segment
+  uint32_t wtmp[kKdWarps];
+  int overflow;
   float red[kKdWarps][5];
+  uint16_t ckey[kKdWarps][kCandPerWarp];  // candidate keys, index order within a warp's segment
+  uint16_t cstu[kKdWarps][kCandPerWarp];  // the student logits (BF16 bits) at the candidates
+  int32_t cidx[kKdWarps][kCandPerWarp];   // their vocabulary indices
 };
 
 // Histogram add into this warp's own histogram (lanes of one warp that hit
@@ -91,7 +114,7 @@ __device__ __forceinline__ void find_bin(KdShared& sh, uint32_t need) {
   __syncthreads();
 }
 
-// Block-wide exclusive scan of v (1024 threads); returns the exclusive prefix
+// Block-wide exclusive scan of v (all threads); returns the exclusive prefix
 // and writes the block total to *total.
 __device__ __forceinline__ uint32_t block_scan(KdShared& sh, uint32_t v, uint32_t* total) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -104,13 +127,13 @@ __device__ __forceinline__ uint32_t block_scan(KdShared& sh, uint32_t v, uint32_
   if (lane == 31) sh.scan[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    uint32_t w = sh.scan[lane];
+    uint32_t w = lane < kKdWarps ? sh.scan[lane] : 0u;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const uint32_t u = __shfl_up_sync(0xFFFFFFFFu, w, o);
       if (lane >= o) w += u;
     }
-    sh.scan[lane] = w;
+    if (lane < kKdWarps) sh.scan[lane] = w;
   }
   __syncthreads();
   const uint32_t excl = incl - v + (warp > 0 ? sh.scan[warp - 1] : 0u);
@@ -160,19 +183,200 @@ struct KdAcc {
   }
 };
 
-__global__ void __launch_bounds__(kKdThreads, 1) topk_kl_kernel(const uint4* __restrict__ teacher,
+// Exclusive prefix of sh.wtmp over warps for warp w (sum of warps below w).
+__device__ __forceinline__ uint32_t warp_prefix(const KdShared& sh, int w) {
+  uint32_t p = 0;
+  for (int i = 0; i < w; ++i) p += sh.wtmp[i];
+  return p;
+}
+
+// Fast path of one row (see the file comment). Returns false, with nothing
+// written, when the row must take the full path. All threads call it.
+__device__ bool kd_fast_row(KdShared& sh, const uint4* trow, const uint16_t* srow16, int64_t nvec, int k,
+                            KdAcc& acc, int32_t* idx_row) {
+  const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+  const unsigned lt_mask = (1u << lane) - 1u;
+
+  // ---- A: sample every kSampleStride-th vector; key of its ks-th largest
+  const int64_t nsv = (nvec + kSampleStride - 1) / kSampleStride;    // sampled vectors
+  const int64_t nse = nsv * 8;                                         // sampled elements
+  const int64_t ks64 = (int64_t)k / kSampleStride + (int64_t)k / (4 * kSampleStride) + 32;
+  uint32_t T0 = 0u;  // all entries are candidates unless the sample is large enough
+  if (ks64 < nse) {
+    const uint32_t ks = (uint32_t)ks64;
+    for (int i = t; i < kKdWarps * 256; i += kKdThreads) (&sh.whist[0][0])[i] = 0u;
+    __syncthreads();
+    for (int64_t m = t; m < nsv; m += kKdThreads) {
+      const uint4 v = trow[m * kSampleStride];
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        hist_add(sh.whist[warp], kd_key(w[e]) >> 8, true);
+        hist_add(sh.whist[warp], kd_key(w[e] >> 16) >> 8, true);
+      }
+    }
+    __syncthreads();
+    reduce_hist(sh);
+    find_bin(sh, ks);
+    const uint32_t b1 = sh.bin, above1 = sh.above;
+    for (int i = t; i < kKdWarps * 256; i += kKdThreads) (&sh.whist[0][0])[i] = 0u;
+    __syncthreads();
+    for (int64_t m = t; m < nsv; m += kKdThreads) {
+      const uint4 v = trow[m * kSampleStride];
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const uint32_t k0 = kd_key(w[e]), k1 = kd_key(w[e] >> 16);
+        hist_add(sh.whist[warp], k0 & 0xFFu, (k0 >> 8) == b1);
+        hist_add(sh.whist[warp], k1 & 0xFFu, (k1 >> 8) == b1);
+      }
+    }
+    __syncthreads();
+    reduce_hist(sh);
+    find_bin(sh, ks - above1);
+    T0 = (b1 << 8) | sh.bin;
+  }
+
+  // ---- B: each warp compacts the entries >= T0 of its contiguous segment
+  const int64_t lo = nvec * warp / kKdWarps, hi = nvec * (warp + 1) / kKdWarps;
+  uint32_t cnt = 0;  // warp-uniform
+  for (int64_t base = lo; base < hi; base += 4 * 32) {
+    uint4 v[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t j = base + u * 32 + lane;
+      v[u] = j < hi ? trow[j] : make_uint4(0, 0, 0, 0);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int64_t j = base + u * 32 + lane;
+      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+      uint32_t keys[8], mask = 0;
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        keys[2 * e] = kd_key(w[e]);
+        keys[2 * e + 1] = kd_key(w[e] >> 16);
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) mask |= (uint32_t)(j < hi && keys[e] >= T0) << e;
+      const uint32_t n = __popc(mask);
+      uint32_t incl = n;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const uint32_t x = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+        if (lane >= o) incl += x;
+      }
+      uint32_t pos = cnt + incl - n;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        if ((mask >> e) & 1u) {
+          if (pos < (uint32_t)kCandPerWarp) {
+            sh.ckey[warp][pos] = (uint16_t)keys[e];
+            sh.cidx[warp][pos] = (int32_t)(8 * j + e);
+          }
+          ++pos;
+        }
+      }
+      cnt += __shfl_sync(0xFFFFFFFFu, incl, 31);
+    }
+  }
+  if (lane == 0) sh.wcount[warp] = cnt;
+  __syncthreads();
+  uint32_t total = 0;
+  bool over = false;
+  for (int w = 0; w < kKdWarps; ++w) {
+    total += sh.wcount[w];
+    over |= sh.wcount[w] > (uint32_t)kCandPerWarp;
+  }
+  if (over || total < (uint32_t)k) {
+    __syncthreads();
+    return false;
+  }
+
+  // ---- C: exact select among the candidates
+  const uint32_t mine = sh.wcount[warp];
+  for (int i = t; i < kKdWarps * 256; i += kKdThreads) (&sh.whist[0][0])[i] = 0u;
+  __syncthreads();
+  for (uint32_t i = lane; i < mine; i += 32) hist_add(sh.whist[warp], (uint32_t)sh.ckey[warp][i] >> 8, true);
+  __syncthreads();
+  reduce_hist(sh);
+  find_bin(sh, (uint32_t)k);
+  const uint32_t b1 = sh.bin, above1 = sh.above;
+  for (int i = t; i < kKdWarps * 256; i += kKdThreads) (&sh.whist[0][0])[i] = 0u;
+  __syncthreads();
+  for (uint32_t i = lane; i < mine; i += 32) {
+    const uint32_t key = sh.ckey[warp][i];
+    hist_add(sh.whist[warp], key & 0xFFu, (key >> 8) == b1);
+  }
+  __syncthreads();
+  reduce_hist(sh);
+  find_bin(sh, (uint32_t)k - above1);
+  const uint32_t T = (b1 << 8) | sh.bin;
+  const uint32_t need_eq = (uint32_t)k - (above1 + sh.above);
+
+  // ---- D: rank ties in index order, accumulate, place the set
+  for (uint32_t i = lane; i < mine; i += 32) sh.cstu[warp][i] = srow16[sh.cidx[warp][i]];  // independent gathers
+  __syncwarp();
+  uint32_t n_eq = 0;
+  for (uint32_t i0 = 0; i0 < mine; i0 += 32) {
+    const uint32_t i = i0 + lane;
+    n_eq += __popc(__ballot_sync(0xFFFFFFFFu, i < mine && sh.ckey[warp][i] == T));
+  }
+  if (lane == 0) sh.wtmp[warp] = n_eq;
+  __syncthreads();
+  uint32_t eq_rank = warp_prefix(sh, warp), n_sel = 0;
+  __syncthreads();
+  for (uint32_t i0 = 0; i0 < mine; i0 += 32) {
+    const uint32_t i = i0 + lane;
+    const uint32_t key = i < mine ? sh.ckey[warp][i] : 0u;
+    const unsigned eqm = __ballot_sync(0xFFFFFFFFu, i < mine && key == T);
+    const bool eq = (eqm >> lane) & 1u;
+    const bool sel = i < mine && (key > T || (eq && eq_rank + __popc(eqm & lt_mask) < need_eq));
+    eq_rank += __popc(eqm);
+    n_sel += __popc(__ballot_sync(0xFFFFFFFFu, sel));
+    if (sel) acc.add(kd_value(key), __uint_as_float((uint32_t)sh.cstu[warp][i] << 16));
+  }
+  if (idx_row) {
+    if (lane == 0) sh.wtmp[warp] = n_sel;
+    __syncthreads();
+    uint32_t pos = warp_prefix(sh, warp);
+    __syncthreads();
+    if (lane == 0) sh.wtmp[warp] = n_eq;
+    __syncthreads();
+    eq_rank = warp_prefix(sh, warp);
+    for (uint32_t i0 = 0; i0 < mine; i0 += 32) {
+      const uint32_t i = i0 + lane;
+      const uint32_t key = i < mine ? sh.ckey[warp][i] : 0u;
+      const unsigned eqm = __ballot_sync(0xFFFFFFFFu, i < mine && key == T);
+      const bool eq = (eqm >> lane) & 1u;
+      const bool sel = i < mine && (key > T || (eq && eq_rank + __popc(eqm & lt_mask) < need_eq));
+      eq_rank += __popc(eqm);
+      const unsigned selm = __ballot_sync(0xFFFFFFFFu, sel);
+      if (sel) idx_row[pos + __popc(selm & lt_mask)] = sh.cidx[warp][i];
+      pos += __popc(selm);
+    }
+  }
+  __syncthreads();
+  return true;
+}
+
+__global__ void __launch_bounds__(kKdThreads, 2) topk_kl_kernel(const uint4* __restrict__ teacher,
                                                                  const uint4* __restrict__ student, int64_t rows,
                                                                  int64_t V, int k, float* __restrict__ loss,
                                                                  int32_t* __restrict__ idx_out,
                                                                  float* __restrict__ grad_out) {
-  __shared__ KdShared sh;
+  extern __shared__ __align__(16) uint8_t kd_smem[];
+  KdShared& sh = *reinterpret_cast<KdShared*>(kd_smem);
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const int64_t nvec = V / 8;
   const int64_t trips = (nvec + kKdThreads - 1) / kKdThreads;
   for (int64_t row = blockIdx.x; row < rows; row += gridDim.x) {
     const uint4* trow = teacher + row * nvec;
     const uint4* srow = student + row * nvec;
-
+    KdAcc acc;
+    acc.init();
+    if (!kd_fast_row(sh, trow, reinterpret_cast<const uint16_t*>(srow), nvec, k, acc,
+                     idx_out ? idx_out + row * k : nullptr)) {
     // ---- pass 1: histogram of the key's high byte
     for (int i = t; i < kKdWarps * 256; i += kKdThreads) (&sh.whist[0][0])[i] = 0u;
     __syncthreads();
@@ -234,8 +438,6 @@ __global__ void __launch_bounds__(kKdThreads, 1) topk_kl_kernel(const uint4* __r
     __syncthreads();
 
     // ---- pass 3: select in index order, accumulate
-    KdAcc acc;
-    acc.init();
     uint4 v_next = t < nvec ? trow[t] : make_uint4(0, 0, 0, 0);
     uint4 s_next = t < nvec ? srow[t] : make_uint4(0, 0, 0, 0);
     for (int64_t it = 0; it < trips; ++it) {
@@ -287,6 +489,8 @@ __global__ void __launch_bounds__(kKdThreads, 1) topk_kl_kernel(const uint4* __r
       }
       __syncthreads();
     }
+
+    }  // full path
 
     // ---- block reduction of the accumulators
 #pragma unroll
@@ -344,9 +548,13 @@ __global__ void __launch_bounds__(kKdThreads, 1) topk_kl_kernel(const uint4* __r
 cudaError_t launch_topk_kl(const void* teacher, const void* student, int64_t rows, int64_t V, int k, float* loss,
                            int32_t* idx, float* grad, int num_sms, cudaStream_t s) {
   if (rows == 0) return cudaSuccess;
-  const int grid = (int)(rows < num_sms ? rows : num_sms);
+  static const cudaError_t attr = cudaFuncSetAttribute(topk_kl_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                       (int)sizeof(KdShared));
+  if (attr != cudaSuccess) return attr;
+  const int64_t slots = 2 * (int64_t)num_sms;
+  const int grid = (int)(rows < slots ? rows : slots);
   note_launch();
-  topk_kl_kernel<<<grid, kKdThreads, 0, s>>>(static_cast<const uint4*>(teacher), static_cast<const uint4*>(student),
+  topk_kl_kernel<<<grid, kKdThreads, sizeof(KdShared), s>>>(static_cast<const uint4*>(teacher), static_cast<const uint4*>(student),
                                              rows, V, k, loss, idx, grad);
   return cudaGetLastError();
 }
