@@ -32,7 +32,9 @@ def _check(nv, t, s, k):
     assert np.all(gerr <= gtol), float(np.max(gerr / gtol))
 
 
-@pytest.mark.parametrize("rows,V,k", [(5, 1024, 64), (3, 64, 64), (4, 256, 1), (2, 8192, 4096)])
+# (2, 65536, 8192) has more candidates than the per-row capacity, so it takes
+# the full three-pass path; the others take the sampled path
+@pytest.mark.parametrize("rows,V,k", [(5, 1024, 64), (3, 64, 64), (4, 256, 1), (2, 8192, 4096), (2, 65536, 8192)])
 def test_topk_kl_small(nv, rows, V, k):
     rng = np.random.default_rng(rows * V + k)
     t = np.round(rng.standard_normal((rows, V)) * 4) / 4          # many ties at every threshold
