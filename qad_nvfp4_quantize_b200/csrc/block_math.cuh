@@ -207,6 +207,45 @@ __device__ __forceinline__ void quantize_block(const f32x2 (&xs)[8], float bmax,
   encode_block<kDeq, kErr>(xs, d, __frcp_rn(d), b);
 }
 
+// Per-CTA table, built once the global scale g is known: the block step
+// d = RN(g * s) and RN(1/d) for every E4M3 scale code 0..127 (code 0: d = 0,
+// code 127 is NaN), and the scale-code divisors RN(6g), RN(4g). Lookups give
+// exactly the values quantize_block computes.
+struct StepTable {
+  float d[128];
+  float r[128];
+  float div6, div4;
+};
+
+__device__ __forceinline__ StepTable& step_table() {
+  __shared__ StepTable t;
+  return t;
+}
+
+// Called by every thread of the CTA; ends with __syncthreads().
+__device__ __forceinline__ void build_step_table(float g) {
+  StepTable& t = step_table();
+  for (int c = threadIdx.x; c < 128; c += blockDim.x) {
+    const float d = __fmul_rn(g, scale_value((uint32_t)c));
+    t.d[c] = d;
+    t.r[c] = __frcp_rn(d);
+  }
+  if (threadIdx.x == 0) {
+    t.div6 = __fmul_rn(6.0f, g);
+    t.div4 = __fmul_rn(4.0f, g);
+  }
+  __syncthreads();
+}
+
+// quantize_block with the CTA's step table (same results; kFour selects M = 4).
+template <bool kDeq, bool kErr, bool kFour>
+__device__ __forceinline__ void quantize_block_tab(const f32x2 (&xs)[8], float bmax, Block& b) {
+  const StepTable& t = step_table();
+  const uint32_t c = e4m3_code(__fdiv_rn(bmax, kFour ? t.div4 : t.div6));
+  b.sc = c > 1u ? c : 1u;
+  encode_block<kDeq, kErr>(xs, t.d[b.sc], t.r[b.sc], b);
+}
+
 template <bool kDeq, bool kErr>
 __device__ __forceinline__ void quantize_block(const Raw16& raw, float bmax, float g, float mt, Block& b) {
   f32x2 xs[8];

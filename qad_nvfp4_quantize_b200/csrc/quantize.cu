@@ -136,11 +136,11 @@ struct QuantOp {
     f32x2 xs[8];
     unpack_block(v, xs);
     Block b6;
-    quantize_block<false, kFos>(xs, bmax, g, 6.0f, b6);
+    quantize_block_tab<false, kFos, false>(xs, bmax, b6);
     uint32_t sc = b6.sc, q0 = b6.q0, q1 = b6.q1, pick4 = 0;
     if (kFos) {
       Block b4;
-      quantize_block<false, true>(xs, bmax, g, 4.0f, b4);
+      quantize_block_tab<false, true, true>(xs, bmax, b4);
       pick4 = b4.err < b6.err;  // tie keeps M = 6
       if (pick4) {
         sc = b4.sc;
@@ -156,7 +156,7 @@ struct QuantOp {
     }
   }
 
-  __device__ __forceinline__ void prepare(float) const {}
+  __device__ __forceinline__ void prepare(float g) const { build_step_table(g); }
 
   // Work independent of the values: zero padding-row scales; a max-mode call
   // that asked for a choice map gets zeros.
@@ -183,10 +183,10 @@ struct FakeOp {
     f32x2 xs[8];
     unpack_block(v, xs);
     Block b6;
-    quantize_block<true, kFos>(xs, bmax, g, 6.0f, b6);
+    quantize_block_tab<true, kFos, false>(xs, bmax, b6);
     if (kFos) {
       Block b4;
-      quantize_block<true, true>(xs, bmax, g, 4.0f, b4);
+      quantize_block_tab<true, true, true>(xs, bmax, b4);
       if (b4.err < b6.err) {
         store_bf16x16(y, c, b4.deq);
         return;
@@ -194,7 +194,7 @@ struct FakeOp {
     }
     store_bf16x16(y, c, b6.deq);
   }
-  __device__ __forceinline__ void prepare(float) const {}
+  __device__ __forceinline__ void prepare(float g) const { build_step_table(g); }
   __device__ __forceinline__ void finish() const {}
 
   __device__ static __forceinline__ uint32_t to_bf16x2(f32x2 v) {
@@ -219,8 +219,8 @@ struct FrozenFakeOp {
   __device__ __forceinline__ void operator()(const Raw16& v, const Chunk& c, float g, int lane) const {
     (void)lane;
     const uint32_t sc = c.valid ? scales_frozen[scale_offset(c.row, c.col >> 4, K >> 6)] : 1u;
-    const float d = __fmul_rn(g, scale_value(sc));
-    const float r = __frcp_rn(d);
+    const float d = step_table().d[sc & 127u];
+    const float r = step_table().r[sc & 127u];
     const f32x2 rr = pack2(r, r), dd = pack2(d, d);
     f32x2 sv[8], out[8];
 #pragma unroll
@@ -231,7 +231,7 @@ struct FrozenFakeOp {
     for (int i = 0; i < 8; ++i) out[i] = mul2(dd, out[i]);
     FakeOp<false>::store_bf16x16(y, c, out);
   }
-  __device__ __forceinline__ void prepare(float) const {}
+  __device__ __forceinline__ void prepare(float g) const { build_step_table(g); }
   __device__ __forceinline__ void finish() const {}
 };
 
@@ -264,7 +264,7 @@ struct SteOp {
   uint4* gx;
   int64_t M, K;
 
-  __device__ __forceinline__ void prepare(float) const {}
+  __device__ __forceinline__ void prepare(float g) const { build_step_table(g); }
   __device__ __forceinline__ void operator()(const Raw16& v, const Chunk& c, float g, int lane) const {
     (void)lane;
     const float bmax = block_absmax(v);
@@ -273,13 +273,13 @@ struct SteOp {
     uint32_t sc;
     if (kFos) {
       Block b6, b4;
-      quantize_block<false, true>(xs, bmax, g, 6.0f, b6);
-      quantize_block<false, true>(xs, bmax, g, 4.0f, b4);
+      quantize_block_tab<false, true, false>(xs, bmax, b6);
+      quantize_block_tab<false, true, true>(xs, bmax, b4);
       sc = b4.err < b6.err ? b4.sc : b6.sc;
     } else {
       sc = block_scale_code(bmax, g, 6.0f);
     }
-    ste_store(gy, gx, c, xs, __frcp_rn(__fmul_rn(g, scale_value(sc))));
+    ste_store(gy, gx, c, xs, step_table().r[sc]);
   }
   __device__ __forceinline__ void finish() const {}
 };
@@ -291,13 +291,13 @@ struct FrozenSteOp {
   const uint8_t* scales_frozen;
   int64_t M, K;
 
-  __device__ __forceinline__ void prepare(float) const {}
+  __device__ __forceinline__ void prepare(float g) const { build_step_table(g); }
   __device__ __forceinline__ void operator()(const Raw16& v, const Chunk& c, float g, int lane) const {
     (void)lane;
     const uint32_t sc = c.valid ? scales_frozen[scale_offset(c.row, c.col >> 4, K >> 6)] : 1u;
     f32x2 xs[8];
     unpack_block(v, xs);
-    ste_store(gy, gx, c, xs, __frcp_rn(__fmul_rn(g, scale_value(sc))));
+    ste_store(gy, gx, c, xs, step_table().r[sc & 127u]);
   }
   __device__ __forceinline__ void finish() const {}
 };
@@ -316,40 +316,27 @@ struct MseOp {
   uint8_t* choice;
   int64_t M, K;
 
-  __device__ static __forceinline__ float* table() {
-    __shared__ float t[2 * 128];  // d[c], then RN(1/d[c])
-    return t;
-  }
-
-  __device__ __forceinline__ void prepare(float g) const {
-    float* t = table();
-    for (int c = threadIdx.x; c < 128; c += blockDim.x) {
-      const float d = __fmul_rn(g, scale_value(c >= 1 && c <= 126 ? (uint32_t)c : 1u));
-      t[c] = d;
-      t[128 + c] = __frcp_rn(d);
-    }
-    __syncthreads();
-  }
+  __device__ __forceinline__ void prepare(float g) const { build_step_table(g); }
 
   __device__ __forceinline__ void operator()(const Raw16& v, const Chunk& c, float g, int lane) const {
     (void)g;
     (void)lane;
-    const float* t = table();
+    const StepTable& t = step_table();
     const float bmax = block_absmax(v);
     f32x2 xs[8];
     unpack_block(v, xs);
     Block b;
-    encode_block<false, true>(xs, t[126], t[128 + 126], b);
+    encode_block<false, true>(xs, t.d[126], t.r[126], b);
     uint32_t best_sc = 126, q0 = b.q0, q1 = b.q1;
     float best = b.err;
     for (int code = 125; code >= 1; --code) {
-      const float d = t[code];
+      const float d = t.d[code];
       const float dm = __fmul_rn(d, 6.0f);
       if (dm < bmax) {
         const float df = __fsub_rn(bmax, dm);
         if (__fmul_rn(df, df) > best) break;
       }
-      encode_block<false, true>(xs, d, t[128 + code], b);
+      encode_block<false, true>(xs, d, t.r[code], b);
       if (b.err <= best) {  // ties move to the lower code
         best = b.err;
         best_sc = (uint32_t)code;
