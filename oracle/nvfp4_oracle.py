@@ -19,10 +19,10 @@ Pages cited (titles as printed on each page):
                (dynamic vs frozen scales, Figure 2).
 * [QWEN36-QAD] "Model-Optimizer in practice: recovering Qwen3.6-35B-A3B W4A4
                NVFP4 accuracy with quantization-aware distillation" --
-               "Why W4A4 rather than W4A16" and "2. PTQ" (routed experts,
-               fused gate/up/down projections).
+               "Why W4A4 rather than W4A16", "2. PTQ" (routed experts,
+               fused gate/up/down projections) and "QAD" (top-k logit KD).
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 
 R1  E2M1 and E4M3 conversions round to nearest, ties to the even code, and
     saturate (E2M1 to +-6, E4M3 to 448). The sign of an E2M1 code is the sign
@@ -53,7 +53,7 @@ R11 QAD backward through the simulated quantization ([NEMO-QAD] Figure 2:
     dL/dx = dL/dy where |x * r| <= 6 for the block's r = RN(1/(g*s)) (FP32
     product), else 0. Rounding is passed straight through; saturation is not.
     The scales are those of the forward: recomputed (dynamic) or frozen.
-R12 Top-k logit KL ([P1] "QAD": "--logit_kl_topk 4096" restricts the KD loss
+R12 Top-k logit KL ([QWEN36-QAD] "QAD": --logit_kl_topk 4096 restricts the KD loss
     to the teacher's top-4096 vocabulary entries; the loss compares teacher
     and student logits element-wise over the vocabulary): per row, the k
     entries with the largest teacher logits (ties to the lower index) form

@@ -89,7 +89,9 @@ def bf16_to_f32(t: torch.Tensor) -> np.ndarray:
 
 
 def kd_logits(seed: int = 0, rows: int = 2048, V: int = 248320, k_peaked: int = 64):
-    """Teacher / student logits for the top-k KL loss ([P1] "QAD", vocabulary of
+    """Teacher / student logits for the top-k KL loss ("Model-Optimizer in
+    practice: recovering Qwen3.6-35B-A3B W4A4 NVFP4 accuracy with QAD",
+    section "QAD": vocabulary of
     248,320 entries): teacher = N(0, 2) with k_peaked entries per row raised
     by 8 (a peaked distribution), student = teacher + N(0, 0.5); both BF16."""
     rt, rp, rs = _streams(seed, 3)
