@@ -313,8 +313,11 @@ __global__ void __launch_bounds__(kRowThreads) moe_quantize_rows_kernel(
     for (int u = 0; u < kRowUnroll; ++u) {
       if (ch0 + u * nwarps >= n_chunks) break;  // warp-uniform
       Block b;
-      quantize_block<false, false>(vv[u], block_absmax(vv[u]), g_s[ex[u]], 6.0f, b);
-      if (pr[u] < 0) b.sc = b.q0 = b.q1 = 0u;  // pad row
+      if (pr[u] >= 0) {
+        quantize_block<false, false>(vv[u], block_absmax(vv[u]), g_s[ex[u]], 6.0f, b);
+      } else {
+        b.sc = b.q0 = b.q1 = 0u;  // pad row: zero codes and scales, no arithmetic
+      }
       if (cc[u].valid) {
         codes[(cc[u].row * K + cc[u].col) >> 4] = make_uint2(b.q0, b.q1);
         scales[scale_offset(cc[u].row, cc[u].col >> 4, kgroups)] = (uint8_t)b.sc;
