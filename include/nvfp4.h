@@ -185,6 +185,8 @@ nvfp4_status nvfp4_gemm(const uint8_t* Aq, const uint8_t* As, const float* ga,
  * idx       nullable out int32 [rows][k]: the set, ascending index.
  * grad      nullable out FP32 [rows][k]: d loss / d student logit at idx
  *           (needs idx).
+ * Non-finite teacher logits rank by their BF16 bit pattern: +-Inf as
+ *   values, NaN with the sign bit clear above +Inf, with it set below -Inf.
  * Errors: NVFP4_ERR_INVALID_ARG for bad sizes or pointers.
  */
 nvfp4_status nvfp4_topk_kl(const void* teacher, const void* student, int64_t rows, int64_t V, int k,

@@ -24,9 +24,15 @@
 // (each warp its own contiguous segment, so the candidates stay in index
 // order) into shared memory; the exact select, the tie ranking and the
 // accumulation then run on the candidates only, and the student logits are
-// read at the candidates alone. If the sample undershoots (fewer than k
+// read at the candidates alone. The compaction tests two logits per
+// instruction against T0's value (packed BF16 compare) and works on keys
+// only for the few entries that pass; each candidate's student logit is
+// fetched by an asynchronous 4-byte copy into shared memory issued as the
+// candidate is found, so the gathers overlap the rest of the pass. If the sample undershoots (fewer than k
 // candidates) or a segment overflows its capacity, the row takes the full
 // three-pass path.
+#include <cuda_bf16.h>
+
 #include "common.cuh"
 #include "kernels.h"
 
@@ -51,6 +57,17 @@ __device__ __forceinline__ float kd_value(uint32_t key) {
 }
 __device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
 
+// Per half of two BF16 pairs: 0xFFFF where a >= b or either is NaN, else 0.
+__device__ __forceinline__ uint32_t bf16x2_geu_mask(uint32_t a, uint32_t b) {
+  return __hgeu2_mask(*reinterpret_cast<const __nv_bfloat162*>(&a), *reinterpret_cast<const __nv_bfloat162*>(&b));
+}
+
+// 4-byte asynchronous copy global -> shared (completion: cp_async_wait_all).
+__device__ __forceinline__ void cp_async_4(uint32_t smem_addr, const void* gptr) {
+  asm volatile("cp.async.ca.shared.global [%0], [%1], 4;" ::"r"(smem_addr), "l"(gptr) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;" ::: "memory"); }
+
 constexpr int kSampleStride = 16;   // the sample reads every 16th 16-byte vector of a row
 constexpr int kCandPerWarp = 512;   // candidate capacity of one warp's row segment
 
@@ -65,7 +82,7 @@ struct KdShared {
   int overflow;
   float red[kKdWarps][5];
   uint16_t ckey[kKdWarps][kCandPerWarp];  // candidate keys, index order within a warp's segment
-  uint16_t cstu[kKdWarps][kCandPerWarp];  // the student logits (BF16 bits) at the candidates
+  uint32_t cstu[kKdWarps][kCandPerWarp];  // aligned student word holding the candidate's logit
   int32_t cidx[kKdWarps][kCandPerWarp];   // their vocabulary indices
 };
 
@@ -239,7 +256,13 @@ __device__ bool kd_fast_row(KdShared& sh, const uint4* trow, const uint16_t* sro
 
   // ---- B: each warp compacts the entries >= T0 of its contiguous segment
   const int64_t lo = nvec * warp / kKdWarps, hi = nvec * (warp + 1) / kKdWarps;
-  uint32_t cnt = 0;  // warp-uniform
+  // T0 as a BF16 value in both halves; key 0 (every entry a candidate) maps
+  // to a NaN pattern, which the unordered compare passes everywhere.
+  const uint32_t tvb = (T0 & 0x8000u) ? (T0 ^ 0x8000u) : (~T0 & 0xFFFFu);
+  const uint32_t thr2 = tvb | (tvb << 16);
+  const uint32_t cstu_base = (uint32_t)__cvta_generic_to_shared(&sh.cstu[warp][0]);
+  uint32_t cnt = 0;   // slots used (warp-uniform)
+  uint32_t real = 0;  // candidates with key >= T0 (the value test also passes NaN)
   for (int64_t base = lo; base < hi; base += 4 * 32) {
     uint4 v[4];
 #pragma unroll
@@ -247,48 +270,69 @@ __device__ bool kd_fast_row(KdShared& sh, const uint4* trow, const uint16_t* sro
       const int64_t j = base + u * 32 + lane;
       v[u] = j < hi ? trow[j] : make_uint4(0, 0, 0, 0);
     }
+    // One bit per passing element at bit 8e (e = element within the vector).
+    uint64_t q[4];
+    uint32_t n[4];
 #pragma unroll
     for (int u = 0; u < 4; ++u) {
       const int64_t j = base + u * 32 + lane;
-      const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
-      uint32_t keys[8], mask = 0;
+      const uint32_t lo4 = __byte_perm(bf16x2_geu_mask(v[u].x, thr2), bf16x2_geu_mask(v[u].y, thr2), 0x6420) & 0x01010101u;
+      const uint32_t hi4 = __byte_perm(bf16x2_geu_mask(v[u].z, thr2), bf16x2_geu_mask(v[u].w, thr2), 0x6420) & 0x01010101u;
+      q[u] = j < hi ? ((uint64_t)lo4 | ((uint64_t)hi4 << 32)) : 0ull;
+      n[u] = (uint32_t)__popcll(q[u]);
+    }
+    // Slots: one warp scan of the four counts, two per 32-bit word.
+    uint32_t p01 = n[0] | (n[1] << 16), p23 = n[2] | (n[3] << 16);
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        keys[2 * e] = kd_key(w[e]);
-        keys[2 * e + 1] = kd_key(w[e] >> 16);
+    for (int o = 1; o < 32; o <<= 1) {
+      const uint32_t x = __shfl_up_sync(0xFFFFFFFFu, p01, o), y = __shfl_up_sync(0xFFFFFFFFu, p23, o);
+      if (lane >= o) {
+        p01 += x;
+        p23 += y;
       }
+    }
+    const uint32_t t01 = __shfl_sync(0xFFFFFFFFu, p01, 31), t23 = __shfl_sync(0xFFFFFFFFu, p23, 31);
+    const uint32_t incl[4] = {p01 & 0xFFFFu, p01 >> 16, p23 & 0xFFFFu, p23 >> 16};
+    const uint32_t tot[4] = {t01 & 0xFFFFu, t01 >> 16, t23 & 0xFFFFu, t23 >> 16};
 #pragma unroll
-      for (int e = 0; e < 8; ++e) mask |= (uint32_t)(j < hi && keys[e] >= T0) << e;
-      const uint32_t n = __popc(mask);
-      uint32_t incl = n;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t x = __shfl_up_sync(0xFFFFFFFFu, incl, o);
-        if (lane >= o) incl += x;
-      }
-      uint32_t pos = cnt + incl - n;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        if ((mask >> e) & 1u) {
-          if (pos < (uint32_t)kCandPerWarp) {
-            sh.ckey[warp][pos] = (uint16_t)keys[e];
-            sh.cidx[warp][pos] = (int32_t)(8 * j + e);
-          }
-          ++pos;
+    for (int u = 0; u < 4; ++u) {
+      const int64_t j = base + u * 32 + lane;
+      uint64_t bits = q[u];
+      uint32_t pos = cnt + incl[u] - n[u];
+      while (bits) {  // ascending element order
+        const int e = (__ffsll((long long)bits) - 1) >> 3;
+        bits &= bits - 1;
+        const int wi = e >> 1;
+        const uint32_t wv = wi == 0 ? v[u].x : wi == 1 ? v[u].y : wi == 2 ? v[u].z : v[u].w;
+        const uint32_t key = kd_key((e & 1) ? (wv >> 16) : wv);
+        real += key >= T0;
+        if (pos < (uint32_t)kCandPerWarp) {
+          const int64_t idx = 8 * j + e;
+          sh.ckey[warp][pos] = (uint16_t)key;
+          sh.cidx[warp][pos] = (int32_t)idx;
+          cp_async_4(cstu_base + 4u * pos, srow16 + (idx & ~int64_t(1)));
         }
+        ++pos;
       }
-      cnt += __shfl_sync(0xFFFFFFFFu, incl, 31);
+      cnt += tot[u];
     }
   }
-  if (lane == 0) sh.wcount[warp] = cnt;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) real += __shfl_xor_sync(0xFFFFFFFFu, real, o);
+  if (lane == 0) {
+    sh.wcount[warp] = cnt;
+    sh.wtmp[warp] = real;
+  }
   __syncthreads();
   uint32_t total = 0;
   bool over = false;
   for (int w = 0; w < kKdWarps; ++w) {
-    total += sh.wcount[w];
+    total += sh.wtmp[w];
     over |= sh.wcount[w] > (uint32_t)kCandPerWarp;
   }
+  __syncthreads();  // sh.wtmp is reused below
   if (over || total < (uint32_t)k) {
+    cp_async_wait_all();  // no copy may land in a later row's slots
     __syncthreads();
     return false;
   }
@@ -315,7 +359,7 @@ __device__ bool kd_fast_row(KdShared& sh, const uint4* trow, const uint16_t* sro
   const uint32_t need_eq = (uint32_t)k - (above1 + sh.above);
 
   // ---- D: rank ties in index order, accumulate, place the set
-  for (uint32_t i = lane; i < mine; i += 32) sh.cstu[warp][i] = srow16[sh.cidx[warp][i]];  // independent gathers
+  cp_async_wait_all();  // this lane's student copies; then the warp's
   __syncwarp();
   uint32_t n_eq = 0;
   for (uint32_t i0 = 0; i0 < mine; i0 += 32) {
@@ -334,7 +378,10 @@ __device__ bool kd_fast_row(KdShared& sh, const uint4* trow, const uint16_t* sro
     const bool sel = i < mine && (key > T || (eq && eq_rank + __popc(eqm & lt_mask) < need_eq));
     eq_rank += __popc(eqm);
     n_sel += __popc(__ballot_sync(0xFFFFFFFFu, sel));
-    if (sel) acc.add(kd_value(key), __uint_as_float((uint32_t)sh.cstu[warp][i] << 16));
+    if (sel) {
+      const uint32_t sw = sh.cstu[warp][i];
+      acc.add(kd_value(key), __uint_as_float((sh.cidx[warp][i] & 1) ? (sw & 0xFFFF0000u) : (sw << 16)));
+    }
   }
   if (idx_row) {
     if (lane == 0) sh.wtmp[warp] = n_sel;
