@@ -256,13 +256,17 @@ __device__ __forceinline__ void quantize_block(const Raw16& raw, float bmax, flo
 // A warp's unit of work: 512 consecutive elements of one row ("chunk"), one
 // 16-element block per lane. Chunks never straddle rows; a row of K elements
 // has ceil(K/512) chunks and the last one may be partial. The row division is
-// warp-uniform.
-struct Chunk {
-  int64_t row;
+// warp-uniform. Index type I: uint32_t ("narrow") when every element index,
+// scale-byte offset and chunk-row division of the tensor fits 32-bit
+// arithmetic (narrow_chunks on the host decides), else int64_t.
+template <class I>
+struct ChunkT {
+  I row;
   int32_t col;        // this lane's first element within the row
   bool valid;         // col < K
-  int64_t vec;        // 16-byte vector index of the block's first 8 elements
+  I vec;              // 16-byte vector index of the block's first 8 elements
 };
+using Chunk = ChunkT<int64_t>;
 
 __device__ __forceinline__ Chunk chunk_at(int64_t ch, int32_t cpr, uint64_t cpr_magic, int64_t K, int lane) {
   Chunk c;
@@ -274,6 +278,37 @@ __device__ __forceinline__ Chunk chunk_at(int64_t ch, int32_t cpr, uint64_t cpr_
   c.valid = c.col < K;
   c.vec = (c.row * K + c.col) >> 3;
   return c;
+}
+
+// Narrow form: cpr_magic = ceil(2^32 / cpr), exact for ch * cpr < 2^32.
+__device__ __forceinline__ ChunkT<uint32_t> chunk_at_narrow(uint32_t ch, uint32_t cpr, uint32_t cpr_magic,
+                                                            uint32_t K, int lane) {
+  ChunkT<uint32_t> c;
+  const uint32_t r = cpr == 1u ? ch : __umulhi(ch, cpr_magic);
+  c.row = r;
+  c.col = (int32_t)((ch - r * cpr) * 512u + (uint32_t)lane * 16u);
+  c.valid = c.col < (int32_t)K;
+  c.vec = (r * K + (uint32_t)c.col) >> 3;
+  return c;
+}
+
+// Chunk `ch` in the index width I (cpr_magic: the 64-bit or 32-bit divisor
+// magic to match).
+template <class I>
+__device__ __forceinline__ ChunkT<I> chunk_at_t(int64_t ch, int32_t cpr, uint64_t cpr_magic, int64_t K, int lane) {
+  if constexpr (sizeof(I) == 4)
+    return chunk_at_narrow((uint32_t)ch, (uint32_t)cpr, (uint32_t)cpr_magic, (uint32_t)K, lane);
+  else
+    return chunk_at(ch, cpr, cpr_magic, K, lane);
+}
+
+// Byte offset of the lane's block scale in the tiled layout.
+__device__ __forceinline__ int64_t block_scale_offset(const ChunkT<int64_t>& c, int64_t K) {
+  return scale_offset(c.row, c.col >> 4, K >> 6);
+}
+__device__ __forceinline__ uint32_t block_scale_offset(const ChunkT<uint32_t>& c, int64_t K) {
+  const uint32_t row = c.row, cb = (uint32_t)c.col >> 4, kgroups = (uint32_t)(K >> 6);
+  return (((row >> 7) * kgroups + (cb >> 2)) << 9) + ((row & 31u) << 4) + (((row >> 5) & 3u) << 2) + (cb & 3u);
 }
 
 }  // namespace nvfp4

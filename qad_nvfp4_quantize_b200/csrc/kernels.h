@@ -16,6 +16,20 @@ inline uint64_t chunk_magic(int64_t K) {
   return cpr > 1 ? ~uint64_t(0) / cpr + 1 : 0;
 }
 
+// ceil(2^32 / cpr) for the narrow (32-bit) chunk-row division; 0 when cpr == 1.
+inline uint64_t chunk_magic_narrow(int64_t K) {
+  const uint64_t cpr = (uint64_t)((K + 511) / 512);
+  return cpr > 1 ? ((uint64_t(1) << 32) + cpr - 1) / cpr : 0;
+}
+
+// True when a tensor of M rows x K columns can be walked with 32-bit chunk
+// arithmetic: element indices and scale-byte offsets below 2^31 and the
+// 32-bit row division exact (chunks * cpr < 2^32).
+inline bool narrow_chunks(int64_t M, int64_t K) {
+  const int64_t cpr = (K + 511) / 512;
+  return (M + 128) * (cpr * 512) < (int64_t(1) << 31) && M * cpr * cpr < (int64_t(1) << 32);
+}
+
 int amax_partial_count(int64_t n, int num_sms);
 cudaError_t launch_amax_partial(const void* x, int64_t n, uint32_t* partial, int n_partial,
                                 cudaStream_t s);

@@ -23,6 +23,8 @@
 //                and adds into out[token] in FP32 (vector atomics).
 #include <mutex>
 
+#include <type_traits>
+
 #include "block_math.cuh"
 #include "gemm_kernel.cuh"
 #include "kernels.h"
@@ -268,7 +270,7 @@ __global__ void __launch_bounds__(256) moe_token_pass_kernel(const uint4* __rest
 constexpr int kRowThreads = 256;
 constexpr int kRowUnroll = 4;
 
-template <bool kGather>
+template <bool kGather, bool kNarrow>
 __global__ void __launch_bounds__(kRowThreads) moe_quantize_rows_kernel(
     const uint4* __restrict__ src, int64_t K, int topk, const int32_t* __restrict__ row_pair,
     const int32_t* __restrict__ tile_expert, const int32_t* __restrict__ tile_count,
@@ -286,28 +288,28 @@ __global__ void __launch_bounds__(kRowThreads) moe_quantize_rows_kernel(
     }
   }
   __syncthreads();
+  using Idx = typename std::conditional<kNarrow, uint32_t, int64_t>::type;
   const int lane = threadIdx.x & 31;
-  const int64_t rows = (int64_t)(*tile_count) * 128;
+  const int32_t rows = (*tile_count) * 128;
   const int32_t cpr = (int32_t)((K + 511) >> 9);
-  const int64_t n_chunks = rows * cpr;
-  const int64_t kgroups = K >> 6;
-  const int64_t warp = (int64_t)blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
-  const int64_t nwarps = (int64_t)gridDim.x * (kRowThreads / 32);
-  for (int64_t ch0 = warp; ch0 < n_chunks; ch0 += kRowUnroll * nwarps) {
-    Chunk cc[kRowUnroll];
+  const int32_t n_chunks = rows * cpr;  // < 2^30 (the launcher bounds the padded rows)
+  const int32_t warp = (int32_t)blockIdx.x * (kRowThreads / 32) + (threadIdx.x >> 5);
+  const int32_t nwarps = (int32_t)gridDim.x * (kRowThreads / 32);
+  for (int32_t ch0 = warp; ch0 < n_chunks; ch0 += kRowUnroll * nwarps) {
+    ChunkT<Idx> cc[kRowUnroll];
     int32_t pr[kRowUnroll], ex[kRowUnroll];
 #pragma unroll
     for (int u = 0; u < kRowUnroll; ++u) {
-      const int64_t ch = ch0 + u * nwarps;
-      cc[u] = chunk_at(ch < n_chunks ? ch : 0, cpr, cpr_magic, K, lane);
+      const int32_t ch = ch0 + u * nwarps;
+      cc[u] = chunk_at_t<Idx>(ch < n_chunks ? ch : 0, cpr, cpr_magic, K, lane);
       pr[u] = ch < n_chunks ? row_pair[cc[u].row] : -1;
       ex[u] = ch < n_chunks ? tile_expert[cc[u].row >> 7] : 0;
     }
     Raw16 vv[kRowUnroll];
 #pragma unroll
     for (int u = 0; u < kRowUnroll; ++u) {
-      const int64_t srow = kGather ? (int64_t)(pr[u] / topk) : cc[u].row;
-      load_raw16(src, (srow * K + cc[u].col) >> 3, pr[u] >= 0 && cc[u].valid, vv[u]);
+      const Idx srow = kGather ? (Idx)(pr[u] >= 0 ? pr[u] / topk : 0) : cc[u].row;
+      load_raw16(src, (srow * (Idx)K + (Idx)cc[u].col) >> 3, pr[u] >= 0 && cc[u].valid, vv[u]);
     }
 #pragma unroll
     for (int u = 0; u < kRowUnroll; ++u) {
@@ -319,8 +321,8 @@ __global__ void __launch_bounds__(kRowThreads) moe_quantize_rows_kernel(
         b.sc = b.q0 = b.q1 = 0u;  // pad row: zero codes and scales, no arithmetic
       }
       if (cc[u].valid) {
-        codes[(cc[u].row * K + cc[u].col) >> 4] = make_uint2(b.q0, b.q1);
-        scales[scale_offset(cc[u].row, cc[u].col >> 4, kgroups)] = (uint8_t)b.sc;
+        codes[cc[u].vec >> 1] = make_uint2(b.q0, b.q1);
+        scales[block_scale_offset(cc[u], K)] = (uint8_t)b.sc;
       }
     }
   }
@@ -512,6 +514,8 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
   auto U32 = [ws](int64_t off) { return reinterpret_cast<uint32_t*>(ws + off); };
   auto F32 = [ws](int64_t off) { return reinterpret_cast<float*>(ws + off); };
   const int64_t P = L.P, R = L.R;
+  if (R * ((a.H + 511) / 512) >= (int64_t(1) << 30) || R * ((a.I + 511) / 512) >= (int64_t(1) << 30))
+    return cudaErrorInvalidValue;  // 32-bit chunk loops of the row quantizer
   cudaError_t e;
 
   // 1. route: count, scan, place
@@ -548,10 +552,16 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
   const size_t qsmem = (size_t)a.E * sizeof(float);
   // 3. gather + quantize x per expert
   note_launch();
-  moe_quantize_rows_kernel<true><<<qgrid, kRowThreads, qsmem, s>>>(
-      static_cast<const uint4*>(a.x), a.H, a.topk, I32(L.row_pair), I32(L.tile_expert), I32(L.tile_count),
-      U32(L.amax_x), a.E, reinterpret_cast<uint2*>(ws + L.xq_codes), ws + L.xq_scales, F32(L.xq_g), status,
-      chunk_magic(a.H));
+  if (narrow_chunks(R, a.H) && narrow_chunks(a.T, a.H))
+    moe_quantize_rows_kernel<true, true><<<qgrid, kRowThreads, qsmem, s>>>(
+        static_cast<const uint4*>(a.x), a.H, a.topk, I32(L.row_pair), I32(L.tile_expert), I32(L.tile_count),
+        U32(L.amax_x), a.E, reinterpret_cast<uint2*>(ws + L.xq_codes), ws + L.xq_scales, F32(L.xq_g), status,
+        chunk_magic_narrow(a.H));
+  else
+    moe_quantize_rows_kernel<true, false><<<qgrid, kRowThreads, qsmem, s>>>(
+        static_cast<const uint4*>(a.x), a.H, a.topk, I32(L.row_pair), I32(L.tile_expert), I32(L.tile_count),
+        U32(L.amax_x), a.E, reinterpret_cast<uint2*>(ws + L.xq_codes), ws + L.xq_scales, F32(L.xq_g), status,
+        chunk_magic(a.H));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   // 4. gate_up grouped GEMM
@@ -585,10 +595,16 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
 
   // 5. quantize h per expert
   note_launch();
-  moe_quantize_rows_kernel<false><<<qgrid, kRowThreads, qsmem, s>>>(
-      reinterpret_cast<const uint4*>(ws + L.h), a.I, a.topk, I32(L.row_pair), I32(L.tile_expert),
-      I32(L.tile_count), U32(L.amax_h), a.E, reinterpret_cast<uint2*>(ws + L.hq_codes), ws + L.hq_scales,
-      F32(L.hq_g), status, chunk_magic(a.I));
+  if (narrow_chunks(R, a.I))
+    moe_quantize_rows_kernel<false, true><<<qgrid, kRowThreads, qsmem, s>>>(
+        reinterpret_cast<const uint4*>(ws + L.h), a.I, a.topk, I32(L.row_pair), I32(L.tile_expert),
+        I32(L.tile_count), U32(L.amax_h), a.E, reinterpret_cast<uint2*>(ws + L.hq_codes), ws + L.hq_scales,
+        F32(L.hq_g), status, chunk_magic_narrow(a.I));
+  else
+    moe_quantize_rows_kernel<false, false><<<qgrid, kRowThreads, qsmem, s>>>(
+        reinterpret_cast<const uint4*>(ws + L.h), a.I, a.topk, I32(L.row_pair), I32(L.tile_expert),
+        I32(L.tile_count), U32(L.amax_h), a.E, reinterpret_cast<uint2*>(ws + L.hq_codes), ws + L.hq_scales,
+        F32(L.hq_g), status, chunk_magic(a.I));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
   // 6. down grouped GEMM + weighted FP32 combine

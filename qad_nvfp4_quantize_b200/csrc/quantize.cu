@@ -13,6 +13,8 @@
 // per lane, block scales as one byte per lane into the tiled scale layout.
 // Dynamic calls run as a single cooperative launch (fused_dynamic_kernel);
 // static-scale and frozen-scale calls stream once (stream_pass_kernel).
+#include <type_traits>
+
 #include "block_math.cuh"
 #include "kernels.h"
 
@@ -131,7 +133,8 @@ struct QuantOp {
   uint8_t* choice;
   int64_t M, K;
 
-  __device__ __forceinline__ void operator()(const Raw16& v, const Chunk& c, float g, int lane) const {
+  template <class C>
+  __device__ __forceinline__ void operator()(const Raw16& v, const C& c, float g, int lane) const {
     const float bmax = block_absmax(v);
     f32x2 xs[8];
     unpack_block(v, xs);
@@ -151,7 +154,7 @@ struct QuantOp {
     (void)lane;
     if (c.valid) {
       codes[c.vec >> 1] = make_uint2(q0, q1);
-      scales[scale_offset(c.row, c.col >> 4, K >> 6)] = (uint8_t)sc;  // 4 lanes fill one 4-byte group
+      scales[block_scale_offset(c, K)] = (uint8_t)sc;  // 4 lanes fill one 4-byte group
       if (kFos && choice) choice[c.vec >> 1] = (uint8_t)pick4;
     }
   }
@@ -177,7 +180,8 @@ struct FakeOp {
   uint4* y;
   int64_t M, K;
 
-  __device__ __forceinline__ void operator()(const Raw16& v, const Chunk& c, float g, int lane) const {
+  template <class C>
+  __device__ __forceinline__ void operator()(const Raw16& v, const C& c, float g, int lane) const {
     (void)lane;
     const float bmax = block_absmax(v);
     f32x2 xs[8];
@@ -203,7 +207,8 @@ struct FakeOp {
     return f32x2_to_bf16x2(lo, hi);
   }
 
-  __device__ static __forceinline__ void store_bf16x16(uint4* y, const Chunk& c, const f32x2 (&out)[8]) {
+  template <class C>
+  __device__ static __forceinline__ void store_bf16x16(uint4* y, const C& c, const f32x2 (&out)[8]) {
     if (!c.valid) return;
     y[c.vec] = make_uint4(to_bf16x2(out[0]), to_bf16x2(out[1]), to_bf16x2(out[2]), to_bf16x2(out[3]));
     y[c.vec + 1] = make_uint4(to_bf16x2(out[4]), to_bf16x2(out[5]), to_bf16x2(out[6]), to_bf16x2(out[7]));
@@ -216,9 +221,10 @@ struct FrozenFakeOp {
   const uint8_t* scales_frozen;
   int64_t M, K;
 
-  __device__ __forceinline__ void operator()(const Raw16& v, const Chunk& c, float g, int lane) const {
+  template <class C>
+  __device__ __forceinline__ void operator()(const Raw16& v, const C& c, float g, int lane) const {
     (void)lane;
-    const uint32_t sc = c.valid ? scales_frozen[scale_offset(c.row, c.col >> 4, K >> 6)] : 1u;
+    const uint32_t sc = c.valid ? scales_frozen[block_scale_offset(c, K)] : 1u;
     const float d = step_table().d[sc & 127u];
     const float r = step_table().r[sc & 127u];
     const f32x2 rr = pack2(r, r), dd = pack2(d, d);
@@ -246,7 +252,8 @@ __device__ __forceinline__ uint32_t ste_word(uint32_t gy, f32x2 xr) {
   return gy & ((fabsf(lo) <= 6.0f ? 0x0000FFFFu : 0u) | (fabsf(hi) <= 6.0f ? 0xFFFF0000u : 0u));
 }
 
-__device__ __forceinline__ void ste_store(const uint4* gy, uint4* gx, const Chunk& c, const f32x2 (&xs)[8],
+template <class C>
+__device__ __forceinline__ void ste_store(const uint4* gy, uint4* gx, const C& c, const f32x2 (&xs)[8],
                                           float r) {
   if (!c.valid) return;
   const uint4 a = ld_stream(gy + c.vec), b = ld_stream(gy + c.vec + 1);
@@ -265,7 +272,8 @@ struct SteOp {
   int64_t M, K;
 
   __device__ __forceinline__ void prepare(float g) const { build_step_table(g); }
-  __device__ __forceinline__ void operator()(const Raw16& v, const Chunk& c, float g, int lane) const {
+  template <class C>
+  __device__ __forceinline__ void operator()(const Raw16& v, const C& c, float g, int lane) const {
     (void)lane;
     const float bmax = block_absmax(v);
     f32x2 xs[8];
@@ -292,9 +300,10 @@ struct FrozenSteOp {
   int64_t M, K;
 
   __device__ __forceinline__ void prepare(float g) const { build_step_table(g); }
-  __device__ __forceinline__ void operator()(const Raw16& v, const Chunk& c, float g, int lane) const {
+  template <class C>
+  __device__ __forceinline__ void operator()(const Raw16& v, const C& c, float g, int lane) const {
     (void)lane;
-    const uint32_t sc = c.valid ? scales_frozen[scale_offset(c.row, c.col >> 4, K >> 6)] : 1u;
+    const uint32_t sc = c.valid ? scales_frozen[block_scale_offset(c, K)] : 1u;
     f32x2 xs[8];
     unpack_block(v, xs);
     ste_store(gy, gx, c, xs, step_table().r[sc & 127u]);
@@ -318,7 +327,8 @@ struct MseOp {
 
   __device__ __forceinline__ void prepare(float g) const { build_step_table(g); }
 
-  __device__ __forceinline__ void operator()(const Raw16& v, const Chunk& c, float g, int lane) const {
+  template <class C>
+  __device__ __forceinline__ void operator()(const Raw16& v, const C& c, float g, int lane) const {
     (void)g;
     (void)lane;
     const StepTable& t = step_table();
@@ -346,7 +356,7 @@ struct MseOp {
     }
     if (c.valid) {
       codes[c.vec >> 1] = make_uint2(q0, q1);
-      scales[scale_offset(c.row, c.col >> 4, K >> 6)] = (uint8_t)best_sc;
+      scales[block_scale_offset(c, K)] = (uint8_t)best_sc;
       if (choice) choice[c.vec >> 1] = 0;
     }
   }
@@ -358,7 +368,7 @@ struct MseOp {
 // Streaming pass with a known global scale (static g, or g reduced from the
 // partials of a separate amax pass): grid-stride over 512-element chunks.
 // ----------------------------------------------------------------------------
-template <class Op>
+template <class Op, bool kNarrow>
 __global__ void __launch_bounds__(kQThreads) stream_pass_kernel(const uint4* __restrict__ x, int64_t M, int64_t K,
                                                                  const uint32_t* __restrict__ partial, int n_partial,
                                                                  const float* __restrict__ g_static, Op op,
@@ -371,19 +381,20 @@ __global__ void __launch_bounds__(kQThreads) stream_pass_kernel(const uint4* __r
     if (g_out) *g_out = g;
     if (bad) record_status(status, NVFP4_ERR_NONFINITE_INPUT);
   }
+  using Idx = typename std::conditional<kNarrow, uint32_t, int64_t>::type;
   const int32_t cpr = (int32_t)((K + 511) >> 9);
-  const int64_t n_chunks = M * cpr;
+  const int32_t n_chunks = (int32_t)(M * cpr);  // < 2^31 (checked by the launcher)
   const int lane = threadIdx.x & 31;
-  const int64_t warp = (int64_t)blockIdx.x * (kQThreads / 32) + (threadIdx.x >> 5);
-  const int64_t nwarps = (int64_t)gridDim.x * (kQThreads / 32);
+  const int32_t warp = (int32_t)blockIdx.x * (kQThreads / 32) + (threadIdx.x >> 5);
+  const int32_t nwarps = (int32_t)gridDim.x * (kQThreads / 32);
 
   // kUnroll chunks per trip with all loads issued first (memory-level parallelism)
-  for (int64_t ch0 = warp; ch0 < n_chunks; ch0 += kUnroll * nwarps) {
+  for (int32_t ch0 = warp; ch0 < n_chunks; ch0 += kUnroll * nwarps) {
     Raw16 vv[kUnroll];
-    Chunk cc[kUnroll];
+    ChunkT<Idx> cc[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      cc[u] = chunk_at(ch0 + u * nwarps, cpr, cpr_magic, K, lane);
+      cc[u] = chunk_at_t<Idx>(ch0 + u * nwarps, cpr, cpr_magic, K, lane);
       load_raw16(x, cc[u].vec, cc[u].valid && ch0 + u * nwarps < n_chunks, vv[u]);
     }
 #pragma unroll
@@ -446,7 +457,7 @@ __device__ __forceinline__ bool grid_barrier(unsigned long long* ctr, uint64_t t
   return s_ok != 0;
 }
 
-template <class Op>
+template <class Op, bool kNarrow>
 __global__ void __launch_bounds__(kFusedThreads, 1) fused_dynamic_kernel(const uint4* __restrict__ x, int64_t M,
                                                                            int64_t K, uint32_t* partial, uint32_t* bar,
                                                                            Op op, float* g_out, int* status,
@@ -457,23 +468,24 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_dynamic_kernel(const u
   __shared__ int s_bad;
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
+  using Idx = typename std::conditional<kNarrow, uint32_t, int64_t>::type;
   const int32_t cpr = (int32_t)((K + 511) >> 9);
-  const int64_t n_chunks = M * cpr;
-  const int64_t per = (n_chunks + gridDim.x - 1) / gridDim.x;
-  const int64_t lo = (int64_t)blockIdx.x * per;
-  const int64_t hi = lo + per < n_chunks ? lo + per : n_chunks;
-  const int64_t nkeep = hi - lo < kKeepChunks ? (hi - lo > 0 ? hi - lo : 0) : kKeepChunks;
+  const int32_t n_chunks = (int32_t)(M * cpr);  // < 2^31 (checked by the launcher)
+  const int32_t per = (int32_t)(((int64_t)n_chunks + gridDim.x - 1) / gridDim.x);
+  const int32_t lo = (int32_t)min((int64_t)blockIdx.x * per, (int64_t)n_chunks);
+  const int32_t hi = lo + per < n_chunks ? lo + per : n_chunks;
+  const int32_t nkeep = hi - lo < kKeepChunks ? (hi - lo > 0 ? hi - lo : 0) : kKeepChunks;
 
   // ---- phase 1: magnitude maximum, keep the first nkeep chunks
   uint32_t m2 = 0;
-  for (int64_t base = lo + warp; base < hi; base += kLoadUnroll * kFusedWarps) {
+  for (int32_t base = lo + warp; base < hi; base += kLoadUnroll * kFusedWarps) {
     uint4 a[kLoadUnroll], b[kLoadUnroll];
 #pragma unroll
     for (int u = 0; u < kLoadUnroll; ++u) {
-      const int64_t ch = base + u * kFusedWarps;
+      const int32_t ch = base + u * kFusedWarps;
       a[u] = b[u] = make_uint4(0, 0, 0, 0);
       if (ch < hi) {
-        const Chunk c = chunk_at(ch, cpr, cpr_magic, K, lane);
+        const ChunkT<Idx> c = chunk_at_t<Idx>(ch, cpr, cpr_magic, K, lane);
         if (c.valid) {
           a[u] = ld_stream(x + c.vec);
           b[u] = ld_stream(x + c.vec + 1);
@@ -484,7 +496,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_dynamic_kernel(const u
     for (int u = 0; u < kLoadUnroll; ++u) {
       m2 = bmax2(m2, bmax2(bmax2(bmax2(a[u].x, a[u].y), bmax2(a[u].z, a[u].w)),
                            bmax2(bmax2(b[u].x, b[u].y), bmax2(b[u].z, b[u].w))));
-      const int64_t k = base + u * kFusedWarps - lo;
+      const int32_t k = base + u * kFusedWarps - lo;
       if (k < nkeep) {  // lane-contiguous halves: conflict-free 512-byte rows
         keep[k * 64 + lane] = a[u];
         keep[k * 64 + 32 + lane] = b[u];
@@ -532,16 +544,16 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_dynamic_kernel(const u
   }
 
   // ---- phase 2: backwards, re-read chunks that were not kept, then kept ones
-  for (int64_t top = hi - 1 - warp; top >= lo; top -= kFusedUnroll * kFusedWarps) {
+  for (int32_t top = hi - 1 - warp; top >= lo; top -= kFusedUnroll * kFusedWarps) {
     Raw16 vv[kFusedUnroll];
-    Chunk cc[kFusedUnroll];
+    ChunkT<Idx> cc[kFusedUnroll];
 #pragma unroll
     for (int u = 0; u < kFusedUnroll; ++u) {
-      const int64_t ch = top - u * kFusedWarps;
+      const int32_t ch = top - u * kFusedWarps;
       uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
-      cc[u] = chunk_at(ch >= lo ? ch : lo, cpr, cpr_magic, K, lane);
+      cc[u] = chunk_at_t<Idx>(ch >= lo ? ch : lo, cpr, cpr_magic, K, lane);
       if (ch >= lo && cc[u].valid) {
-        const int64_t k = ch - lo;
+        const int32_t k = ch - lo;
         if (k < nkeep) {
           a = keep[k * 64 + lane];
           b = keep[k * 64 + 32 + lane];
@@ -626,12 +638,16 @@ static cudaError_t launch_stream(const void* x, int64_t M, int64_t K, const uint
                                  const float* g_static, const Op& op, float* g_out, int* status, int num_sms,
                                  cudaStream_t s) {
   const int64_t chunks = M * ((K + 511) / 512);
-  if (chunks >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
-  static const int occ = resident_blocks(stream_pass_kernel<Op>, kQThreads, 0);
+  if (chunks >= (int64_t(1) << 30)) return cudaErrorInvalidValue;  // 32-bit chunk loops
+  static const int occ = resident_blocks(stream_pass_kernel<Op, false>, kQThreads, 0);
   const int grid = grid_for(chunks, kQThreads / 32 * kUnroll, num_sms * (occ > 0 ? occ : 1));
   note_launch();
-  stream_pass_kernel<Op><<<grid, kQThreads, 0, s>>>(static_cast<const uint4*>(x), M, K, partial, n_partial, g_static,
-                                                     op, g_out, status, chunk_magic(K));
+  if (narrow_chunks(M, K))
+    stream_pass_kernel<Op, true><<<grid, kQThreads, 0, s>>>(static_cast<const uint4*>(x), M, K, partial, n_partial,
+                                                            g_static, op, g_out, status, chunk_magic_narrow(K));
+  else
+    stream_pass_kernel<Op, false><<<grid, kQThreads, 0, s>>>(static_cast<const uint4*>(x), M, K, partial, n_partial,
+                                                             g_static, op, g_out, status, chunk_magic(K));
   return cudaGetLastError();
 }
 
@@ -641,20 +657,27 @@ template <class Op>
 static cudaError_t launch_fused(const void* x, int64_t M, int64_t K, uint32_t* ws, const Op& op, float* g_out,
                                 int* status, int num_sms, cudaStream_t s) {
   const int64_t chunks = M * ((K + 511) / 512);
-  if (chunks >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
-  static cudaError_t attr = cudaFuncSetAttribute(fused_dynamic_kernel<Op>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                 kFusedSmem);
-  static const int occ = attr == cudaSuccess ? resident_blocks(fused_dynamic_kernel<Op>, kFusedThreads, kFusedSmem) : 0;
-  if (occ < 1 || num_sms > kMaxPartials) return cudaErrorNotSupported;
+  if (chunks >= (int64_t(1) << 30)) return cudaErrorInvalidValue;  // 32-bit chunk loops
+  const bool narrow = narrow_chunks(M, K);
+  const void* kern = narrow ? (const void*)fused_dynamic_kernel<Op, true> : (const void*)fused_dynamic_kernel<Op, false>;
+  static cudaError_t attr_n = cudaFuncSetAttribute(fused_dynamic_kernel<Op, true>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmem);
+  static cudaError_t attr_w = cudaFuncSetAttribute(fused_dynamic_kernel<Op, false>,
+                                                   cudaFuncAttributeMaxDynamicSharedMemorySize, kFusedSmem);
+  static const int occ_n =
+      attr_n == cudaSuccess ? resident_blocks(fused_dynamic_kernel<Op, true>, kFusedThreads, kFusedSmem) : 0;
+  static const int occ_w =
+      attr_w == cudaSuccess ? resident_blocks(fused_dynamic_kernel<Op, false>, kFusedThreads, kFusedSmem) : 0;
+  if ((narrow ? occ_n : occ_w) < 1 || num_sms > kMaxPartials) return cudaErrorNotSupported;
   const uint4* xv = static_cast<const uint4*>(x);
   uint32_t* partial = ws;
   uint32_t* bar = ws + kMaxPartials;
   uint64_t timeout_ns = kFusedTimeoutNs;
-  uint64_t magic = chunk_magic(K);
+  uint64_t magic = narrow ? chunk_magic_narrow(K) : chunk_magic(K);
   void* args[] = {(void*)&xv, (void*)&M, (void*)&K, (void*)&partial, (void*)&bar, (void*)&op, (void*)&g_out,
                   (void*)&status, (void*)&timeout_ns, (void*)&magic};
   note_launch();
-  const cudaError_t e = cudaLaunchCooperativeKernel((const void*)fused_dynamic_kernel<Op>, dim3(num_sms),
+  const cudaError_t e = cudaLaunchCooperativeKernel(kern, dim3(num_sms),
                                                     dim3(kFusedThreads), args, kFusedSmem, s);
   if (e == cudaErrorCooperativeLaunchTooLarge) {
     (void)cudaGetLastError();
@@ -752,27 +775,29 @@ cudaError_t launch_fake_quant_bwd_fused(const void* x, const void* gy, int64_t M
 // K and V stored in NVFP4, QK^T kept in BF16). Same products as fake-quant
 // (d = g*s, then d*q, FP32), so dequantize(quantize(x)) == fake_quant(x).
 // ----------------------------------------------------------------------------
+template <bool kNarrow>
 __global__ void __launch_bounds__(kQThreads) dequantize_kernel(const uint2* __restrict__ codes,
                                                                 const uint8_t* __restrict__ scales,
                                                                 const float* __restrict__ g_ptr, int64_t M,
                                                                 int64_t K, uint64_t cpr_magic, uint4* __restrict__ y) {
+  using Idx = typename std::conditional<kNarrow, uint32_t, int64_t>::type;
   const float g = *g_ptr;
   const int32_t cpr = (int32_t)((K + 511) >> 9);
-  const int64_t n_chunks = M * cpr;
+  const int32_t n_chunks = (int32_t)(M * cpr);  // < 2^31 (checked by the launcher)
   const int lane = threadIdx.x & 31;
-  const int64_t warp = (int64_t)blockIdx.x * (kQThreads / 32) + (threadIdx.x >> 5);
-  const int64_t nwarps = (int64_t)gridDim.x * (kQThreads / 32);
-  for (int64_t ch0 = warp; ch0 < n_chunks; ch0 += kUnroll * nwarps) {
-    Chunk cc[kUnroll];
+  const int32_t warp = (int32_t)blockIdx.x * (kQThreads / 32) + (threadIdx.x >> 5);
+  const int32_t nwarps = (int32_t)gridDim.x * (kQThreads / 32);
+  for (int32_t ch0 = warp; ch0 < n_chunks; ch0 += kUnroll * nwarps) {
+    ChunkT<Idx> cc[kUnroll];
     uint2 q[kUnroll];
     uint32_t sc[kUnroll];
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
-      const int64_t ch = ch0 + u * nwarps;
-      cc[u] = chunk_at(ch < n_chunks ? ch : 0, cpr, cpr_magic, K, lane);
+      const int32_t ch = ch0 + u * nwarps;
+      cc[u] = chunk_at_t<Idx>(ch < n_chunks ? ch : 0, cpr, cpr_magic, K, lane);
       const bool ok = ch < n_chunks && cc[u].valid;
       q[u] = ok ? codes[cc[u].vec >> 1] : make_uint2(0, 0);
-      sc[u] = ok ? scales[scale_offset(cc[u].row, cc[u].col >> 4, K >> 6)] : 1u;
+      sc[u] = ok ? scales[block_scale_offset(cc[u], K)] : 1u;
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
@@ -793,12 +818,16 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const
                               void* y, int num_sms, cudaStream_t s) {
   const int64_t chunks = M * ((K + 511) / 512);
   if (chunks == 0) return cudaSuccess;
-  if (chunks >= (int64_t(1) << 31)) return cudaErrorInvalidValue;
-  static const int occ = resident_blocks(dequantize_kernel, kQThreads, 0);
+  if (chunks >= (int64_t(1) << 30)) return cudaErrorInvalidValue;  // 32-bit chunk loops
+  static const int occ = resident_blocks(dequantize_kernel<false>, kQThreads, 0);
   const int grid = grid_for(chunks, kQThreads / 32 * kUnroll, num_sms * (occ > 0 ? occ : 1));
   note_launch();
-  dequantize_kernel<<<grid, kQThreads, 0, s>>>(reinterpret_cast<const uint2*>(codes), scales, g, M, K,
-                                               chunk_magic(K), static_cast<uint4*>(y));
+  if (narrow_chunks(M, K))
+    dequantize_kernel<true><<<grid, kQThreads, 0, s>>>(reinterpret_cast<const uint2*>(codes), scales, g, M, K,
+                                                       chunk_magic_narrow(K), static_cast<uint4*>(y));
+  else
+    dequantize_kernel<false><<<grid, kQThreads, 0, s>>>(reinterpret_cast<const uint2*>(codes), scales, g, M, K,
+                                                        chunk_magic(K), static_cast<uint4*>(y));
   return cudaGetLastError();
 }
 
