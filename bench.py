@@ -391,7 +391,17 @@ def measure_rows(nv, peaks, flush_buf, stream, iters=10):
     rows["kd_topk_kl"] = {"workload": "2048 x 248320 BF16 teacher/student logits, top-4096 KL per row",
                           "ms": t * 1e3, "GB/s": alg / t / 1e9, "frac_hbm": alg / t / 1e9 / hbm,
                           "algorithmic_bytes": alg}
-    del tl, sl, kl
+    # the training form: loss, the set (idx) and d loss / d student logits on it
+    kidx = torch.empty((R, 4096), dtype=torch.int32, device="cuda")
+    kgrad = torch.empty((R, 4096), dtype=torch.float32, device="cuda")
+    tot, _ = time_loop(lambda ev: nv.topk_kl(tl, sl, 4096, loss_out=kl, idx_out=kidx, grad_out=kgrad),
+                       iters, 2, flush_buf, stream)
+    t = statistics.median(tot) * 1e-3
+    alg = 2.0 * R * V + 2.0 * R * 4096 + 8.0 * R * 4096  # + idx and grad written
+    rows["kd_topk_kl_loss_grad"] = {"workload": "as kd_topk_kl, plus idx [2048x4096] int32 and grad FP32",
+                                    "ms": t * 1e3, "GB/s": alg / t / 1e9, "frac_hbm": alg / t / 1e9 / hbm,
+                                    "algorithmic_bytes": alg}
+    del tl, sl, kl, kidx, kgrad
     torch.cuda.empty_cache()
 
     # lm_head decode: X 128x2048, W 151936x2048 (HBM-bound weight streaming)

@@ -228,9 +228,12 @@ def fake_quant(x: torch.Tensor, mode="max", g: Optional[torch.Tensor] = None,
 
 
 def topk_kl(teacher: torch.Tensor, student: torch.Tensor, k: int, want_idx: bool = False,
-            want_grad: bool = False, loss_out: Optional[torch.Tensor] = None):
+            want_grad: bool = False, loss_out: Optional[torch.Tensor] = None,
+            idx_out: Optional[torch.Tensor] = None, grad_out: Optional[torch.Tensor] = None):
     """Top-k logit KL distillation loss per row (nvfp4_topk_kl). Returns
-    (loss [rows] FP32, idx [rows, k] int32 or None, grad [rows, k] FP32 or None)."""
+    (loss [rows] FP32, idx [rows, k] int32 or None, grad [rows, k] FP32 or None).
+    loss_out / idx_out / grad_out: optional preallocated outputs (idx_out or
+    grad_out given implies want_idx / want_grad)."""
     teacher = _cuda(teacher, "teacher", torch.bfloat16)
     student = _cuda(student, "student", torch.bfloat16)
     if teacher.shape != student.shape or teacher.dim() != 2:
@@ -238,8 +241,14 @@ def topk_kl(teacher: torch.Tensor, student: torch.Tensor, k: int, want_idx: bool
     rows, V = teacher.shape
     dev = teacher.device
     loss = torch.empty(rows, dtype=torch.float32, device=dev) if loss_out is None else loss_out
-    idx = torch.empty((rows, k), dtype=torch.int32, device=dev) if (want_idx or want_grad) else None
-    grad = torch.empty((rows, k), dtype=torch.float32, device=dev) if want_grad else None
+    want_grad = want_grad or grad_out is not None
+    want_idx = want_idx or want_grad or idx_out is not None
+    idx = (torch.empty((rows, k), dtype=torch.int32, device=dev) if idx_out is None else idx_out) if want_idx else None
+    grad = (torch.empty((rows, k), dtype=torch.float32, device=dev) if grad_out is None else grad_out) \
+        if want_grad else None
+    for name, t_, dt in (("idx_out", idx, torch.int32), ("grad_out", grad, torch.float32)):
+        if t_ is not None and (t_.shape != (rows, k) or t_.dtype != dt or not t_.is_contiguous() or t_.device != dev):
+            raise ValueError(f"{name} must be a contiguous [rows, k] {dt} tensor on {dev}")
     _check(lib().nvfp4_topk_kl(_ptr(teacher), _ptr(student), rows, V, k, _ptr(loss), _ptr(idx), _ptr(grad),
                                _stream(dev)), "nvfp4_topk_kl")
     return loss, idx, grad

@@ -79,6 +79,8 @@ struct KdShared {
   uint32_t eq_base, sel_base;
   uint32_t wcount[kKdWarps];  // candidates per warp segment
   uint32_t wtmp[kKdWarps];
+  uint32_t fsel[kKdWarps], feq[kKdWarps];  // fast path: per-warp output base and tie rank base
+  uint32_t fT, fneed;                      // fast path: threshold key and ties taken
   int overflow;
   float red[kKdWarps][5];
   uint16_t ckey[kKdWarps][kCandPerWarp];  // candidate keys, index order within a warp's segment
@@ -391,6 +393,14 @@ __device__ bool kd_fast_row(KdShared& sh, const uint4* trow, const uint16_t* sro
     if (lane == 0) sh.wtmp[warp] = n_eq;
     __syncthreads();
     eq_rank = warp_prefix(sh, warp);
+    if (lane == 0) {  // kept for the gradient pass (kd_fast_grad)
+      sh.fsel[warp] = pos;
+      sh.feq[warp] = eq_rank;
+      if (warp == 0) {
+        sh.fT = T;
+        sh.fneed = need_eq;
+      }
+    }
     for (uint32_t i0 = 0; i0 < mine; i0 += 32) {
       const uint32_t i = i0 + lane;
       const uint32_t key = i < mine ? sh.ckey[warp][i] : 0u;
@@ -405,6 +415,30 @@ __device__ bool kd_fast_row(KdShared& sh, const uint4* trow, const uint16_t* sro
   }
   __syncthreads();
   return true;
+}
+
+// Gradient p_s - p_t of a row the fast path served, written at the same
+// output positions as its idx, from the candidates still in shared memory.
+__device__ void kd_fast_grad(const KdShared& sh, float lse_t, float lse_s, float* grad_row) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const unsigned lt_mask = (1u << lane) - 1u;
+  const uint32_t mine = sh.wcount[warp], T = sh.fT, need_eq = sh.fneed;
+  uint32_t pos = sh.fsel[warp], eq_rank = sh.feq[warp];
+  for (uint32_t i0 = 0; i0 < mine; i0 += 32) {
+    const uint32_t i = i0 + lane;
+    const uint32_t key = i < mine ? sh.ckey[warp][i] : 0u;
+    const unsigned eqm = __ballot_sync(0xFFFFFFFFu, i < mine && key == T);
+    const bool eq = (eqm >> lane) & 1u;
+    const bool sel = i < mine && (key > T || (eq && eq_rank + __popc(eqm & lt_mask) < need_eq));
+    eq_rank += __popc(eqm);
+    const unsigned selm = __ballot_sync(0xFFFFFFFFu, sel);
+    if (sel) {
+      const uint32_t sw = sh.cstu[warp][i];
+      const float sv = __uint_as_float((sh.cidx[warp][i] & 1) ? (sw & 0xFFFF0000u) : (sw << 16));
+      grad_row[pos + __popc(selm & lt_mask)] = expf(sv - lse_s) - expf(kd_value(key) - lse_t);
+    }
+    pos += __popc(selm);
+  }
 }
 
 __global__ void __launch_bounds__(kKdThreads, 2) topk_kl_kernel(const uint4* __restrict__ teacher,
@@ -422,8 +456,9 @@ __global__ void __launch_bounds__(kKdThreads, 2) topk_kl_kernel(const uint4* __r
     const uint4* srow = student + row * nvec;
     KdAcc acc;
     acc.init();
-    if (!kd_fast_row(sh, trow, reinterpret_cast<const uint16_t*>(srow), nvec, k, acc,
-                     idx_out ? idx_out + row * k : nullptr)) {
+    const bool fast = kd_fast_row(sh, trow, reinterpret_cast<const uint16_t*>(srow), nvec, k, acc,
+                                  idx_out ? idx_out + row * k : nullptr);
+    if (!fast) {
     // ---- pass 1: histogram of the key's high byte
     for (int i = t; i < kKdWarps * 256; i += kKdThreads) (&sh.whist[0][0])[i] = 0u;
     __syncthreads();
@@ -578,7 +613,9 @@ __global__ void __launch_bounds__(kKdThreads, 2) topk_kl_kernel(const uint4* __r
     __syncthreads();
 
     // ---- optional pass 4: gradient p_s - p_t at the selected entries
-    if (grad_out && idx_out) {
+    if (grad_out && idx_out && fast) {
+      kd_fast_grad(sh, sh.red[0][0], sh.red[0][1], grad_out + row * k);
+    } else if (grad_out && idx_out) {
       const float lse_t = sh.red[0][0], lse_s = sh.red[0][1];
       const uint16_t* t16 = reinterpret_cast<const uint16_t*>(trow);
       const uint16_t* s16 = reinterpret_cast<const uint16_t*>(srow);

@@ -142,10 +142,15 @@ __global__ void __launch_bounds__(kScanThreads, 1) moe_route_scan_kernel(
   const int e = threadIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int32_t total = 0;
   if (e < E) {
-    for (int c = 0; c < G; ++c) {
-      const int32_t v = cta_count[(int64_t)c * E + e];
-      cta_base[(int64_t)c * E + e] = total;
-      total += v;
+    for (int c0 = 0; c0 < G; c0 += 8) {  // eight independent loads in flight
+      int32_t v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = c0 + u < G ? cta_count[(int64_t)(c0 + u) * E + e] : 0;
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        if (c0 + u < G) cta_base[(int64_t)(c0 + u) * E + e] = total;
+        total += v[u];
+      }
     }
     counts[e] = total;
     amax_x[e] = 0u;

@@ -285,3 +285,38 @@ def test_kv_cache_round_trip(nv):
         np.testing.assert_array_equal(bf16_np(y), ref)
         np.testing.assert_array_equal(to_np(y.view(torch.int16)),
                                       to_np(nv.fake_quant(kv.cuda(), "four_over_six").view(torch.int16)))
+
+
+def test_long_rows_take_the_64bit_chunk_path(nv):
+    # 4 rows of 2^24 + 64 elements: M * (chunks per row)^2 >= 2^32, so every
+    # kernel walks the tensor with 64-bit chunk arithmetic; sampled column
+    # windows (the ragged last chunk included) against the oracle with the
+    # GPU's global scale, which must equal the oracle's over the whole tensor
+    M, K = 4, (1 << 24) + 64
+    gen = torch.Generator().manual_seed(61)
+    x = (torch.randn((M, K), generator=gen) * 0.3).to(torch.bfloat16)
+    x[2, K - 7] = 5.0                                           # amax in the ragged tail
+    xf = bf16_np(x)
+    g_ref = o.global_scale(xf)[0]
+    xd = x.cuda()
+    windows = [0, 512 * 1000 + 64, 1 << 23, K - 4096]
+    for mode in ("max", "four_over_six"):
+        q = nv.quantize(xd, mode)
+        assert to_np(q.g)[0] == g_ref
+        codes = o.unpack_codes(to_np(q.codes))
+        scales = o.scales_from_tiled(to_np(q.scales), M, K)
+        y = bf16_np(nv.fake_quant(xd, mode))
+        for c0 in windows:
+            ref = o.quantize(xf[:, c0:c0 + 4096], mode, g_ref)
+            assert np.array_equal(codes[:, c0:c0 + 4096], ref["codes"])
+            assert np.array_equal(scales[:, c0 // 16:(c0 + 4096) // 16], ref["scales"])
+            fq = o.bf16_round(o.dequantize(ref["codes"], ref["scales"], g_ref))
+            np.testing.assert_array_equal(y[:, c0:c0 + 4096], fq)
+        if mode == "four_over_six":
+            dq = bf16_np(nv.dequantize(q))
+            np.testing.assert_array_equal(dq, y)
+    qs = nv.quantize(xd, "max", g=torch.tensor([np.float32(0.01)]).cuda())  # static g: streaming kernel
+    codes = o.unpack_codes(to_np(qs.codes))
+    for c0 in windows:
+        ref = o.quantize(xf[:, c0:c0 + 4096], "max", np.float32(0.01))
+        assert np.array_equal(codes[:, c0:c0 + 4096], ref["codes"])
