@@ -55,7 +55,7 @@ def load_peaks():
 
 KERNEL_SOURCES = {
     "gemm_dense_mlp": ["common.cuh", "gemm_kernel.cuh", "gemm.cu"],
-    "quantize_dense_mlp": ["common.cuh", "quantize.cu"],
+    "quantize_dense_mlp": ["common.cuh", "block_math.cuh", "kernels.h", "quantize.cu"],
 }
 
 
