@@ -14,6 +14,13 @@
 
 namespace nvfp4 {
 
+// Programmatic dependent launch: wait until the preceding grid has completed
+// and its memory operations are visible (returns at once when this grid was
+// not launched as a programmatic dependent); let the next grid, launched as a
+// programmatic dependent of this one, start its set-up.
+NVFP4_DEVINL void grid_dependency_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+NVFP4_DEVINL void grid_dependents_launch() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
+
 // ----------------------------------------------------------------------------
 // Status word. Kernels get its device address as a parameter and record the
 // first non-OK condition with atomicCAS (later conditions do not overwrite).

@@ -171,9 +171,21 @@ cudaError_t launch_gemm(const uint8_t* Aq, const uint8_t* As, const float* ga, c
   if (encode_store_map_bf16(&tmC, C, (uint64_t)N, (uint64_t)M) != CUDA_SUCCESS) return cudaErrorInvalidValue;
   const int tiles = p.m_tiles * p.n_tiles;
   const int grid = tiles < num_sms ? tiles : num_sms;
+  // Programmatic dependent launch: the CTAs' set-up (barriers, tensor
+  // memory, descriptor prefetch) overlaps the tail of the kernel that wrote A
+  // (the dynamic quantize); the kernel waits for it before reading A.
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kGemmThreads);
+  cfg.dynamicSmemBytes = gemm_smem_bytes<DenseProblem>();
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   note_launch();
-  nvf4_gemm_kernel<DenseProblem><<<grid, kGemmThreads, gemm_smem_bytes<DenseProblem>(), s>>>(tmA, tmB, tmC, p, status, kGemmTimeoutNs);
-  return cudaGetLastError();
+  return cudaLaunchKernelEx(&cfg, nvf4_gemm_kernel<DenseProblem>, tmA, tmB, tmC, p, status, kGemmTimeoutNs);
 }
 
 }  // namespace nvfp4

@@ -142,6 +142,10 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
   if (warp == 0) {
     // ------------------------------------------------------------ producer
     // The whole warp runs the loop (warp-uniform state); elect.sync issues.
+    // Launched as a programmatic dependent of the kernel that wrote A, the
+    // set-up above overlapped that kernel's tail; its outputs are read only
+    // after this wait (a no-op for an ordinary launch).
+    grid_dependency_wait();
     uint32_t stage = 0, phase = 0;
     uint32_t armed = 0;  // bit s: stage s armed; bit 8+s: its phase
     bool ok = true;
@@ -259,6 +263,7 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
     __syncwarp();
   } else {
     // ------------------------------------------------------------ epilogue
+    grid_dependency_wait();          // global scales written by the previous kernel
     const int q = warp & 3;          // tensor-memory lane quarter of this warp
     const int h = (warp - 2) >> 2;   // which half of the tile's columns
     uint32_t acc_phase = 0;

@@ -543,6 +543,8 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_dynamic_kernel(const u
     if (s_bad) record_status(status, NVFP4_ERR_NONFINITE_INPUT);
   }
 
+  grid_dependents_launch();  // a dependent GEMM may set up while phase 2 runs
+
   // ---- phase 2: backwards, re-read chunks that were not kept, then kept ones
   for (int32_t top = hi - 1 - warp; top >= lo; top -= kFusedUnroll * kFusedWarps) {
     Raw16 vv[kFusedUnroll];
