@@ -8,10 +8,11 @@
 // set; loss = KL(p_t || p_s) = sum p_t (t - s) - lse_t + lse_s with
 // p_t = exp(t - lse_t); d loss / d s = p_s - p_t on the set.
 //
-// One CTA of 512 threads per row (persistent over rows, two CTAs per SM). The set is found
-// by a two-digit radix select on order-preserving 16-bit keys of the BF16
-// teacher logits (high byte, then low byte among the high-byte bin that holds
-// the k-th largest), which gives the threshold key T, the count above it, and
+// One CTA of 512 threads per row (persistent over rows, two CTAs per SM).
+// The set is found by a two-digit radix select on order-preserving 16-bit
+// keys of the BF16 teacher logits (high byte, then low byte among the
+// high-byte bin that holds the k-th largest), which gives the threshold key
+// T, the count above it, and
 // how many entries equal to T the set takes (the lowest indices). A third
 // pass walks the row in index order, ranks the entries equal to T with a
 // block scan, and accumulates the two log-sum-exps and sum p_t (t - s)
@@ -28,9 +29,10 @@
 // instruction against T0's value (packed BF16 compare) and works on keys
 // only for the few entries that pass; each candidate's student logit is
 // fetched by an asynchronous 4-byte copy into shared memory issued as the
-// candidate is found, so the gathers overlap the rest of the pass. If the sample undershoots (fewer than k
-// candidates) or a segment overflows its capacity, the row takes the full
-// three-pass path.
+// candidate is found, so the gathers overlap the rest of the pass; the set
+// and the gradient are written from those shared-memory candidates. If the
+// sample undershoots (fewer than k candidates) or a segment overflows its
+// capacity, the row takes the full three-pass path.
 #include <cuda_bf16.h>
 
 #include "common.cuh"
