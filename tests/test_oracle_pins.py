@@ -137,6 +137,27 @@ def test_storage_is_4_5_bits(fmt):
     assert fmt["quantization_recipe"]["block_sizes"]["-1"] == o.BLOCK
 
 
+def test_nibble_order_hand_worked_bytes():
+    """Element 2j goes to the low nibble of byte j: codes [1, 2] (+0.5, +1.0)
+    pack to 0x21, codes [0xA, 0x7] (-1.0, +6.0) to 0x7A; a row quantized from
+    values already on the grid (g*s = 1 exactly) packs the same way."""
+    assert o.pack_codes(np.array([[1, 2]], np.uint8)).tolist() == [[0x21]]
+    assert o.pack_codes(np.array([[0xA, 0x7, 0x0, 0xF]], np.uint8)).tolist() == [[0x7A, 0xF0]]
+    assert o.unpack_codes(np.array([[0x21, 0x7A]], np.uint8)).tolist() == [[1, 2, 0xA, 0x7]]
+    # g = 2^-3 and s = 8 (E4M3 exact) give d = 1: a block whose maximum is 6
+    # keeps the values as codes. Element 0 = 0.5 (code 1), element 1 = 1.0
+    # (code 2), element 2 = -1.0 (code 0xA), element 3 = 6.0 (code 7).
+    x = np.zeros((1, 16), np.float32)
+    x[0, :4] = [0.5, 1.0, -1.0, 6.0]
+    q = o.quantize(x, "max", np.float32(0.125))
+    assert q["scales"].tolist() == [[lib_e4m3_code(8.0)]]
+    assert o.pack_codes(q["codes"])[0, :2].tolist() == [0x21, 0x7A]
+
+
+def lib_e4m3_code(t):
+    return int(np.float32(t).astype(ml_dtypes.float8_e4m3fn).view(np.uint8))
+
+
 @pytest.mark.parametrize("dist", ["normal", "student_t", "outliers", "tiny"])
 @pytest.mark.parametrize("mode", ["max", "four_over_six"])
 def test_scale_audit_invariants(fmt, dist, mode):
@@ -478,6 +499,59 @@ def test_moe_single_expert_is_the_dense_mlp():
     y = gh * gw2 * (ha @ w2a.T)
     assert np.allclose(ref["stages"][0]["gate_up"], gu, rtol=1e-12, atol=1e-15)
     assert np.allclose(ref["out"], y, rtol=1e-9, atol=1e-12)
+
+
+def _loop_expert_mlp(x_rows, q13, q2):
+    """Gated MLP of one expert over the rows routed to it (dynamic activation
+    quantization over exactly those rows), with plain per-element loops and
+    library conversions; returns y [rows, H] in FP64."""
+    def lib_quant(a):
+        g = np.float32(np.float32(np.abs(a).max()) / np.float32(2688.0))
+        out = np.zeros(a.shape, np.float64)
+        for r in range(a.shape[0]):
+            for b in range(a.shape[1] // 16):
+                blk = a[r, 16 * b:16 * b + 16]
+                s = _lib_scale(np.abs(blk).max(), g, 6.0)
+                rr = np.float32(1.0) / np.float32(g * s)
+                out[r, 16 * b:16 * b + 16] = [float(s) * float(lib_e2m1_value(np.float32(v) * rr)) for v in blk]
+        return out, float(g)
+    xa, gx = lib_quant(x_rows)
+    gu = gx * float(q13["g"]) * (xa @ o.dequantize_f64(q13["codes"], q13["scales"]).T)
+    inter = gu.shape[1] // 2
+    h = gu[:, :inter] / (1 + np.exp(-gu[:, :inter])) * gu[:, inter:]
+    h = torch.from_numpy(h).to(torch.bfloat16).double().numpy()
+    ha, gh = lib_quant(h.astype(np.float32))
+    return gh * float(q2["g"]) * (ha @ o.dequantize_f64(q2["codes"], q2["scales"]).T)
+
+
+def test_moe_top2_combine_hand_worked():
+    """k = 2 with distinct routing weights per (token, slot): out[t] =
+    w[t,0] * y_{e0}(t) + w[t,1] * y_{e1}(t), rebuilt token by token from a
+    per-expert loop MLP. Indexing the weights by token instead of by
+    (token, slot) pair, or swapping the slots, changes the result."""
+    rng = np.random.default_rng(15)
+    T, H, I, E = 4, 32, 16, 3
+    x = torch.from_numpy(rng.standard_normal((T, H)).astype(np.float32)).to(torch.bfloat16).float().numpy()
+    ids = np.array([[0, 2], [1, 0], [2, 1], [0, 1]], np.int32)
+    w = np.array([[0.9, 0.1], [0.25, 0.75], [0.6, 0.4], [0.3, 0.7]], np.float32)
+    q13 = [o.quantize((rng.standard_normal((2 * I, H)) * 0.02).astype(np.float32)) for _ in range(E)]
+    q2 = [o.quantize((rng.standard_normal((H, I)) * 0.02).astype(np.float32)) for _ in range(E)]
+    ref = o.moe_reference(x, ids, w, q13, q2)
+    ys = {}
+    for e in range(E):
+        toks = [t for t in range(T) for j in range(2) if ids[t, j] == e]   # stable: token order
+        ys[e] = dict(zip(toks, _loop_expert_mlp(x[toks], q13[e], q2[e])))
+    want = np.zeros((T, H))
+    for t in range(T):
+        for j in range(2):
+            want[t] += float(w[t, j]) * ys[ids[t, j]][t]
+    assert np.allclose(ref["out"], want, rtol=1e-9, atol=1e-12)
+    # the weights matter: the slot-swapped combine is far from it
+    swapped = np.zeros((T, H))
+    for t in range(T):
+        for j in range(2):
+            swapped[t] += float(w[t, 1 - j]) * ys[ids[t, j]][t]
+    assert not np.allclose(ref["out"], swapped, rtol=1e-3, atol=1e-6)
 
 
 # ------------------------------------------------------- QAD backward (STE) ---
