@@ -134,9 +134,9 @@ class ClockSampler:
                 rows.append((ts, float(parts[1]), float(parts[2]), parts[5:9]))
             except ValueError:
                 continue
-        if not rows:
+        inside = [r for r in rows if t0 - 0.05 <= r[0] <= t1 + 0.05]
+        if not inside:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
-        inside = [r for r in rows if t0 - 0.05 <= r[0] <= t1 + 0.05] or rows
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for r in inside for i, v in enumerate(r[3]) if v.lower() == "active"})
         loaded = [r[1] for r in inside]
@@ -198,6 +198,20 @@ def blas_threads():
         return 1
 
 
+def host_cpu():
+    """CPU model and logical core count of the host the oracle runs on."""
+    model = "unknown"
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return {"cpu_model": model, "nproc": os.cpu_count()}
+
+
 def oracle_setup(seed: int, rows: int):
     from oracle import nvfp4_oracle as o
     from qad_nvfp4_quantize_b200 import inputs
@@ -216,7 +230,9 @@ def cpu_baseline(seed: int, rows: int = 96):
     flops = 2.0 * rows * DENSE["N"] * DENSE["K"]
     return {"value": flops / dt / 1e12, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
             "sample": f"{rows} of 4096 activation rows: oracle quantize + FP64 GEMM against all 17408 "
-                      f"statically quantized weight rows ({dt:.1f} s)"}
+                      f"statically quantized weight rows ({dt:.1f} s)",
+            "cores_note": "cores = threads of the BLAS pool the FP64 GEMM runs on; the quantize steps are "
+                          "single-threaded numpy", **host_cpu()}
 
 
 def run_reference(args, rank, world):
@@ -238,13 +254,36 @@ def run_reference(args, rank, world):
             "config": {"workload": "dense_mlp", "M": DENSE["M"], "N": DENSE["N"], "K": DENSE["K"],
                        "step_sample_rows": rows},
             "cpu_baseline": {"value": val, "unit": UNIT, "cores": blas_threads(), "kind": "oracle",
-                             "sample": f"{rows} activation rows per step (oracle quantize + FP64 GEMM)"},
+                             "sample": f"{rows} activation rows per step (oracle quantize + FP64 GEMM)",
+                             **host_cpu()},
             "e2e": {"value": val, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
     return 0
 
 
 # ----------------------------------------------------------------------------- GPU arm
+
+def measure_fp4_peak(nv, stream, sampler, iters=20000, bursts=5):
+    """Best-of-`bursts` rate of the FP4 MMA probe (TFLOP/s), with the SM clock
+    the sampler saw while it ran."""
+    nv.probe_mma_peak(200)                                  # warm-up
+    torch.cuda.synchronize()
+    best = 0.0
+    t0 = time.time()
+    for _ in range(bursts):
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        fl = nv.probe_mma_peak(iters)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        best = max(best, fl / (e0.elapsed_time(e1) * 1e-3) / 1e12)
+    t1 = time.time()
+    if nv.device_status() != 0:
+        raise RuntimeError("the FP4 MMA probe reported a device error")
+    c = sampler.summary(t0, t1)
+    return best, {"tflops": best, "iters": iters, "bursts": bursts, "ms_total": (t1 - t0) * 1e3,
+                  "sm_mhz": c["sm_mhz"], "samples": c["samples"], "reasons": c["reasons"]}
+
 
 def parity_gate(nv, x_dev, xq, wq, w_cpu_rows=None):
     """Verify before timing: quantized activations of sampled rows bit-exact,
@@ -299,12 +338,27 @@ def time_loop(fn, steps, warmup, flush_buf, stream, marks=0, launches=None):
     return total, seg
 
 
-def measure_rows(nv, peaks, flush_buf, stream, iters=10):
+def row_loop(fn, flush_buf, stream, spans, name, min_s=0.25, min_iters=10, max_iters=3000, marks=0):
+    """time_loop for one row, run long enough (about min_s of wall time) for
+    the clock sampler to see it; the row's wall span goes to spans[name]."""
+    tot, _ = time_loop(fn, 2, 2, flush_buf, stream, marks=marks)
+    per = max(statistics.median(tot) * 1e-3 + 60e-6, 1e-6)      # + the L2 flush between steps
+    n = int(min(max_iters, max(min_iters, min_s / per)))
+    t0 = time.time()
+    tot, seg = time_loop(fn, n, 1, flush_buf, stream, marks=marks)
+    spans[name] = (t0, time.time(), n)
+    return tot, seg
+
+
+def measure_rows(nv, peaks, flush_buf, stream, spans, iters=10):
     """Each other hot-path row on its own workload (device time, L2 flushed)."""
     from qad_nvfp4_quantize_b200 import inputs
     rows = {}
     hbm = peaks["hbm"]
-    fp4_peak = peaks["bf16"] * FP4_OVER_BF16
+    fp4_peak = peaks["fp4"]
+
+    def time_loop(fn, steps, warmup, flush_buf, stream, name=None, marks=0):  # noqa: F811 (per-row form)
+        return row_loop(fn, flush_buf, stream, spans, name, marks=marks)
 
     # four_over_six static calibration + QAD fake-quant + W4A4 GEMM (W 14336x4096, X 16384x4096)
     d = inputs.four_over_six_linear(0)
@@ -312,7 +366,7 @@ def measure_rows(nv, peaks, flush_buf, stream, iters=10):
     x = d["x"].cuda()
     del d
     wq = nv.quantize(w, "four_over_six", want_choice=True)
-    tot, _ = time_loop(lambda ev: nv.quantize(w, "four_over_six", want_choice=True, out=wq), iters, 2, flush_buf, stream)
+    tot, _ = time_loop(lambda ev: nv.quantize(w, "four_over_six", want_choice=True, out=wq), iters, 2, flush_buf, stream, name='four_over_six_calibration')
     t = statistics.median(tot) * 1e-3
     n = w.numel()
     alg = n * (2 + 0.5 + 1 / 16 + 1 / 16)     # read W, write codes, scales, choice
@@ -320,7 +374,7 @@ def measure_rows(nv, peaks, flush_buf, stream, iters=10):
                                          "GB/s": alg / t / 1e9, "frac_hbm": alg / t / 1e9 / hbm,
                                          "algorithmic_bytes": alg}
     wq_mse = nv.quantize(w, "mse")
-    tot, _ = time_loop(lambda ev: nv.quantize(w, "mse", out=wq_mse), 3, 1, flush_buf, stream)
+    tot, _ = time_loop(lambda ev: nv.quantize(w, "mse", out=wq_mse), 3, 1, flush_buf, stream, name='mse_calibration')
     t = statistics.median(tot) * 1e-3
     alg = n * (2 + 0.5 + 1 / 16)
     rows["mse_calibration"] = {"workload": "W 14336x4096 BF16, 0.1% entries x20; all 126 E4M3 scales per block "
@@ -329,14 +383,14 @@ def measure_rows(nv, peaks, flush_buf, stream, iters=10):
                                "blocks_per_s": n / 16 / t, "algorithmic_bytes": alg}
     del wq_mse
     y = torch.empty_like(x)
-    tot, _ = time_loop(lambda ev: nv.fake_quant(x, "max", out=y), iters, 2, flush_buf, stream)
+    tot, _ = time_loop(lambda ev: nv.fake_quant(x, "max", out=y), iters, 2, flush_buf, stream, name='fake_quant_dynamic')
     t = statistics.median(tot) * 1e-3
     alg = x.numel() * 4.0
     rows["fake_quant_dynamic"] = {"workload": "X 16384x4096 BF16 -> BF16", "ms": t * 1e3, "GB/s": alg / t / 1e9,
                                   "frac_hbm": alg / t / 1e9 / hbm, "algorithmic_bytes": alg}
     gy = torch.randn_like(x)
     gx = torch.empty_like(x)
-    tot, _ = time_loop(lambda ev: nv.fake_quant_backward(x, gy, "max", out=gx), iters, 2, flush_buf, stream)
+    tot, _ = time_loop(lambda ev: nv.fake_quant_backward(x, gy, "max", out=gx), iters, 2, flush_buf, stream, name='qad_backward_ste_dynamic')
     t = statistics.median(tot) * 1e-3
     alg = x.numel() * 6.0
     rows["qad_backward_ste_dynamic"] = {"workload": "X 16384x4096 BF16 and dL/dy BF16 -> dL/dx BF16 (clipped STE, "
@@ -344,17 +398,33 @@ def measure_rows(nv, peaks, flush_buf, stream, iters=10):
                                         "frac_hbm": alg / t / 1e9 / hbm, "algorithmic_bytes": alg}
     del gy, gx
     xq = nv.quantize(x)
-    tot, _ = time_loop(lambda ev: nv.quantize(x, out=xq), iters, 2, flush_buf, stream)
+    tot, _ = time_loop(lambda ev: nv.quantize(x, out=xq), iters, 2, flush_buf, stream, name='quantize_dynamic_cfg5_x')
     t = statistics.median(tot) * 1e-3
     alg = x.numel() * 2.5625
     rows["quantize_dynamic_cfg5_x"] = {"workload": "X 16384x4096 BF16 (larger than L2)", "ms": t * 1e3,
                                        "GB/s": alg / t / 1e9, "frac_hbm": alg / t / 1e9 / hbm,
                                        "algorithmic_bytes": alg}
     C = torch.empty((x.shape[0], w.shape[0]), dtype=torch.bfloat16, device="cuda")
-    tot, _ = time_loop(lambda ev: nv.gemm(xq, wq, out=C), iters, 2, flush_buf, stream)
+    tot, _ = time_loop(lambda ev: nv.gemm(xq, wq, out=C), iters, 2, flush_buf, stream, name='gemm_fos_16384x14336x4096')
     t = statistics.median(tot) * 1e-3
     fl = 2.0 * x.shape[0] * w.shape[0] * x.shape[1]
     rows["gemm_fos_16384x14336x4096"] = {"ms": t * 1e3, "TFLOP/s": fl / t / 1e12, "frac_fp4_peak": fl / t / 1e12 / fp4_peak}
+
+    # the same linear as one quant+GEMM step (dynamic X quantize, then the
+    # GEMM as its programmatic dependent), timed like the dense_mlp headline
+    def fos_step(ev):
+        nv.quantize(x, out=xq)
+        ev[0].record(stream)
+        nv.gemm(xq, wq, out=C)
+    tot, seg = time_loop(fos_step, iters, 2, flush_buf, stream, name="step_four_over_six_linear", marks=1)
+    t = statistics.median(tot) * 1e-3
+    tq = statistics.median([sg[0] for sg in seg]) * 1e-3
+    tg = statistics.median([sg[1] for sg in seg]) * 1e-3
+    rows["step_four_over_six_linear"] = {
+        "workload": "X 16384x4096 N(0,1) dynamic NVFP4 quantize + GEMM against W 14336x4096 four_over_six",
+        "ms": t * 1e3, "TFLOP/s": fl / t / 1e12, "frac_fp4_peak": fl / t / 1e12 / fp4_peak,
+        "quantize_ms": tq * 1e3, "quantize_frac_hbm": x.numel() * 2.5625 / tq / 1e9 / hbm,
+        "gemm_ms": tg * 1e3, "gemm_frac_fp4_peak": fl / tg / 1e12 / fp4_peak}
     del w, x, y, xq, wq, C
     torch.cuda.empty_cache()
 
@@ -363,12 +433,12 @@ def measure_rows(nv, peaks, flush_buf, stream, iters=10):
     kv = torch.randn((2 * 32768, 1024), device="cuda").to(torch.bfloat16)
     kvq = nv.quantize(kv, "four_over_six")
     kvy = torch.empty_like(kv)
-    tot, _ = time_loop(lambda ev: nv.dequantize(kvq, out=kvy), iters, 2, flush_buf, stream)
+    tot, _ = time_loop(lambda ev: nv.dequantize(kvq, out=kvy), iters, 2, flush_buf, stream, name='kv_cache_dequantize')
     t = statistics.median(tot) * 1e-3
     alg = kv.numel() * (0.5 + 1 / 16 + 2)
     rows["kv_cache_dequantize"] = {"workload": "K,V 2x32768x1024 NVFP4 -> BF16", "ms": t * 1e3, "GB/s": alg / t / 1e9,
                                    "frac_hbm": alg / t / 1e9 / hbm, "algorithmic_bytes": alg}
-    tot, _ = time_loop(lambda ev: nv.quantize(kv, "four_over_six", out=kvq), iters, 2, flush_buf, stream)
+    tot, _ = time_loop(lambda ev: nv.quantize(kv, "four_over_six", out=kvq), iters, 2, flush_buf, stream, name='kv_cache_quantize_fos')
     t = statistics.median(tot) * 1e-3
     alg = kv.numel() * (2 + 0.5 + 1 / 16)
     rows["kv_cache_quantize_fos"] = {"workload": "K,V 2x32768x1024 BF16 -> NVFP4 four_over_six", "ms": t * 1e3,
@@ -385,7 +455,7 @@ def measure_rows(nv, peaks, flush_buf, stream, iters=10):
     sl = (tl + torch.randn((R, V), device="cuda", generator=gen) * 0.5).to(torch.bfloat16)
     tl = tl.to(torch.bfloat16)
     kl = torch.empty(R, dtype=torch.float32, device="cuda")
-    tot, _ = time_loop(lambda ev: nv.topk_kl(tl, sl, 4096, loss_out=kl), iters, 2, flush_buf, stream)
+    tot, _ = time_loop(lambda ev: nv.topk_kl(tl, sl, 4096, loss_out=kl), iters, 2, flush_buf, stream, name='kd_topk_kl')
     t = statistics.median(tot) * 1e-3
     alg = 2.0 * R * V + 2.0 * R * 4096  # teacher rows read once; student logits needed only on the set
     rows["kd_topk_kl"] = {"workload": "2048 x 248320 BF16 teacher/student logits, top-4096 KL per row",
@@ -395,7 +465,7 @@ def measure_rows(nv, peaks, flush_buf, stream, iters=10):
     kidx = torch.empty((R, 4096), dtype=torch.int32, device="cuda")
     kgrad = torch.empty((R, 4096), dtype=torch.float32, device="cuda")
     tot, _ = time_loop(lambda ev: nv.topk_kl(tl, sl, 4096, loss_out=kl, idx_out=kidx, grad_out=kgrad),
-                       iters, 2, flush_buf, stream)
+                       iters, 2, flush_buf, stream, name='kd_topk_kl_loss_grad')
     t = statistics.median(tot) * 1e-3
     alg = 2.0 * R * V + 2.0 * R * 4096 + 8.0 * R * 4096  # + idx and grad written
     rows["kd_topk_kl_loss_grad"] = {"workload": "as kd_topk_kl, plus idx [2048x4096] int32 and grad FP32",
@@ -411,7 +481,7 @@ def measure_rows(nv, peaks, flush_buf, stream, iters=10):
     wq = nv.quantize(w)
     xq = nv.quantize(x)
     C = torch.empty((128, w.shape[0]), dtype=torch.bfloat16, device="cuda")
-    tot, _ = time_loop(lambda ev: nv.gemm(xq, wq, out=C), iters, 2, flush_buf, stream)
+    tot, _ = time_loop(lambda ev: nv.gemm(xq, wq, out=C), iters, 2, flush_buf, stream, name='lm_head_gemm')
     t = statistics.median(tot) * 1e-3
     M, N, K = 128, w.shape[0], 2048
     alg = N * K * 0.5625 + M * K * 0.5625 + M * N * 2
@@ -430,7 +500,7 @@ def measure_rows(nv, peaks, flush_buf, stream, iters=10):
     del d
     out, ws = nv.moe_grouped_gemm(x, ids, tw, 512, w13, g13, w2, g2)
     tot, _ = time_loop(lambda ev: nv.moe_grouped_gemm(x, ids, tw, 512, w13, g13, w2, g2, out=out, workspace=ws),
-                       iters, 2, flush_buf, stream)
+                       iters, 2, flush_buf, stream, name='moe_routed_experts')
     t = statistics.median(tot) * 1e-3
     T, H, E, I = 8192, 2048, 256, 512
     alg = T * H * 2 + E * (2 * I * H + H * I) * 0.5625 + T * H * 4
@@ -474,6 +544,8 @@ def run_gpu(args, rank, world, local):
 
     sampler = ClockSampler(local).start()
     sampler.wait_first(3.0)
+    # the dense FP4 tensor peak, measured: the MMA rate probe (no memory traffic)
+    peaks["fp4"], peaks["fp4_probe"] = measure_fp4_peak(nv, stream, sampler)
     barrier(world)
     torch.cuda.synchronize()
     t_wall0 = time.time()
@@ -483,7 +555,6 @@ def run_gpu(args, rank, world, local):
     barrier(world)
     torch.cuda.synchronize()
     step_ms = dist_max(float(np.mean(total)), world)
-    sampler.stop()
     clocks = sampler.summary(t_wall0, t_wall1)
     quant_ms = float(np.mean([s[0] for s in seg]))
     gemm_ms = float(np.mean([s[1] for s in seg]))
@@ -537,12 +608,15 @@ def run_gpu(args, rank, world, local):
     e2e_val = flops * world / (e2e_ms * 1e-3) / 1e12
     del xs, xqs, C_hosts
 
-    fp4_peak = peaks["bf16"] * FP4_OVER_BF16
+    fp4_peak = peaks["fp4"]
     achieved = flops / (gemm_ms * 1e-3) / 1e12
     roofline = {"bound": "tensor", "kernel": "nvf4_gemm_kernel<DenseProblem>", "achieved": achieved,
                 "peak": fp4_peak, "unit": "TFLOP/s", "frac": achieved / fp4_peak,
                 "traffic": recorded_traffic("gemm_dense_mlp"),
-                "peak_source": f"{peaks['source']} bf16 burst {peaks['bf16']} x {FP4_OVER_BF16} (nominal FP4/BF16)",
+                "peak_source": "measured MMA: nvfp4_probe_mma_peak, kind::mxf4nvf4 128x256x64 back to back on "
+                               "shared-memory operands, one CTA per SM, best of 5 bursts",
+                "peak_probe": peaks["fp4_probe"],
+                "peak_bf16_x4": peaks["bf16"] * FP4_OVER_BF16,
                 "algorithmic_flops_per_launch": flops}
     quant_bytes = M * K * 2.5625
     line = {"metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
@@ -567,7 +641,14 @@ def run_gpu(args, rank, world, local):
                        "samples": clocks["samples"]},
             "wall_s_timed_region": t_wall1 - t_wall0}
     if world == 1 and not args.no_rows:
-        line["rows"] = measure_rows(nv, peaks, flush_buf, stream)
+        del xq, C
+        spans = {}
+        line["rows"] = measure_rows(nv, peaks, flush_buf, stream, spans)
+        for name, (t0, t1, n) in spans.items():
+            c = sampler.summary(t0, t1)
+            line["rows"][name]["iters"] = n
+            line["rows"][name]["clocks"] = {"sm_mhz": c["sm_mhz"], "samples": c["samples"], "reasons": c["reasons"]}
+    sampler.stop()
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(0)
     if rank == 0:

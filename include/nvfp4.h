@@ -90,11 +90,18 @@ const char* nvfp4_status_string(nvfp4_status s);
  * ceil(rows/128) * (K/64) * 512. Returns 0 if K % 64 != 0. Host only. */
 size_t nvfp4_scale_bytes(int64_t rows, int64_t K);
 
-/* Workspace bytes nvfp4_quantize / nvfp4_fake_quant need to compute a dynamic
- * global scale for an [M x K] input (0 is never returned). The workspace
- * holds a grid-wide barrier: zero-fill it once before its first use; every
- * completed call leaves it ready for the next (after a call that reported
- * NVFP4_ERR_TIMEOUT, zero-fill it again). Host only. */
+/* Workspace bytes nvfp4_quantize / nvfp4_fake_quant /
+ * nvfp4_fake_quant_backward need to compute a dynamic global scale for an
+ * [M x K] input (0 is never returned). The workspace holds a grid-wide
+ * barrier whose arrival counter assumes one CTA per SM of one device:
+ *  - zero-fill it once before its first use; every completed call leaves it
+ *    ready for the next;
+ *  - after a call that reported NVFP4_ERR_TIMEOUT, zero-fill it again;
+ *  - use one workspace per device (never hand the same buffer to calls on
+ *    devices with different SM counts);
+ *  - calls that share a workspace must be ordered on the GPU (one stream, or
+ *    events between streams); give each stream its own workspace otherwise.
+ * Host only. */
 size_t nvfp4_quantize_workspace_bytes(int64_t M, int64_t K);
 
 /*
@@ -290,7 +297,9 @@ nvfp4_status nvfp4_moe_workspace_layout(int64_t T, int64_t H, int64_t I, int E, 
  *   enqueue step receives only its input and output pointers, or code that
  *   runs where the device allocator is unavailable or forbidden. (The pages
  *   have no counterpart; this is a deployment convenience.) Same arguments,
- *   outputs and device status as nvfp4_quantize.
+ *   outputs and device status as nvfp4_quantize, except that only modes MAX
+ *   and FOUR_OVER_SIX are accepted (NVFP4_MODE_MSE returns
+ *   NVFP4_ERR_INVALID_ARG).
  * Scratch: the dynamic global scale is reduced through a library-owned static
  *   device array of 4096 32-bit slots (16 KiB, held on every GPU that loads
  *   the library until exit), one slot per 2^18 input elements: M*K may be at
@@ -320,6 +329,29 @@ nvfp4_status nvfp4_get_device_status(nvfp4_stream_t stream, int clear, nvfp4_sta
  * on a flag that nothing sets gives up after `timeout_ns` nanoseconds and
  * records NVFP4_ERR_TIMEOUT in the device status word. */
 nvfp4_status nvfp4_selftest_timeout(uint64_t timeout_ns, nvfp4_stream_t stream);
+
+/* Test hook for the GEMM's own bounded waits: nvfp4_gemm with the same
+ * arguments, except that the TMA producer of the first CTA leaves the first
+ * pipeline stage of its first tile unissued (nothing is copied, nothing is in
+ * flight for it) and every wait gives up after `timeout_ns` (0 < timeout_ns
+ * <= 10 s). The MMA warp's wait on that stage runs out, the CTA records
+ * NVFP4_ERR_TIMEOUT in the device status word, lets its issued copies and
+ * MMAs finish (bounded), frees its tensor memory and returns; C is then
+ * unspecified and the context stays usable. Needs M > 0. The pages have no
+ * counterpart: this exercises the library's failure detection. */
+nvfp4_status nvfp4_selftest_gemm_timeout(const uint8_t* Aq, const uint8_t* As, const float* ga,
+                                         const uint8_t* Bq, const uint8_t* Bs, const float* gb,
+                                         int64_t M, int64_t N, int64_t K, void* C, uint64_t timeout_ns,
+                                         nvfp4_stream_t stream);
+
+/* FP4 tensor-core rate probe (diagnostic; the pages have no counterpart):
+ * launches one CTA per SM that issues `iters` x 4 block-scaled MMAs
+ * (kind::mxf4nvf4, M=128, N=256, K=64 -- the W4A4 GEMM's instruction) on
+ * operands resident in shared memory, with no global-memory traffic, and
+ * waits (bounded) for them. *flops_per_launch (host) receives the launch's
+ * FLOP count, 2*128*256*256*iters*SMs; divided by the launch's duration it
+ * is the measured dense FP4 peak. 1 <= iters <= 2^20. */
+nvfp4_status nvfp4_probe_mma_peak(int iters, double* flops_per_launch, nvfp4_stream_t stream);
 
 /* Number of kernels this library has launched in the process so far, summed
  * over all devices and threads (a host-side counter incremented at every

@@ -20,6 +20,7 @@ __all__ = [
     "check_device", "scale_bytes", "quantize", "fake_quant", "fake_quant_backward", "dequantize", "topk_kl", "gemm", "moe_grouped_gemm",
     "moe_workspace_layout", "convert_e2m1", "convert_e4m3", "device_status", "selftest_timeout",
     "quantize_workspace_bytes", "moe_workspace_bytes", "quantize_experts", "quantize_noalloc",
+    "selftest_gemm_timeout", "kernel_launches", "probe_mma_peak",
 ]
 
 MODE_MAX = 0
@@ -72,7 +73,9 @@ _SIGS = {
     "nvfp4_convert_e4m3": (I32, [P, I64, P, P]),
     "nvfp4_get_device_status": (I32, [P, I32, ctypes.POINTER(ctypes.c_int)]),
     "nvfp4_selftest_timeout": (I32, [U64, P]),
+    "nvfp4_selftest_gemm_timeout": (I32, [P, P, P, P, P, P, I64, I64, I64, P, U64, P]),
     "nvfp4_kernel_launches": (U64, []),
+    "nvfp4_probe_mma_peak": (I32, [I32, ctypes.POINTER(ctypes.c_double), P]),
 }
 
 
@@ -135,18 +138,35 @@ def moe_workspace_bytes(T: int, H: int, I: int, E: int, topk: int) -> int:
     return int(lib().nvfp4_moe_workspace_bytes(T, H, I, E, topk))
 
 
-# Per-device scratch for the amax reduction (the library itself never allocates).
-# It holds a grid barrier and must start zero-filled.
+# Scratch for the dynamic global scale (the library itself never allocates).
+# It holds a grid-wide barrier, so it must start zero-filled and two calls
+# that use it must never overlap on the GPU: one workspace per (device,
+# stream), so calls issued on different streams never share one. After a
+# call reports a timed-out wait the barrier state is stale; device_status()
+# zero-fills every workspace of that device again when it reads that status.
 _ws_cache: dict = {}
+_ws_lock = threading.Lock()
 
 
 def _workspace(device: torch.device, nbytes: int) -> torch.Tensor:
-    key = (device.index, "q")
-    ws = _ws_cache.get(key)
-    if ws is None or ws.numel() < nbytes:
-        ws = torch.zeros(nbytes, dtype=torch.uint8, device=device)
-        _ws_cache[key] = ws
-    return ws
+    stream = torch.cuda.current_stream(device)
+    key = (device.index, stream.cuda_stream)
+    with _ws_lock:
+        entry = _ws_cache.get(key)
+        if entry is None or entry[1].numel() < nbytes:
+            entry = (stream, torch.zeros(nbytes, dtype=torch.uint8, device=device))
+            _ws_cache[key] = entry
+    return entry[1]
+
+
+def _reset_workspaces(device_index: int) -> None:
+    """Zero-fill every cached workspace of one device (after a timed-out wait).
+    Each is cleared on the stream that uses it, after the work queued there."""
+    with _ws_lock:
+        items = [entry for key, entry in _ws_cache.items() if key[0] == device_index]
+    for stream, ws in items:
+        with torch.cuda.stream(stream):
+            ws.zero_()
 
 
 class Quantized(NamedTuple):
@@ -363,16 +383,40 @@ def convert_e4m3(v: torch.Tensor) -> torch.Tensor:
 
 
 def device_status(clear: bool = True, device=None) -> int:
-    """Synchronize the current stream and return (and reset) the device status word."""
+    """Synchronize the current stream and return (and reset) the device status word.
+    A timed-out wait (status 6) also zero-fills this device's cached
+    quantize workspaces, whose grid-barrier counters it left stale."""
     dev = torch.device("cuda", torch.cuda.current_device() if device is None else device)
     v = ctypes.c_int(0)
     _check(lib().nvfp4_get_device_status(_stream(dev), int(clear), ctypes.byref(v)), "nvfp4_get_device_status")
+    if v.value == 6:
+        _reset_workspaces(dev.index)
     return v.value
 
 
 def kernel_launches() -> int:
     """Kernels this library has launched in the process so far (nvfp4_kernel_launches)."""
     return int(lib().nvfp4_kernel_launches())
+
+
+def probe_mma_peak(iters: int, device=None) -> float:
+    """Launch the FP4 MMA rate probe (nvfp4_probe_mma_peak) on the current
+    stream; returns the launch's FLOP count (time it with CUDA events)."""
+    dev = torch.device("cuda", torch.cuda.current_device() if device is None else device)
+    f = ctypes.c_double(0.0)
+    _check(lib().nvfp4_probe_mma_peak(iters, ctypes.byref(f), _stream(dev)), "nvfp4_probe_mma_peak")
+    return f.value
+
+
+def selftest_gemm_timeout(a: Quantized, b: Quantized, timeout_ns: int, out: Optional[torch.Tensor] = None):
+    """nvfp4_selftest_gemm_timeout: the GEMM with its first stage left unissued
+    in one CTA, so that its bounded wait runs out (device status 6)."""
+    dev = b.codes.device
+    C = torch.empty((a.rows, b.rows), dtype=torch.bfloat16, device=dev) if out is None else out
+    _check(lib().nvfp4_selftest_gemm_timeout(_ptr(a.codes), _ptr(a.scales), _ptr(a.g), _ptr(b.codes),
+                                             _ptr(b.scales), _ptr(b.g), a.rows, b.rows, a.K, _ptr(C), timeout_ns,
+                                             _stream(dev)), "nvfp4_selftest_gemm_timeout")
+    return C
 
 
 def selftest_timeout(timeout_ns: int, device=None) -> None:

@@ -273,6 +273,22 @@ nvfp4_status nvfp4_get_device_status(nvfp4_stream_t stream, int clear, nvfp4_sta
 
 uint64_t nvfp4_kernel_launches(void) { return g_launches.load(std::memory_order_relaxed); }
 
+nvfp4_status nvfp4_selftest_gemm_timeout(const uint8_t* Aq, const uint8_t* As, const float* ga, const uint8_t* Bq,
+                                          const uint8_t* Bs, const float* gb, int64_t M, int64_t N, int64_t K,
+                                          void* C, uint64_t timeout_ns, nvfp4_stream_t stream) {
+  if (timeout_ns == 0 || timeout_ns > 10000000000ull) return NVFP4_ERR_INVALID_ARG;  // (0, 10 s]
+  if (M <= 0 || N <= 0 || K <= 0 || K % 64 || N % 16 || M >= (1ll << 31) || N >= (1ll << 31))
+    return NVFP4_ERR_INVALID_ARG;
+  if (!Aq || !As || !ga || !Bq || !Bs || !gb || !C || !aligned16(Aq) || !aligned16(As) || !aligned16(Bq) ||
+      !aligned16(Bs) || !aligned16(C))
+    return NVFP4_ERR_INVALID_ARG;
+  DeviceInfo* d;
+  nvfp4_status st = current_device(&d);
+  if (st != NVFP4_OK) return st;
+  return launched(nvfp4::launch_gemm(Aq, As, ga, Bq, Bs, gb, M, N, K, C, d->status, d->num_sms,
+                                     reinterpret_cast<cudaStream_t>(stream), timeout_ns, 1));
+}
+
 nvfp4_status nvfp4_selftest_timeout(uint64_t timeout_ns, nvfp4_stream_t stream) {
   if (timeout_ns > 10000000000ull) return NVFP4_ERR_INVALID_ARG;  // at most 10 s
   DeviceInfo* d;

@@ -146,8 +146,9 @@ constexpr uint64_t kGemmTimeoutNs = 2000000000ull;  // 2 s per wait: far beyond 
 
 cudaError_t launch_gemm(const uint8_t* Aq, const uint8_t* As, const float* ga, const uint8_t* Bq,
                         const uint8_t* Bs, const float* gb, int64_t M, int64_t N, int64_t K, void* C,
-                        int* status, int num_sms, cudaStream_t s) {
+                        int* status, int num_sms, cudaStream_t s, uint64_t timeout_ns, int skip_first_stage) {
   if (M == 0) return cudaSuccess;
+  if (timeout_ns == 0) timeout_ns = kGemmTimeoutNs;
   CUtensorMap tmA, tmB;
   if (encode_tensor_map_2d(&tmA, Aq, (uint64_t)K / 2, (uint64_t)M, (uint64_t)K / 2, kBK / 2, kBM) != CUDA_SUCCESS)
     return cudaErrorInvalidValue;
@@ -185,7 +186,8 @@ cudaError_t launch_gemm(const uint8_t* Aq, const uint8_t* As, const float* ga, c
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   note_launch();
-  return cudaLaunchKernelEx(&cfg, nvf4_gemm_kernel<DenseProblem>, tmA, tmB, tmC, p, status, kGemmTimeoutNs);
+  return cudaLaunchKernelEx(&cfg, nvf4_gemm_kernel<DenseProblem>, tmA, tmB, tmC, p, status, timeout_ns,
+                            skip_first_stage);
 }
 
 }  // namespace nvfp4

@@ -24,7 +24,10 @@
 // the previous stages may still read.
 // Every mbarrier wait is bounded; on expiry the CTA records
 // NVFP4_ERR_TIMEOUT, drains its in-flight copies and MMAs (bounded) and
-// returns with its tensor memory freed.
+// returns with its tensor memory freed. With `skip_first_stage` set (a test
+// hook), the producer of CTA 0 leaves the first stage of its first tile
+// unissued -- no copy is in flight for it -- so the MMA warp's wait on that
+// stage runs out and the drain path above is taken.
 #pragma once
 
 #include "common.cuh"
@@ -95,7 +98,7 @@ template <class Prob>
 __global__ void __launch_bounds__(kGemmThreads, 1)
     nvf4_gemm_kernel(const __grid_constant__ CUtensorMap tmA, const __grid_constant__ CUtensorMap tmB,
                      const __grid_constant__ CUtensorMap tmC, const Prob prob, int* status,
-                     uint64_t timeout_ns) {
+                     uint64_t timeout_ns, int skip_first_stage) {
   using Lay = GemmSmem<Prob::kPipeStages, Prob::kEpiWarpBytes>;
   constexpr int kStages = Lay::kStages;
   extern __shared__ uint8_t smem_raw[];
@@ -155,6 +158,14 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         if (!mbar_wait_warp(&empty[stage], phase ^ 1, abort_flag, timeout_ns)) {
           ok = false;
           break;
+        }
+        if (skip_first_stage && blockIdx.x == 0 && t == 0 && kt == 0) {
+          // test hook: nothing armed, nothing in flight for this stage
+          if (++stage == kStages) {
+            stage = 0;
+            phase ^= 1;
+          }
+          continue;
         }
         const int nkb = min(4, kgroups - 4 * kt);
         const uint32_t sf_bytes = (uint32_t)nkb * kSFAtom;

@@ -66,10 +66,12 @@ cudaError_t launch_convert(const float* in, int64_t n, uint8_t* out, bool e4m3, 
 cudaError_t launch_selftest_timeout(uint64_t timeout_ns, int* status, cudaStream_t s);
 
 // Dense W4A4 GEMM (gemm.cu). Returns cudaErrorInvalidValue if a tensor map
-// cannot be encoded.
+// cannot be encoded. timeout_ns = 0 takes the library's 2 s wait bound;
+// skip_first_stage != 0 is the bounded-wait test hook (nvf4_gemm_kernel).
 cudaError_t launch_gemm(const uint8_t* Aq, const uint8_t* As, const float* ga, const uint8_t* Bq,
                         const uint8_t* Bs, const float* gb, int64_t M, int64_t N, int64_t K,
-                        void* C, int* status, int num_sms, cudaStream_t s);
+                        void* C, int* status, int num_sms, cudaStream_t s, uint64_t timeout_ns = 0,
+                        int skip_first_stage = 0);
 
 // Routed-expert pipeline (moe.cu).
 struct MoeArgs {

@@ -594,7 +594,7 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
     const int grid = (int)(max_tiles < num_sms ? max_tiles : num_sms);
     note_launch();
     nvf4_gemm_kernel<GateUpProblem><<<grid, kGemmThreads, gemm_smem_bytes<GateUpProblem>(), s>>>(
-        tmA, tmB, tmA /* output map unused: direct stores */, p, status, kMoeTimeoutNs);
+        tmA, tmB, tmA /* output map unused: direct stores */, p, status, kMoeTimeoutNs, 0);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
 
@@ -639,7 +639,7 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
     const int grid = (int)(max_tiles < num_sms ? max_tiles : num_sms);
     note_launch();
     nvf4_gemm_kernel<DownProblem><<<grid, kGemmThreads, gemm_smem_bytes<DownProblem>(), s>>>(
-        tmA, tmB, tmA /* output map unused: bulk reductions */, p, status, kMoeTimeoutNs);
+        tmA, tmB, tmA /* output map unused: bulk reductions */, p, status, kMoeTimeoutNs, 0);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;

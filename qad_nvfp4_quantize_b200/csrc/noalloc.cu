@@ -78,8 +78,14 @@ extern "C" nvfp4_status nvfp4_quantize_noalloc(const void* x, int64_t M, int64_t
   if (!g_in) {
     const nvfp4_status sst = scratch_address(&partial);
     if (sst != NVFP4_OK) return sst;
-    np = (int)((n + kNoallocElemsPerSlot - 1) / kNoallocElemsPerSlot);
-    if (np < 1) np = 1;
+    // as many amax CTAs (one slot each) as the two-pass quantize uses for
+    // its own partials, and at least one per 2^18 elements; never more than
+    // the array holds (n <= 2^30 gives at most kNoallocSlots)
+    int64_t want = (n + kNoallocElemsPerSlot - 1) / kNoallocElemsPerSlot;
+    const int64_t grid = nvfp4::amax_partial_count(n, num_sms);
+    if (want < grid) want = grid;
+    if (want > kNoallocSlots) want = kNoallocSlots;
+    np = (int)(want < 1 ? 1 : want);
     if (nvfp4::launch_amax_partial(x, n, partial, np, s) != cudaSuccess) return NVFP4_ERR_CUDA;
   }
   return nvfp4::launch_quantize(x, M, K, (int)mode, partial, np, g_in, codes, scales,

@@ -70,3 +70,45 @@ def test_gemm_closed_form(nv):
     w = -torch.ones((48, K), dtype=torch.bfloat16, device="cuda")
     C = nv.gemm(nv.quantize(x), nv.quantize(w))
     assert torch.all(C.float() == -K)
+
+
+def test_gemm_bounded_wait_runs_out_and_context_survives(nv):
+    """The first CTA's producer leaves its first stage unissued, so the MMA
+    warp's own bounded wait (1 ms here) runs out: the call reports
+    NVFP4_ERR_TIMEOUT through the device status word, the other CTAs finish
+    their tiles, and the next GEMM on the same context matches the oracle."""
+    rng = np.random.default_rng(77)
+    M, N, K = 512, 1024, 1024                    # 4 x 4 tiles: CTA 0 times out, 15 finish
+    x = inputs.to_bf16((rng.standard_t(3, (M, K)) * 0.5).astype(np.float32))
+    w = inputs.to_bf16((rng.standard_normal((N, K)) * 0.02).astype(np.float32))
+    qa = nv.quantize(x.cuda(), "max")
+    qb = nv.quantize(w.cuda(), "max")
+    assert nv.device_status(clear=True) == 0
+    nv.selftest_gemm_timeout(qa, qb, 1_000_000)
+    assert nv.device_status(clear=True) == 6
+    C = bf16_np(nv.gemm(qa, qb)).astype(np.float64)
+    assert nv.device_status(clear=True) == 0
+    ac, as_, ag = _operands(qa, M, K)
+    bc, bs, bg = _operands(qb, N, K)
+    C_ref, S = o.gemm_reference(ac, as_, ag, bc, bs, bg)
+    gemm_check(C, C_ref, S, "after a timed-out GEMM")
+
+
+def test_dynamic_quantize_on_two_streams(nv):
+    """Two dynamic quantizations issued on two streams with no ordering
+    between them: each stream has its own workspace (grid barrier and amax
+    partials), so each call's global scale equals the oracle's."""
+    rng = np.random.default_rng(78)
+    xs = [inputs.to_bf16((rng.standard_t(3, (2048, 2048)) * s).astype(np.float32)) for s in (0.5, 3.0)]
+    xd = [x.cuda() for x in xs]
+    torch.cuda.synchronize()
+    streams = [torch.cuda.Stream(), torch.cuda.Stream()]
+    outs = [None, None]
+    for _ in range(3):
+        for i in (0, 1):
+            with torch.cuda.stream(streams[i]):
+                outs[i] = nv.quantize(xd[i], "max")
+        torch.cuda.synchronize()
+        for i in (0, 1):
+            assert to_np(outs[i].g)[0] == o.global_scale(bf16_np(xs[i]))[0], i
+    assert nv.device_status(clear=True) == 0
