@@ -338,9 +338,13 @@ def time_loop(fn, steps, warmup, flush_buf, stream, marks=0, launches=None):
     return total, seg
 
 
-def row_loop(fn, flush_buf, stream, spans, name, min_s=0.25, min_iters=10, max_iters=3000, marks=0):
+ROW_MIN_S = 0.25   # wall time per row (--row-min-s)
+
+
+def row_loop(fn, flush_buf, stream, spans, name, min_s=None, min_iters=10, max_iters=3000, marks=0):
     """time_loop for one row, run long enough (about min_s of wall time) for
     the clock sampler to see it; the row's wall span goes to spans[name]."""
+    min_s = ROW_MIN_S if min_s is None else min_s
     tot, _ = time_loop(fn, 2, 2, flush_buf, stream, marks=marks)
     per = max(statistics.median(tot) * 1e-3 + 60e-6, 1e-6)      # + the L2 flush between steps
     n = int(min(max_iters, max(min_iters, min_s / per)))
@@ -606,7 +610,7 @@ def run_gpu(args, rank, world, local):
     torch.cuda.synchronize()
     e2e_ms = dist_max(e0.elapsed_time(e1) / e2e_steps, world)
     e2e_val = flops * world / (e2e_ms * 1e-3) / 1e12
-    del xs, xqs, C_hosts
+    del xs, xqs, C_hosts, Cs
 
     fp4_peak = peaks["fp4"]
     achieved = flops / (gemm_ms * 1e-3) / 1e12
@@ -656,6 +660,74 @@ def run_gpu(args, rank, world, local):
     return 0
 
 
+def kernels_once():
+    """Every library kernel once, at the workloads' sizes, inside a
+    cudaProfilerStart/Stop range (the set-up launches stay outside it): the
+    command the per-kernel ncu summaries under profiles/ are captured from,
+    with ncu --profile-from-start off."""
+    import qad_nvfp4_quantize_b200 as nv
+    from qad_nvfp4_quantize_b200 import inputs
+    torch.cuda.set_device(0)
+    nv.check_device()
+    d = inputs.four_over_six_linear(0)
+    w5, x5 = d["w"].cuda(), d["x"].cuda()                  # W 14336x4096, X 16384x4096
+    del d
+    gy = torch.randn_like(x5)
+    y5, gx5 = torch.empty_like(x5), torch.empty_like(x5)
+    xq5 = nv.quantize(x5)
+    wq5 = nv.quantize(w5, "four_over_six", want_choice=True)
+    wmse = nv.quantize(w5, "mse")
+    kv = torch.randn((2 * 32768, 1024), device="cuda").to(torch.bfloat16)
+    kvq = nv.quantize(kv, "four_over_six")
+    kvy = torch.empty_like(kv)
+    g_static = torch.tensor([0.01], device="cuda")
+    d = inputs.dense_mlp(0)
+    xd, wd = d["x"].cuda(), nv.quantize(d["w"].cuda())
+    del d
+    xqd = nv.quantize(xd)
+    Cd = torch.empty((xd.shape[0], wd.rows), dtype=torch.bfloat16, device="cuda")
+    d = inputs.lm_head(0)
+    wl, xl = nv.quantize(d["w"].cuda()), nv.quantize(d["x"].cuda())
+    del d
+    Cl = torch.empty((128, wl.rows), dtype=torch.bfloat16, device="cuda")
+    m = inputs.moe_experts(0)
+    mx, mids, mw = m["x"].cuda(), m["topk_ids"].cuda(), m["topk_w"].cuda()
+    w13, g13 = nv.quantize_experts(m["w13"].cuda())
+    w2, g2 = nv.quantize_experts(m["w2"].cuda())
+    del m
+    mout, mws = nv.moe_grouped_gemm(mx, mids, mw, 512, w13, g13, w2, g2)
+    R, V = 512, 248320                                     # 508 MB of logits: larger than L2
+    gen = torch.Generator(device="cuda").manual_seed(7)
+    tl = torch.randn((R, V), device="cuda", generator=gen) * 2.0
+    sl = (tl + torch.randn((R, V), device="cuda", generator=gen) * 0.5).to(torch.bfloat16)
+    tl = tl.to(torch.bfloat16)
+    kl = torch.empty(R, dtype=torch.float32, device="cuda")
+    nv.probe_mma_peak(100)
+    torch.cuda.synchronize()
+    torch.cuda.empty_cache()
+    torch.cuda.profiler.start()
+    nv.quantize(xd, "max", out=xqd)                                    # dense_mlp X 4096x5120
+    nv.gemm(xqd, wd, out=Cd)                                           # dense_mlp GEMM (programmatic dependent)
+    nv.quantize(x5, "max", out=xq5)                                    # X 16384x4096
+    nv.quantize(w5, "four_over_six", want_choice=True, out=wq5)        # W 14336x4096 four_over_six
+    nv.fake_quant(x5, "max", out=y5)
+    nv.fake_quant_backward(x5, gy, "max", out=gx5)
+    nv.quantize(w5, "mse", out=wmse)
+    nv.dequantize(kvq, out=kvy)
+    nv.fake_quant(x5, g=xq5.g, scales=xq5.scales, out=y5)             # frozen scales
+    nv.quantize(x5, "max", g=g_static, out=xq5)                        # static global scale
+    nv.gemm(xl, wl, out=Cl)                                            # lm_head 128x151936x2048
+    nv.moe_grouped_gemm(mx, mids, mw, 512, w13, g13, w2, g2, out=mout, workspace=mws)
+    nv.topk_kl(tl, sl, 4096, loss_out=kl)
+    nv.probe_mma_peak(2000)
+    torch.cuda.synchronize()
+    torch.cuda.profiler.stop()
+    if nv.device_status() != 0:
+        raise RuntimeError("a kernel reported a device error")
+    print("kernels-once ok", flush=True)
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -664,7 +736,15 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-rows", action="store_true", help="skip the per-row measurements")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--row-min-s", type=float, default=0.25,
+                    help="wall time each row is timed for (at least 10 steps)")
+    ap.add_argument("--kernels-once", action="store_true",
+                    help="run every library kernel once inside a profiler range (for ncu) and exit")
     args = ap.parse_args()
+    if args.kernels_once:
+        sys.exit(kernels_once())
+    global ROW_MIN_S
+    ROW_MIN_S = args.row_min_s
     if args.warmup < 3:
         args.warmup = 3
     rank, world, local = dist_setup()

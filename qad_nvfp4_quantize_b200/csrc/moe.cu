@@ -8,19 +8,18 @@
 // section "the A4 side: dynamic activations").
 //
 // Pipeline (all on the caller's stream, no host synchronisation):
-//   1 route      stable counting sort of the T*topk (token, slot) pairs by
-//                expert; expert segments padded to 128 rows; per-m-tile
-//                expert table; per-expert amax slots zeroed.
-//   2 token pass per token: row amax -> per-expert amax (atomicMax over the
-//                experts it is routed to); zero the output row.
-//   3 gather+quantize  each padded row gets its token's x quantized with its
-//                expert's dynamic global scale (pad rows: zero codes/scales).
-//   4 gate_up    grouped tcgen05 GEMM; a tile holds 128 gate and the matching
+//   1 front A    per token: row amax -> per-CTA amax of every expert it is
+//                routed to; per-CTA pair counts per expert; zero out[t].
+//   2 front B    (programmatic dependent of A) expert totals, 128-padded
+//                segment offsets, per-expert global scales, a stable sort of
+//                the (token, slot) pairs by expert, and each token's x row
+//                quantized once per routed expert into that expert's rows.
+//   3 gate_up    grouped tcgen05 GEMM; a tile holds 128 gate and the matching
 //                128 up columns; epilogue h = SiLU(gate)*up -> BF16, plus the
-//                per-expert amax of h.
-//   5 quantize h per expert, dynamic global scale.
-//   6 down       grouped tcgen05 GEMM; epilogue scales by the routing weight
-//                and adds into out[token] in FP32 (vector atomics).
+//                per-expert amax of h (pad rows: h = 0, not in the amax).
+//   4 quantize h per expert, dynamic global scale.
+//   5 down       grouped tcgen05 GEMM; epilogue scales by the routing weight
+//                and adds into out[token] in FP32 (bulk reduce-adds).
 #include <mutex>
 
 #include <type_traits>
@@ -41,12 +40,15 @@ int64_t scale_bytes_(int64_t rows, int64_t K) { return ((rows + 127) / 128) * (K
 
 }  // namespace
 
-constexpr int kRouteCtasMax = 128;  // routing CTAs (each owns a contiguous pair range)
+constexpr int kFrontCtasMax = 256;      // front-end CTAs (each owns a contiguous token range)
+constexpr int kFrontThreads = 512;
+constexpr int kFrontWarps = kFrontThreads / 32;
+constexpr int kFrontBatchPairs = 4096;  // (token, slot) pairs placed and quantized per batch
 
 // Workspace layout (all regions 256-byte aligned).
 struct MoeLayout {
-  int64_t R, P;
-  int64_t counts, offsets, cursor, row_pair, tile_expert, tile_count, amax_x, amax_h, cta_count, cta_base;
+  int64_t R, P, Ep;
+  int64_t counts, offsets, row_pair, tile_expert, tile_count, amax_h, cta_count, cta_amax;
   int64_t xq_codes, xq_scales, xq_g, h, hq_codes, hq_scales, hq_g, total;
 };
 
@@ -59,6 +61,7 @@ static MoeLayout moe_layout(int64_t T, int64_t H, int64_t I, int E, int topk) {
   MoeLayout L;
   L.P = T * topk;
   L.R = moe_rows_capacity(T, topk, E);
+  L.Ep = ((int64_t)E + 3) & ~int64_t(3);  // per-CTA table rows padded to 16 bytes
   int64_t o = 0;
   auto take = [&o](int64_t bytes) {
     const int64_t at = o;
@@ -67,14 +70,12 @@ static MoeLayout moe_layout(int64_t T, int64_t H, int64_t I, int E, int topk) {
   };
   L.counts = take(4 * (int64_t)E);
   L.offsets = take(4 * ((int64_t)E + 1));
-  L.cursor = take(4 * (int64_t)E);
   L.row_pair = take(4 * L.R);
   L.tile_expert = take(4 * (L.R / 128));
   L.tile_count = take(4);
-  L.amax_x = take(4 * (int64_t)E);
   L.amax_h = take(4 * (int64_t)E);
-  L.cta_count = take(4 * (int64_t)kRouteCtasMax * E);
-  L.cta_base = take(4 * (int64_t)kRouteCtasMax * E);
+  L.cta_count = take(4 * (int64_t)kFrontCtasMax * L.Ep);
+  L.cta_amax = take(4 * (int64_t)kFrontCtasMax * L.Ep);
   L.xq_codes = take(L.R * H / 2);
   L.xq_scales = take(scale_bytes_(L.R, H));
   L.xq_g = take(4 * (int64_t)E);
@@ -87,209 +88,340 @@ static MoeLayout moe_layout(int64_t T, int64_t H, int64_t I, int E, int topk) {
 }
 
 // ----------------------------------------------------------------------------
-// 1. Routing: a stable counting sort of the P = T*topk pairs by expert, in
-// three launches. G routing CTAs each own the contiguous pair range
-// [c*P/G, (c+1)*P/G).
-//   count  per-CTA expert histograms -> cta_count[c][e]
-//   scan   one CTA: per expert, exclusive prefix over CTAs -> cta_base[c][e],
-//          totals -> counts, 128-padded segment offsets, m-tile -> expert
-//          table, pad rows of row_pair = -1, per-expert amax slots zeroed
-//   place  each CTA ranks its pairs again: per-warp histograms give each
-//          warp its base inside every expert segment, and within a warp pairs
-//          are ranked with __match_any_sync, so the order inside an expert is
-//          increasing pair index (stable).
+// 1. Front pass A. G CTAs; CTA c owns tokens [T*c/G, T*(c+1)/G). Per token:
+// the magnitude maximum of x[t] (BF16 bits & 0x7FFF; Inf and NaN order
+// above every finite value) goes into a shared-memory maximum for every
+// expert the token is routed to, the token's (token, slot) pairs are counted
+// per expert, and its output row is zeroed (the down projection adds into
+// it). The two tables leave as row c of cta_amax and cta_count (rows of Ep
+// entries, the padding zero). Routing ids outside [0, E) are reported and
+// skipped.
 // ----------------------------------------------------------------------------
-constexpr int kRouteThreads = 256;
-constexpr int kRouteWarps = kRouteThreads / 32;
-
-__device__ __forceinline__ void route_range(int64_t P, int G, int c, int64_t& lo, int64_t& hi) {
-  lo = P * c / G;
-  hi = P * (c + 1) / G;
-}
-
-__global__ void __launch_bounds__(kRouteThreads) moe_route_count_kernel(const int32_t* __restrict__ topk_ids,
-                                                                         int64_t P, int E,
-                                                                         int32_t* __restrict__ cta_count,
-                                                                         int* status) {
-  extern __shared__ int32_t hist[];  // [E]
-  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+__global__ void __launch_bounds__(kFrontThreads) moe_front_count_kernel(
+    const uint4* __restrict__ x, int64_t T, int64_t H, const int32_t* __restrict__ topk_ids, int topk, int E,
+    int Ep, int32_t* __restrict__ cta_count, uint32_t* __restrict__ cta_amax, float4* __restrict__ out,
+    int* status) {
+  extern __shared__ uint32_t front_a[];
+  uint32_t* hist = front_a;        // [Ep]
+  uint32_t* amax = front_a + Ep;   // [Ep]
+  for (int e = threadIdx.x; e < Ep; e += blockDim.x) {
+    hist[e] = 0u;
+    amax[e] = 0u;
+  }
   __syncthreads();
-  int64_t lo, hi;
-  route_range(P, gridDim.x, blockIdx.x, lo, hi);
+  grid_dependents_launch();  // front pass B may start its set-up
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int64_t t0 = T * blockIdx.x / gridDim.x, t1 = T * (blockIdx.x + 1) / gridDim.x;
+  const int64_t hv = H / 8;   // 16-byte vectors per row
   bool bad = false;
-  for (int64_t p = lo + threadIdx.x; p < hi; p += blockDim.x) {
-    const int e = topk_ids[p];
-    if (e < 0 || e >= E) {
-      bad = true;
-      continue;
+  for (int64_t t = t0 + warp; t < t1; t += kFrontWarps) {
+    const uint4* row = x + t * hv;
+    uint32_t m2 = 0;
+    for (int64_t i0 = lane; i0 < hv; i0 += 32 * 8) {
+      uint4 v[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = i0 + 32 * u < hv ? ld_stream(row + i0 + 32 * u) : make_uint4(0, 0, 0, 0);
+#pragma unroll
+      for (int u = 0; u < 8; ++u) {
+        m2 = __vmaxu2(m2, v[u].x & 0x7FFF7FFFu);
+        m2 = __vmaxu2(m2, v[u].y & 0x7FFF7FFFu);
+        m2 = __vmaxu2(m2, v[u].z & 0x7FFF7FFFu);
+        m2 = __vmaxu2(m2, v[u].w & 0x7FFF7FFFu);
+      }
     }
-    atomicAdd(&hist[e], 1);
+    uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFullMask, m, o));
+    for (int j = lane; j < topk; j += 32) {
+      const int e = topk_ids[t * topk + j];
+      if (e >= 0 && e < E) {
+        atomicAdd(&hist[e], 1u);
+        atomicMax(&amax[e], m);
+      } else {
+        bad = true;
+      }
+    }
+    float4* orow = out + t * (H / 4);
+    for (int64_t i = lane; i < H / 4; i += 32) orow[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
   if (bad) record_status(status, NVFP4_ERR_INVALID_ARG);
   __syncthreads();
-  for (int e = threadIdx.x; e < E; e += blockDim.x) cta_count[(int64_t)blockIdx.x * E + e] = hist[e];
+  for (int e = threadIdx.x; e < Ep; e += blockDim.x) {
+    cta_count[(int64_t)blockIdx.x * Ep + e] = (int32_t)hist[e];
+    cta_amax[(int64_t)blockIdx.x * Ep + e] = amax[e];
+  }
 }
 
-constexpr int kScanThreads = 1024;
-
-__global__ void __launch_bounds__(kScanThreads, 1) moe_route_scan_kernel(
-    const int32_t* __restrict__ cta_count, int G, int E, int32_t* __restrict__ cta_base,
-    int32_t* __restrict__ counts, int32_t* __restrict__ offsets, int32_t* __restrict__ row_pair,
-    int32_t* __restrict__ tile_expert, int32_t* __restrict__ tile_count, uint32_t* __restrict__ amax_x,
-    uint32_t* __restrict__ amax_h) {
-  __shared__ int32_t seg[kScanThreads + 1];   // padded segment sizes, then offsets
-  __shared__ int32_t wsum[kScanThreads / 32];
-  const int e = threadIdx.x, lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  int32_t total = 0;
-  if (e < E) {
-    for (int c0 = 0; c0 < G; c0 += 8) {  // eight independent loads in flight
-      int32_t v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = c0 + u < G ? cta_count[(int64_t)(c0 + u) * E + e] : 0;
-#pragma unroll
-      for (int u = 0; u < 8; ++u) {
-        if (c0 + u < G) cta_base[(int64_t)(c0 + u) * E + e] = total;
-        total += v[u];
-      }
-    }
-    counts[e] = total;
-    amax_x[e] = 0u;
-    amax_h[e] = 0u;
-  }
-  const int32_t padded = e < E ? (total + 127) & ~127 : 0;
-  // exclusive scan of padded sizes over experts (thread e = expert e)
-  int32_t incl = padded;
+// Exclusive scan over `n` <= 2 * kFrontThreads values held two per thread
+// (v0 at index 2*tid, v1 at 2*tid+1); returns the exclusive prefix of v0.
+// Every thread of the CTA calls it.
+__device__ __forceinline__ int32_t block_excl_scan2(int32_t v0, int32_t v1, int32_t* wsum) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int32_t pair = v0 + v1;
+  int32_t incl = pair;
 #pragma unroll
   for (int o = 1; o < 32; o <<= 1) {
-    const int32_t v = __shfl_up_sync(0xFFFFFFFFu, incl, o);
+    const int32_t v = __shfl_up_sync(kFullMask, incl, o);
     if (lane >= o) incl += v;
   }
   if (lane == 31) wsum[warp] = incl;
   __syncthreads();
   if (warp == 0) {
-    int32_t w = wsum[lane];
+    int32_t w = lane < kFrontWarps ? wsum[lane] : 0;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
-      const int32_t v = __shfl_up_sync(0xFFFFFFFFu, w, o);
+      const int32_t v = __shfl_up_sync(kFullMask, w, o);
       if (lane >= o) w += v;
     }
-    wsum[lane] = w;  // inclusive over warps
+    if (lane < kFrontWarps) wsum[lane] = w;  // inclusive over warps
   }
   __syncthreads();
-  const int32_t excl = incl - padded + (warp > 0 ? wsum[warp - 1] : 0);
-  if (e < E) {
-    offsets[e] = excl;
-    for (int32_t t = excl / 128; t < (excl + padded) / 128; ++t) tile_expert[t] = e;
-    for (int32_t r = excl + total; r < excl + padded; ++r) row_pair[r] = -1;  // pad rows
-  }
-  if (e == E - 1) {
-    offsets[E] = excl + padded;
-    *tile_count = (excl + padded) / 128;
-  }
-}
-
-__global__ void __launch_bounds__(kRouteThreads) moe_route_place_kernel(const int32_t* __restrict__ topk_ids,
-                                                                         int64_t P, int E,
-                                                                         const int32_t* __restrict__ cta_base,
-                                                                         const int32_t* __restrict__ offsets,
-                                                                         int32_t* __restrict__ row_pair) {
-  extern __shared__ int32_t wcount[];  // [kRouteWarps][E]
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (int i = threadIdx.x; i < kRouteWarps * E; i += blockDim.x) wcount[i] = 0;
-  __syncthreads();
-  int64_t lo, hi;
-  route_range(P, gridDim.x, blockIdx.x, lo, hi);
-  const int64_t wlo = lo + (hi - lo) * warp / kRouteWarps, whi = lo + (hi - lo) * (warp + 1) / kRouteWarps;
-  for (int64_t p = wlo + lane; p < whi; p += 32) {
-    const int e = topk_ids[p];
-    if (e >= 0 && e < E) atomicAdd(&wcount[warp * E + e], 1);
-  }
-  __syncthreads();
-  // per expert: segment offset + this CTA's base + exclusive prefix over warps
-  for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    int32_t run = offsets[e] + cta_base[(int64_t)blockIdx.x * E + e];
-    for (int w = 0; w < kRouteWarps; ++w) {
-      const int32_t c = wcount[w * E + e];
-      wcount[w * E + e] = run;
-      run += c;
-    }
-  }
-  __syncthreads();
-  for (int64_t base = wlo; base < whi; base += 32) {
-    const int64_t p = base + lane;
-    int e = p < whi ? topk_ids[p] : -1;
-    if (e >= E) e = -1;
-    const unsigned same = __match_any_sync(kFullMask, e);
-    const int rank = __popc(same & ((1u << lane) - 1u));
-    const int leader = __ffs(same) - 1;
-    if (e >= 0) row_pair[wcount[warp * E + e] + rank] = (int32_t)p;
-    __syncwarp();
-    if (e >= 0 && lane == leader) wcount[warp * E + e] += __popc(same);
-    __syncwarp();
-  }
+  const int32_t r = incl - pair + (warp > 0 ? wsum[warp - 1] : 0);
+  __syncthreads();  // wsum may be reused
+  return r;
 }
 
 // ----------------------------------------------------------------------------
-// 2. Token pass: row amax of x[t] -> atomicMax into the amax of every expert
-// the token is routed to; zero out[t]. One warp per token.
+// 2. Front pass B, a programmatic dependent of pass A on the same G CTAs and
+// token ranges. Every CTA reduces the per-CTA tables over all CTAs (16-byte
+// loads, S row slices per group of four experts): expert totals -> segments
+// padded to 128 rows (exclusive scan over experts), each expert's global
+// scale g = amax/2688 over the rows routed to it, and this CTA's base inside
+// each segment (the pairs of the CTAs before it). CTA 0 publishes counts,
+// offsets, the tile count and the global scales, and zeroes the amax slots
+// of h; the m-tile -> expert entries and pad-row markers of expert e are
+// written by CTA e % G. Then, batch by batch, the CTA ranks its pairs per
+// expert in pair order (per-warp counts, a prefix over warps, and
+// __match_any_sync inside each group of 32 pairs: a stable sort), records the
+// pair of every row, and quantizes each token's row once per routed expert
+// straight into that expert's rows: a row's 16-element blocks are loaded and
+// their maxima taken once, the block scales and codes follow each expert's g.
+// Pad rows of the gathered activations are left as they are: the gate/up
+// epilogue writes zero for them and keeps them out of the amax of h.
 // ----------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) moe_token_pass_kernel(const uint4* __restrict__ x, int64_t T, int64_t H,
-                                                              const int32_t* __restrict__ topk_ids, int topk,
-                                                              int E, uint32_t* __restrict__ amax_x,
-                                                              float4* __restrict__ out) {
-  const int lane = threadIdx.x & 31;
-  const int64_t nw = (int64_t)gridDim.x * (blockDim.x >> 5);
-  for (int64_t t = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); t < T; t += nw) {
-    const uint4* row = x + t * (H / 8);
-    uint32_t m2 = 0;
-    for (int64_t i = lane; i < H / 8; i += 32) {
-      const uint4 v = row[i];
-      m2 = __vmaxu2(m2, v.x & 0x7FFF7FFFu);
-      m2 = __vmaxu2(m2, v.y & 0x7FFF7FFFu);
-      m2 = __vmaxu2(m2, v.z & 0x7FFF7FFFu);
-      m2 = __vmaxu2(m2, v.w & 0x7FFF7FFFu);
+struct FrontB {
+  const uint4* x;
+  int64_t T, H;
+  const int32_t* topk_ids;
+  int topk, E, Ep;
+  const int32_t* cta_count;
+  const uint32_t* cta_amax;
+  int32_t *counts, *offsets, *row_pair, *tile_expert, *tile_count;
+  float* xq_g;
+  uint32_t* amax_h;
+  uint2* xq_codes;
+  uint8_t* xq_scales;
+  int* status;
+};
+
+template <class Idx>
+__global__ void __launch_bounds__(kFrontThreads, 1) moe_front_place_quantize_kernel(const FrontB a) {
+  extern __shared__ int32_t front_b[];
+  const int E = a.E, Ep = a.Ep, topk = a.topk;
+  const int G = gridDim.x, c = blockIdx.x;
+  int32_t* base = front_b;                                  // [Ep]  running row of each expert
+  float* g_s = reinterpret_cast<float*>(base + Ep);        // [Ep]
+  int32_t* wcnt = base + 2 * Ep;                            // [kFrontWarps][Ep]
+  int32_t* pos_s = wcnt + kFrontWarps * Ep;                 // [kFrontBatchPairs]
+  int32_t* exp_s = pos_s + kFrontBatchPairs;                // [kFrontBatchPairs]
+  __shared__ int32_t wsum[kFrontWarps];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+  grid_dependency_wait();  // pass A's tables are complete and visible
+
+  // ---- column reduction of the per-CTA tables: groups of four experts x S row slices
+  {
+    const int groups = Ep / 4;
+    // three [S][Ep] partial tables in the space of wcnt, pos_s and exp_s
+    const int cap = (kFrontWarps * Ep + 2 * kFrontBatchPairs) / (3 * Ep);
+    int S = kFrontThreads / groups;
+    S = S > cap ? cap : S;
+    S = S > G ? G : S;
+    S = S < 1 ? 1 : S;
+    int32_t* tot = wcnt;                    // [S][Ep]
+    int32_t* below = wcnt + S * Ep;         // [S][Ep]
+    uint32_t* mx = reinterpret_cast<uint32_t*>(wcnt + 2 * S * Ep);  // [S][Ep]
+    for (int item = threadIdx.x; item < groups * S; item += blockDim.x) {
+      const int g4 = item % groups, sl = item / groups;
+      const int r0 = G * sl / S, r1 = G * (sl + 1) / S;
+      int4 t4 = make_int4(0, 0, 0, 0), b4 = make_int4(0, 0, 0, 0);
+      uint4 m4 = make_uint4(0, 0, 0, 0);
+      const int4* cc = reinterpret_cast<const int4*>(a.cta_count) + g4;
+      const uint4* ca = reinterpret_cast<const uint4*>(a.cta_amax) + g4;
+#pragma unroll 8
+      for (int r = r0; r < r1; ++r) {
+        const int4 v = __ldcg(cc + (int64_t)r * groups);
+        const uint4 w = __ldcg(ca + (int64_t)r * groups);
+        t4.x += v.x; t4.y += v.y; t4.z += v.z; t4.w += v.w;
+        if (r < c) {
+          b4.x += v.x; b4.y += v.y; b4.z += v.z; b4.w += v.w;
+        }
+        m4.x = max(m4.x, w.x); m4.y = max(m4.y, w.y); m4.z = max(m4.z, w.z); m4.w = max(m4.w, w.w);
+      }
+      int32_t* tp = tot + sl * Ep + 4 * g4;
+      int32_t* bp = below + sl * Ep + 4 * g4;
+      uint32_t* mp = mx + sl * Ep + 4 * g4;
+      tp[0] = t4.x; tp[1] = t4.y; tp[2] = t4.z; tp[3] = t4.w;
+      bp[0] = b4.x; bp[1] = b4.y; bp[2] = b4.z; bp[3] = b4.w;
+      mp[0] = m4.x; mp[1] = m4.y; mp[2] = m4.z; mp[3] = m4.w;
     }
-    uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+    __syncthreads();
+    // thread i owns experts 2i and 2i+1
+    int32_t tv[2] = {0, 0}, bv[2] = {0, 0};
+    uint32_t mv[2] = {0u, 0u};
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFullMask, m, o));
-    if (lane < topk) {
-      const int e = topk_ids[t * topk + lane];
-      if (e >= 0 && e < E) atomicMax(&amax_x[e], m);
+    for (int k = 0; k < 2; ++k) {
+      const int e = 2 * threadIdx.x + k;
+      if (e < E)
+        for (int sl = 0; sl < S; ++sl) {
+          tv[k] += tot[sl * Ep + e];
+          bv[k] += below[sl * Ep + e];
+          mv[k] = max(mv[k], mx[sl * Ep + e]);
+        }
     }
-    float4* orow = out + t * (H / 4);
-    for (int64_t i = lane; i < H / 4; i += 32) orow[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    const int32_t p0 = (tv[0] + 127) & ~127, p1 = (tv[1] + 127) & ~127;
+    const int32_t ex0 = block_excl_scan2(p0, p1, wsum);    // ends with __syncthreads: tables may be reused
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+      const int e = 2 * threadIdx.x + k;
+      if (e >= E) continue;
+      const int32_t off = k == 0 ? ex0 : ex0 + p0;
+      const int32_t padded = k == 0 ? p0 : p1;
+      base[e] = off + bv[k];
+      const float gv = global_scale_from_amax(__uint_as_float(mv[k] << 16));
+      g_s[e] = gv;
+      if (c == 0) {
+        a.counts[e] = tv[k];
+        a.offsets[e] = off;
+        a.xq_g[e] = gv;
+        a.amax_h[e] = 0u;
+        if (mv[k] >= 0x7F80u) record_status(a.status, NVFP4_ERR_NONFINITE_INPUT);
+        if (e == E - 1) {
+          a.offsets[E] = off + padded;
+          *a.tile_count = (off + padded) / 128;
+        }
+      }
+      if (e % G == c) {
+        for (int32_t t = off / 128; t < (off + padded) / 128; ++t) a.tile_expert[t] = e;
+        for (int32_t r = off + tv[k]; r < off + padded; ++r) a.row_pair[r] = -1;  // pad rows
+      }
+    }
+    __syncthreads();
+  }
+
+  // ---- placement and quantization, batch by batch
+  const int64_t t0 = a.T * c / G, t1 = a.T * (c + 1) / G;
+  const int64_t tok_per_batch = kFrontBatchPairs / topk > 0 ? kFrontBatchPairs / topk : 1;
+  const int32_t cpr = (int32_t)((a.H + 511) >> 9);
+  const int64_t hv = a.H / 8;
+  const int64_t kgroups = a.H / 64;
+  for (int64_t tb0 = t0; tb0 < t1; tb0 += tok_per_batch) {
+    const int64_t tb1 = tb0 + tok_per_batch < t1 ? tb0 + tok_per_batch : t1;
+    const int64_t pb0 = tb0 * topk, np = (tb1 - tb0) * topk;
+    for (int i = threadIdx.x; i < kFrontWarps * Ep; i += blockDim.x) wcnt[i] = 0;
+    __syncthreads();
+    const int64_t wlo = pb0 + np * warp / kFrontWarps, whi = pb0 + np * (warp + 1) / kFrontWarps;
+    for (int64_t p = wlo + lane; p < whi; p += 32) {
+      const int e = a.topk_ids[p];
+      if (e >= 0 && e < E) atomicAdd(&wcnt[warp * Ep + e], 1);
+    }
+    __syncthreads();
+    for (int e = threadIdx.x; e < E; e += blockDim.x) {
+      int32_t run = base[e];
+      for (int w = 0; w < kFrontWarps; ++w) {
+        const int32_t n = wcnt[w * Ep + e];
+        wcnt[w * Ep + e] = run;
+        run += n;
+      }
+      base[e] = run;
+    }
+    __syncthreads();
+    for (int64_t q0 = wlo; q0 < whi; q0 += 32) {
+      const int64_t p = q0 + lane;
+      int e = p < whi ? a.topk_ids[p] : -1;
+      if (e >= E) e = -1;
+      const unsigned same = __match_any_sync(kFullMask, e);
+      const int rank = __popc(same & ((1u << lane) - 1u));
+      const int leader = __ffs(same) - 1;
+      int32_t row = -1;
+      if (e >= 0) {
+        row = wcnt[warp * Ep + e] + rank;
+        a.row_pair[row] = (int32_t)p;
+      }
+      if (p < whi) {
+        pos_s[p - pb0] = row;
+        exp_s[p - pb0] = e;
+      }
+      __syncwarp();
+      if (e >= 0 && lane == leader) wcnt[warp * Ep + e] += __popc(same);
+      __syncwarp();
+    }
+    __syncthreads();
+    // one warp per token: its blocks loaded once, quantized once per routed expert
+    for (int64_t t = tb0 + warp; t < tb1; t += kFrontWarps) {
+      const int32_t* pp = pos_s + (t - tb0) * topk;
+      const int32_t* pe = exp_s + (t - tb0) * topk;
+      for (int32_t ch0 = 0; ch0 < cpr; ch0 += 4) {
+        Raw16 raw[4];
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          const int32_t col = (ch0 + u) * 512 + lane * 16;
+          load_raw16(a.x, (Idx)t * (Idx)hv + (Idx)(col >> 3), ch0 + u < cpr && col < a.H, raw[u]);
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+          if (ch0 + u >= cpr) break;  // warp-uniform
+          const int32_t col = (ch0 + u) * 512 + lane * 16;
+          const bool valid = col < a.H;
+          const float bmax = block_absmax(raw[u]);
+          f32x2 xs[8];
+          unpack_block(raw[u], xs);
+          for (int j = 0; j < topk; ++j) {
+            const int e = pe[j];
+            if (e < 0) continue;  // warp-uniform
+            const Idx row = (Idx)pp[j];
+            Block b;
+            quantize_block<false, false>(xs, bmax, g_s[e], 6.0f, b);
+            if (valid) {
+              a.xq_codes[(row * (Idx)a.H + (Idx)col) >> 4] = make_uint2(b.q0, b.q1);
+              a.xq_scales[(((row >> 7) * (Idx)kgroups + (Idx)(col >> 6)) << 9) + ((row & 31) << 4) +
+                          (((row >> 5) & 3) << 2) + (Idx)((col >> 4) & 3)] = (uint8_t)b.sc;
+            }
+          }
+        }
+      }
+    }
+    __syncthreads();  // pos_s / exp_s / wcnt are rewritten by the next batch
   }
 }
 
 // ----------------------------------------------------------------------------
-// 3 / 5. Row-gathered quantization with a per-expert dynamic global scale.
-// A warp's unit is a 512-element chunk of one padded row, one 16-element
-// block per lane (block_math.cuh). Each trip takes kRowUnroll chunks: first
-// their row lookups, then all their (gathered) loads, then the arithmetic, so
-// several chunks' loads are in flight together. Source row of padded row p:
-// kGather ? x[row_pair[p] / topk] : src[p]; pad rows get zero codes and
-// scales. amax_bits[e] is the BF16 magnitude (kGather) or the FP32 bits (h)
-// of expert e's amax; every CTA turns them into global scales in shared
-// memory once.
+// 4. Quantization of h with a per-expert dynamic global scale. A warp's unit
+// is a 512-element chunk of one padded row, one 16-element block per lane
+// (block_math.cuh). Each trip takes kRowUnroll chunks: first their row
+// lookups, then all their loads, then the arithmetic, so several chunks'
+// loads are in flight together. Pad rows get zero codes and scales.
+// amax_bits[e] holds the FP32 bits of expert e's amax of h (written by the
+// gate/up epilogue); every CTA turns them into global scales in shared memory
+// once.
 // ----------------------------------------------------------------------------
 constexpr int kRowThreads = 256;
 constexpr int kRowUnroll = 4;
 
-template <bool kGather, bool kNarrow>
-__global__ void __launch_bounds__(kRowThreads) moe_quantize_rows_kernel(
-    const uint4* __restrict__ src, int64_t K, int topk, const int32_t* __restrict__ row_pair,
+template <bool kNarrow>
+__global__ void __launch_bounds__(kRowThreads) moe_quantize_h_kernel(
+    const uint4* __restrict__ src, int64_t K, const int32_t* __restrict__ row_pair,
     const int32_t* __restrict__ tile_expert, const int32_t* __restrict__ tile_count,
     const uint32_t* __restrict__ amax_bits, int E, uint2* __restrict__ codes, uint8_t* __restrict__ scales,
     float* __restrict__ g_out, int* status, uint64_t cpr_magic) {
   extern __shared__ float g_s[];  // [E]
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    const uint32_t a = amax_bits[e];
-    const float amax = kGather ? __uint_as_float(a << 16) : __uint_as_float(a);
+    const float amax = __uint_as_float(amax_bits[e]);
     const float g = global_scale_from_amax(amax);
     g_s[e] = g;
     if (blockIdx.x == 0) {
       g_out[e] = g;
-      if (kGather ? a >= 0x7F80u : !(amax <= 3.0e38f)) record_status(status, NVFP4_ERR_NONFINITE_INPUT);
+      if (!(amax <= 3.0e38f)) record_status(status, NVFP4_ERR_NONFINITE_INPUT);
     }
   }
   __syncthreads();
@@ -312,10 +444,7 @@ __global__ void __launch_bounds__(kRowThreads) moe_quantize_rows_kernel(
     }
     Raw16 vv[kRowUnroll];
 #pragma unroll
-    for (int u = 0; u < kRowUnroll; ++u) {
-      const Idx srow = kGather ? (Idx)(pr[u] >= 0 ? pr[u] / topk : 0) : cc[u].row;
-      load_raw16(src, (srow * (Idx)K + (Idx)cc[u].col) >> 3, pr[u] >= 0 && cc[u].valid, vv[u]);
-    }
+    for (int u = 0; u < kRowUnroll; ++u) load_raw16(src, cc[u].vec, pr[u] >= 0 && cc[u].valid, vv[u]);
 #pragma unroll
     for (int u = 0; u < kRowUnroll; ++u) {
       if (ch0 + u * nwarps >= n_chunks) break;  // warp-uniform
@@ -334,7 +463,7 @@ __global__ void __launch_bounds__(kRowThreads) moe_quantize_rows_kernel(
 }
 
 // ----------------------------------------------------------------------------
-// 4. gate_up grouped GEMM problem. Tiles are n-fastest: the I/128 column tiles
+// 3. gate_up grouped GEMM problem. Tiles are n-fastest: the I/128 column tiles
 // of one m-tile run on neighbouring CTAs (A read once), and the m-tiles of an
 // expert are adjacent (its weight tiles are re-read from L2).
 // ----------------------------------------------------------------------------
@@ -354,6 +483,7 @@ struct GateUpProblem {
   const float* gb;         // w13_g [E]
   __nv_bfloat16* h;        // [R][I]
   uint32_t* amax_h;
+  const int32_t* row_pair; // -1 marks a pad row
 
   __device__ __forceinline__ int num_tiles() const { return (*tile_count) * n_tiles; }
 
@@ -384,6 +514,9 @@ struct GateUpProblem {
                                         const uint32_t (&acc)[4][32], uint8_t*, const CUtensorMap*) const {
     const int row = job.m0 + q * 32 + lane;
     const float alpha = __fmul_rn(ga[job.expert], gb[job.expert]);
+    // pad rows: their gathered activations were never written, so their
+    // accumulators are meaningless; h gets zeros and stays out of the amax
+    const uint32_t live = row_pair[row] >= 0 ? 0xFFFFFFFFu : 0u;
     __nv_bfloat16* hrow = h + (size_t)row * I + job.n0 + hh * 64;
     uint32_t mx = 0;
 #pragma unroll
@@ -403,7 +536,7 @@ struct GateUpProblem {
             const float silu = __fdividef(z, __fadd_rn(1.0f, __expf(-z)));
             hv[k] = __fmul_rn(silu, up);
           }
-          packed[u] = f32x2_to_bf16x2(hv[0], hv[1]);
+          packed[u] = f32x2_to_bf16x2(hv[0], hv[1]) & live;
           mx = __vmaxu2(mx, packed[u] & 0x7FFF7FFFu);
         }
         *reinterpret_cast<uint4*>(hrow + 32 * j + c) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
@@ -417,7 +550,7 @@ struct GateUpProblem {
 };
 
 // ----------------------------------------------------------------------------
-// 6. down grouped GEMM problem: out[token] += w * (g_h * g_w2) * acc.
+// 5. down grouped GEMM problem: out[token] += w * (g_h * g_w2) * acc.
 // The rows of a tile belong to different tokens, so the sum over a token's
 // experts is a reduction into out. Each epilogue lane stages 32 FP32 values
 // of its row (128 bytes, rows 144 bytes apart so the 32 lanes' writes fall on
@@ -518,58 +651,77 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
   auto I32 = [ws](int64_t off) { return reinterpret_cast<int32_t*>(ws + off); };
   auto U32 = [ws](int64_t off) { return reinterpret_cast<uint32_t*>(ws + off); };
   auto F32 = [ws](int64_t off) { return reinterpret_cast<float*>(ws + off); };
-  const int64_t P = L.P, R = L.R;
+  const int64_t R = L.R;
   if (R * ((a.H + 511) / 512) >= (int64_t(1) << 30) || R * ((a.I + 511) / 512) >= (int64_t(1) << 30))
     return cudaErrorInvalidValue;  // 32-bit chunk loops of the row quantizer
   cudaError_t e;
 
-  // 1. route: count, scan, place
+  // 1-2. front end: per-CTA counts and amax, then placement and quantization
   {
-    int64_t G64 = (P + 511) / 512;
-    const int G = (int)(G64 < 1 ? 1 : (G64 > kRouteCtasMax ? kRouteCtasMax : G64));
+    int G = num_sms < kFrontCtasMax ? num_sms : kFrontCtasMax;
+    if (G < 1) G = 1;
+    const int Ep = (int)L.Ep;
     note_launch();
-    moe_route_count_kernel<<<G, kRouteThreads, (size_t)a.E * sizeof(int32_t), s>>>(a.topk_ids, P, a.E,
-                                                                                    I32(L.cta_count), status);
+    moe_front_count_kernel<<<G, kFrontThreads, (size_t)2 * Ep * sizeof(uint32_t), s>>>(
+        static_cast<const uint4*>(a.x), a.T, a.H, a.topk_ids, a.topk, a.E, Ep, I32(L.cta_count), U32(L.cta_amax),
+        reinterpret_cast<float4*>(a.out), status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    FrontB fb;
+    fb.x = static_cast<const uint4*>(a.x);
+    fb.T = a.T;
+    fb.H = a.H;
+    fb.topk_ids = a.topk_ids;
+    fb.topk = a.topk;
+    fb.E = a.E;
+    fb.Ep = Ep;
+    fb.cta_count = I32(L.cta_count);
+    fb.cta_amax = U32(L.cta_amax);
+    fb.counts = I32(L.counts);
+    fb.offsets = I32(L.offsets);
+    fb.row_pair = I32(L.row_pair);
+    fb.tile_expert = I32(L.tile_expert);
+    fb.tile_count = I32(L.tile_count);
+    fb.xq_g = F32(L.xq_g);
+    fb.amax_h = U32(L.amax_h);
+    fb.xq_codes = reinterpret_cast<uint2*>(ws + L.xq_codes);
+    fb.xq_scales = ws + L.xq_scales;
+    fb.status = status;
+    const size_t smem = (size_t)(2 + kFrontWarps) * Ep * sizeof(int32_t) + 2 * kFrontBatchPairs * sizeof(int32_t);
+    const bool narrow = narrow_chunks(R, a.H) && narrow_chunks(a.T, a.H);
+    const void* kern = narrow ? (const void*)moe_front_place_quantize_kernel<uint32_t>
+                              : (const void*)moe_front_place_quantize_kernel<int64_t>;
+    static std::once_flag once;
+    static cudaError_t attr_err = cudaSuccess;
+    std::call_once(once, [] {
+      const int big = (int)((2 + kFrontWarps) * 1024 * sizeof(int32_t) + 2 * kFrontBatchPairs * sizeof(int32_t));
+      attr_err = cudaFuncSetAttribute(moe_front_place_quantize_kernel<uint32_t>,
+                                      cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+      if (attr_err == cudaSuccess)
+        attr_err = cudaFuncSetAttribute(moe_front_place_quantize_kernel<int64_t>,
+                                        cudaFuncAttributeMaxDynamicSharedMemorySize, big);
+    });
+    if (attr_err != cudaSuccess) return attr_err;
+    // programmatic dependent of pass A: its CTAs start while pass A runs and
+    // wait (griddepcontrol.wait) for pass A's tables before reading them
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(G);
+    cfg.blockDim = dim3(kFrontThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    void* args[] = {(void*)&fb};
     note_launch();
-    moe_route_scan_kernel<<<1, kScanThreads, 0, s>>>(I32(L.cta_count), G, a.E, I32(L.cta_base), I32(L.counts),
-                                                      I32(L.offsets), I32(L.row_pair), I32(L.tile_expert),
-                                                      I32(L.tile_count), U32(L.amax_x), U32(L.amax_h));
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    note_launch();
-    moe_route_place_kernel<<<G, kRouteThreads, (size_t)kRouteWarps * a.E * sizeof(int32_t), s>>>(
-        a.topk_ids, P, a.E, I32(L.cta_base), I32(L.offsets), I32(L.row_pair));
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
-  }
-
-  // 2. token pass
-  {
-    int64_t blocks = (a.T + 7) / 8;
-    if (blocks > (int64_t)num_sms * 8) blocks = (int64_t)num_sms * 8;
-    if (blocks < 1) blocks = 1;
-    note_launch();
-    moe_token_pass_kernel<<<(int)blocks, 256, 0, s>>>(static_cast<const uint4*>(a.x), a.T, a.H, a.topk_ids,
-                                                       a.topk, a.E, U32(L.amax_x), reinterpret_cast<float4*>(a.out));
-    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    if ((e = cudaLaunchKernelExC(&cfg, kern, args)) != cudaSuccess) return e;
   }
 
   const int qgrid = num_sms * 4;
   const size_t qsmem = (size_t)a.E * sizeof(float);
-  // 3. gather + quantize x per expert
-  note_launch();
-  if (narrow_chunks(R, a.H) && narrow_chunks(a.T, a.H))
-    moe_quantize_rows_kernel<true, true><<<qgrid, kRowThreads, qsmem, s>>>(
-        static_cast<const uint4*>(a.x), a.H, a.topk, I32(L.row_pair), I32(L.tile_expert), I32(L.tile_count),
-        U32(L.amax_x), a.E, reinterpret_cast<uint2*>(ws + L.xq_codes), ws + L.xq_scales, F32(L.xq_g), status,
-        chunk_magic_narrow(a.H));
-  else
-    moe_quantize_rows_kernel<true, false><<<qgrid, kRowThreads, qsmem, s>>>(
-        static_cast<const uint4*>(a.x), a.H, a.topk, I32(L.row_pair), I32(L.tile_expert), I32(L.tile_count),
-        U32(L.amax_x), a.E, reinterpret_cast<uint2*>(ws + L.xq_codes), ws + L.xq_scales, F32(L.xq_g), status,
-        chunk_magic(a.H));
-  if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-  // 4. gate_up grouped GEMM
+  // 3. gate_up grouped GEMM
   {
     CUtensorMap tmA, tmB;
     if (encode_tensor_map_2d(&tmA, ws + L.xq_codes, a.H / 2, R, a.H / 2, kBK / 2, kBM) != CUDA_SUCCESS ||
@@ -589,6 +741,7 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
     p.gb = a.w13_g;
     p.h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
     p.amax_h = U32(L.amax_h);
+    p.row_pair = I32(L.row_pair);
     if ((e = prepare_moe_kernel<GateUpProblem>()) != cudaSuccess) return e;
     int64_t max_tiles = (R / 128) * p.n_tiles;
     const int grid = (int)(max_tiles < num_sms ? max_tiles : num_sms);
@@ -598,21 +751,21 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
 
-  // 5. quantize h per expert
+  // 4. quantize h per expert
   note_launch();
   if (narrow_chunks(R, a.I))
-    moe_quantize_rows_kernel<false, true><<<qgrid, kRowThreads, qsmem, s>>>(
-        reinterpret_cast<const uint4*>(ws + L.h), a.I, a.topk, I32(L.row_pair), I32(L.tile_expert),
-        I32(L.tile_count), U32(L.amax_h), a.E, reinterpret_cast<uint2*>(ws + L.hq_codes), ws + L.hq_scales,
-        F32(L.hq_g), status, chunk_magic_narrow(a.I));
+    moe_quantize_h_kernel<true><<<qgrid, kRowThreads, qsmem, s>>>(
+        reinterpret_cast<const uint4*>(ws + L.h), a.I, I32(L.row_pair), I32(L.tile_expert), I32(L.tile_count),
+        U32(L.amax_h), a.E, reinterpret_cast<uint2*>(ws + L.hq_codes), ws + L.hq_scales, F32(L.hq_g), status,
+        chunk_magic_narrow(a.I));
   else
-    moe_quantize_rows_kernel<false, false><<<qgrid, kRowThreads, qsmem, s>>>(
-        reinterpret_cast<const uint4*>(ws + L.h), a.I, a.topk, I32(L.row_pair), I32(L.tile_expert),
-        I32(L.tile_count), U32(L.amax_h), a.E, reinterpret_cast<uint2*>(ws + L.hq_codes), ws + L.hq_scales,
-        F32(L.hq_g), status, chunk_magic(a.I));
+    moe_quantize_h_kernel<false><<<qgrid, kRowThreads, qsmem, s>>>(
+        reinterpret_cast<const uint4*>(ws + L.h), a.I, I32(L.row_pair), I32(L.tile_expert), I32(L.tile_count),
+        U32(L.amax_h), a.E, reinterpret_cast<uint2*>(ws + L.hq_codes), ws + L.hq_scales, F32(L.hq_g), status,
+        chunk_magic(a.I));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
 
-  // 6. down grouped GEMM + weighted FP32 combine
+  // 5. down grouped GEMM + weighted FP32 combine
   {
     CUtensorMap tmA, tmB;
     if (encode_tensor_map_2d(&tmA, ws + L.hq_codes, a.I / 2, R, a.I / 2, kBK / 2, kBM) != CUDA_SUCCESS ||
