@@ -102,5 +102,8 @@ void note_launch();
 CUresult encode_tensor_map_2d(CUtensorMap* map, const void* base, uint64_t inner_bytes,
                               uint64_t rows, uint64_t row_stride_bytes, uint32_t box_inner,
                               uint32_t box_rows);
+// Row-major BF16 [rows][cols] written in 32-row x 16-column boxes from a
+// 32-byte-swizzled staging box (cols * 2 a multiple of 16).
+CUresult encode_store_map_bf16(CUtensorMap* map, void* base, uint64_t cols, uint64_t rows);
 
 }  // namespace nvfp4

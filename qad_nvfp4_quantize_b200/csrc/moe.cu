@@ -44,6 +44,7 @@ constexpr int kFrontCtasMax = 256;      // front-end CTAs (each owns a contiguou
 constexpr int kFrontThreads = 512;
 constexpr int kFrontWarps = kFrontThreads / 32;
 constexpr int kFrontBatchPairs = 4096;  // (token, slot) pairs placed and quantized per batch
+constexpr int kFrontTabExperts = 512;   // per-expert block-step tables in shared memory up to this E
 
 // Workspace layout (all regions 256-byte aligned).
 struct MoeLayout {
@@ -97,7 +98,10 @@ static MoeLayout moe_layout(int64_t T, int64_t H, int64_t I, int E, int topk) {
 // entries, the padding zero). Routing ids outside [0, E) are reported and
 // skipped.
 // ----------------------------------------------------------------------------
-__global__ void __launch_bounds__(kFrontThreads) moe_front_count_kernel(
+constexpr int kCountThreads = 1024;
+constexpr int kCountWarps = kCountThreads / 32;
+
+__global__ void __launch_bounds__(kCountThreads) moe_front_count_kernel(
     const uint4* __restrict__ x, int64_t T, int64_t H, const int32_t* __restrict__ topk_ids, int topk, int E,
     int Ep, int32_t* __restrict__ cta_count, uint32_t* __restrict__ cta_amax, float4* __restrict__ out,
     int* status) {
@@ -114,35 +118,52 @@ __global__ void __launch_bounds__(kFrontThreads) moe_front_count_kernel(
   const int64_t t0 = T * blockIdx.x / gridDim.x, t1 = T * (blockIdx.x + 1) / gridDim.x;
   const int64_t hv = H / 8;   // 16-byte vectors per row
   bool bad = false;
-  for (int64_t t = t0 + warp; t < t1; t += kFrontWarps) {
-    const uint4* row = x + t * hv;
-    uint32_t m2 = 0;
+  // two tokens per warp per trip, all their loads issued first
+  for (int64_t ta = t0 + warp; ta < t1; ta += 2 * kCountWarps) {
+    const int64_t tb = ta + kCountWarps;
+    const uint4* row_a = x + ta * hv;
+    const uint4* row_b = x + (tb < t1 ? tb : ta) * hv;
+    uint32_t ma2 = 0, mb2 = 0;
     for (int64_t i0 = lane; i0 < hv; i0 += 32 * 8) {
-      uint4 v[8];
-#pragma unroll
-      for (int u = 0; u < 8; ++u) v[u] = i0 + 32 * u < hv ? ld_stream(row + i0 + 32 * u) : make_uint4(0, 0, 0, 0);
+      uint4 va[8], vb[8];
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
-        m2 = __vmaxu2(m2, v[u].x & 0x7FFF7FFFu);
-        m2 = __vmaxu2(m2, v[u].y & 0x7FFF7FFFu);
-        m2 = __vmaxu2(m2, v[u].z & 0x7FFF7FFFu);
-        m2 = __vmaxu2(m2, v[u].w & 0x7FFF7FFFu);
+        const bool in = i0 + 32 * u < hv;
+        va[u] = in ? ld_stream(row_a + i0 + 32 * u) : make_uint4(0, 0, 0, 0);
+        vb[u] = in && tb < t1 ? ld_stream(row_b + i0 + 32 * u) : make_uint4(0, 0, 0, 0);
       }
-    }
-    uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFullMask, m, o));
-    for (int j = lane; j < topk; j += 32) {
-      const int e = topk_ids[t * topk + j];
-      if (e >= 0 && e < E) {
-        atomicAdd(&hist[e], 1u);
-        atomicMax(&amax[e], m);
-      } else {
-        bad = true;
+      for (int u = 0; u < 8; ++u) {
+        ma2 = __vmaxu2(ma2, va[u].x & 0x7FFF7FFFu);
+        ma2 = __vmaxu2(ma2, va[u].y & 0x7FFF7FFFu);
+        ma2 = __vmaxu2(ma2, va[u].z & 0x7FFF7FFFu);
+        ma2 = __vmaxu2(ma2, va[u].w & 0x7FFF7FFFu);
+        mb2 = __vmaxu2(mb2, vb[u].x & 0x7FFF7FFFu);
+        mb2 = __vmaxu2(mb2, vb[u].y & 0x7FFF7FFFu);
+        mb2 = __vmaxu2(mb2, vb[u].z & 0x7FFF7FFFu);
+        mb2 = __vmaxu2(mb2, vb[u].w & 0x7FFF7FFFu);
       }
     }
-    float4* orow = out + t * (H / 4);
-    for (int64_t i = lane; i < H / 4; i += 32) orow[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int side = 0; side < 2; ++side) {
+      const int64_t t = side ? tb : ta;
+      if (t >= t1) break;  // warp-uniform
+      const uint32_t m2 = side ? mb2 : ma2;
+      uint32_t m = max(m2 & 0xFFFFu, m2 >> 16);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) m = max(m, __shfl_xor_sync(kFullMask, m, o));
+      for (int j = lane; j < topk; j += 32) {
+        const int e = topk_ids[t * topk + j];
+        if (e >= 0 && e < E) {
+          atomicAdd(&hist[e], 1u);
+          atomicMax(&amax[e], m);
+        } else {
+          bad = true;
+        }
+      }
+      float4* orow = out + t * (H / 4);
+      for (int64_t i = lane; i < H / 4; i += 32) orow[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
   }
   if (bad) record_status(status, NVFP4_ERR_INVALID_ARG);
   __syncthreads();
@@ -224,6 +245,7 @@ __global__ void __launch_bounds__(kFrontThreads, 1) moe_front_place_quantize_ker
   int32_t* wcnt = base + 2 * Ep;                            // [kFrontWarps][Ep]
   int32_t* pos_s = wcnt + kFrontWarps * Ep;                 // [kFrontBatchPairs]
   int32_t* exp_s = pos_s + kFrontBatchPairs;                // [kFrontBatchPairs]
+  GStep* gst = reinterpret_cast<GStep*>(exp_s + kFrontBatchPairs);  // [E] when E <= kFrontTabExperts
   __shared__ int32_t wsum[kFrontWarps];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
@@ -307,6 +329,9 @@ __global__ void __launch_bounds__(kFrontThreads, 1) moe_front_place_quantize_ker
       }
     }
     __syncthreads();
+    if (E <= kFrontTabExperts)
+      for (int i = threadIdx.x; i < E * 16; i += blockDim.x) gstep_fill(gst[i >> 4], g_s[i >> 4], i & 15);
+    __syncthreads();
   }
 
   // ---- placement and quantization, batch by batch
@@ -381,7 +406,10 @@ __global__ void __launch_bounds__(kFrontThreads, 1) moe_front_place_quantize_ker
             if (e < 0) continue;  // warp-uniform
             const Idx row = (Idx)pp[j];
             Block b;
-            quantize_block<false, false>(xs, bmax, g_s[e], 6.0f, b);
+            if (E <= kFrontTabExperts && gstep_valid(g_s[e]))  // warp-uniform
+              quantize_block_gstep(xs, bmax, gst[e], b);
+            else
+              quantize_block<false, false>(xs, bmax, g_s[e], 6.0f, b);
             if (valid) {
               a.xq_codes[(row * (Idx)a.H + (Idx)col) >> 4] = make_uint2(b.q0, b.q1);
               a.xq_scales[(((row >> 7) * (Idx)kgroups + (Idx)(col >> 6)) << 9) + ((row & 31) << 4) +
@@ -407,6 +435,7 @@ __global__ void __launch_bounds__(kFrontThreads, 1) moe_front_place_quantize_ker
 // ----------------------------------------------------------------------------
 constexpr int kRowThreads = 256;
 constexpr int kRowUnroll = 4;
+constexpr int kHTabExperts = 256;  // block-step tables in shared memory up to this E
 
 template <bool kNarrow>
 __global__ void __launch_bounds__(kRowThreads) moe_quantize_h_kernel(
@@ -414,7 +443,8 @@ __global__ void __launch_bounds__(kRowThreads) moe_quantize_h_kernel(
     const int32_t* __restrict__ tile_expert, const int32_t* __restrict__ tile_count,
     const uint32_t* __restrict__ amax_bits, int E, uint2* __restrict__ codes, uint8_t* __restrict__ scales,
     float* __restrict__ g_out, int* status, uint64_t cpr_magic) {
-  extern __shared__ float g_s[];  // [E]
+  extern __shared__ float g_s[];  // [E], then (E <= kHTabExperts) the block-step tables [E]
+  GStep* gst = reinterpret_cast<GStep*>(g_s + ((E + 3) & ~3));
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     const float amax = __uint_as_float(amax_bits[e]);
     const float g = global_scale_from_amax(amax);
@@ -425,6 +455,11 @@ __global__ void __launch_bounds__(kRowThreads) moe_quantize_h_kernel(
     }
   }
   __syncthreads();
+  const bool tab = E <= kHTabExperts;
+  if (tab) {
+    for (int i = threadIdx.x; i < E * 16; i += blockDim.x) gstep_fill(gst[i >> 4], g_s[i >> 4], i & 15);
+    __syncthreads();
+  }
   using Idx = typename std::conditional<kNarrow, uint32_t, int64_t>::type;
   const int lane = threadIdx.x & 31;
   const int32_t rows = (*tile_count) * 128;
@@ -450,7 +485,14 @@ __global__ void __launch_bounds__(kRowThreads) moe_quantize_h_kernel(
       if (ch0 + u * nwarps >= n_chunks) break;  // warp-uniform
       Block b;
       if (pr[u] >= 0) {
-        quantize_block<false, false>(vv[u], block_absmax(vv[u]), g_s[ex[u]], 6.0f, b);
+        const float gv = g_s[ex[u]];
+        if (tab && gstep_valid(gv)) {  // warp-uniform: a chunk lies in one row
+          f32x2 xs[8];
+          unpack_block(vv[u], xs);
+          quantize_block_gstep(xs, block_absmax(vv[u]), gst[ex[u]], b);
+        } else {
+          quantize_block<false, false>(vv[u], block_absmax(vv[u]), gv, 6.0f, b);
+        }
       } else {
         b.sc = b.q0 = b.q1 = 0u;  // pad row: zero codes and scales, no arithmetic
       }
@@ -469,7 +511,7 @@ __global__ void __launch_bounds__(kRowThreads) moe_quantize_h_kernel(
 // ----------------------------------------------------------------------------
 struct GateUpProblem {
   static constexpr int kPipeStages = 4;
-  static constexpr uint32_t kEpiWarpBytes = 0;  // direct stores
+  static constexpr uint32_t kEpiWarpBytes = kEpiBytes;  // 32 x 16 BF16 staging box per warp
   int K;             // H
   int I;
   int n_tiles;       // I / 128
@@ -510,19 +552,26 @@ struct GateUpProblem {
     return (uint32_t)(j < 2 ? h * 64 + 32 * j : 128 + h * 64 + 32 * (j - 2));
   }
 
+  // Epilogue of one warp (rows q*32.., gate columns hh*64..): h =
+  // SiLU(gate)*up in BF16, written through the warp's shared staging box
+  // (32 rows x 16 columns, 32-byte swizzle) with TMA stores, so each tile's h
+  // leaves as whole 32-byte row pieces; plus the per-expert amax of h.
   __device__ __forceinline__ void store(const TileJob& job, int q, int hh, int lane,
-                                        const uint32_t (&acc)[4][32], uint8_t*, const CUtensorMap*) const {
-    const int row = job.m0 + q * 32 + lane;
+                                        const uint32_t (&acc)[4][32], uint8_t* stg, const CUtensorMap* tmH) const {
+    const int row0 = job.m0 + q * 32;
     const float alpha = __fmul_rn(ga[job.expert], gb[job.expert]);
     // pad rows: their gathered activations were never written, so their
     // accumulators are meaningless; h gets zeros and stays out of the amax
-    const uint32_t live = row_pair[row] >= 0 ? 0xFFFFFFFFu : 0u;
-    __nv_bfloat16* hrow = h + (size_t)row * I + job.n0 + hh * 64;
+    const uint32_t live = row_pair[row0 + lane] >= 0 ? 0xFFFFFFFFu : 0u;
+    const uint32_t sbase = smem_u32(stg);
     uint32_t mx = 0;
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
+    for (int c0 = 0; c0 < 64; c0 += kEpiCols) {
+      if (lane == 0) bulk_wait_read_all();  // the previous box has left shared memory
+      __syncwarp();
 #pragma unroll
-      for (int c = 0; c < 32; c += 8) {
+      for (int ch = 0; ch < kEpiCols / 8; ++ch) {
+        const int j = (c0 + ch * 8) / 32, c = (c0 + ch * 8) % 32;
         uint32_t packed[4];
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -539,7 +588,15 @@ struct GateUpProblem {
           packed[u] = f32x2_to_bf16x2(hv[0], hv[1]) & live;
           mx = __vmaxu2(mx, packed[u] & 0x7FFF7FFFu);
         }
-        *reinterpret_cast<uint4*>(hrow + 32 * j + c) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        // 32-byte swizzle: 16-byte chunk index XOR bit 2 of the row
+        st_shared_v4(sbase + lane * (kEpiCols * 2) + ((ch ^ ((lane >> 2) & 1)) << 4),
+                     make_uint4(packed[0], packed[1], packed[2], packed[3]));
+      }
+      fence_proxy_async_smem();
+      __syncwarp();
+      if (lane == 0) {
+        tma_store_2d(tmH, stg, job.n0 + hh * 64 + c0, row0);
+        bulk_commit_group();
       }
     }
     uint32_t m = max(mx & 0xFFFFu, mx >> 16);
@@ -662,7 +719,7 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
     if (G < 1) G = 1;
     const int Ep = (int)L.Ep;
     note_launch();
-    moe_front_count_kernel<<<G, kFrontThreads, (size_t)2 * Ep * sizeof(uint32_t), s>>>(
+    moe_front_count_kernel<<<G, kCountThreads, (size_t)2 * Ep * sizeof(uint32_t), s>>>(
         static_cast<const uint4*>(a.x), a.T, a.H, a.topk_ids, a.topk, a.E, Ep, I32(L.cta_count), U32(L.cta_amax),
         reinterpret_cast<float4*>(a.out), status);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -686,14 +743,18 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
     fb.xq_codes = reinterpret_cast<uint2*>(ws + L.xq_codes);
     fb.xq_scales = ws + L.xq_scales;
     fb.status = status;
-    const size_t smem = (size_t)(2 + kFrontWarps) * Ep * sizeof(int32_t) + 2 * kFrontBatchPairs * sizeof(int32_t);
+    const size_t smem = (size_t)(2 + kFrontWarps) * Ep * sizeof(int32_t) + 2 * kFrontBatchPairs * sizeof(int32_t) +
+                        (a.E <= kFrontTabExperts ? (size_t)a.E * sizeof(GStep) : 0);
     const bool narrow = narrow_chunks(R, a.H) && narrow_chunks(a.T, a.H);
     const void* kern = narrow ? (const void*)moe_front_place_quantize_kernel<uint32_t>
                               : (const void*)moe_front_place_quantize_kernel<int64_t>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-      const int big = (int)((2 + kFrontWarps) * 1024 * sizeof(int32_t) + 2 * kFrontBatchPairs * sizeof(int32_t));
+      const size_t tab = (size_t)(2 + kFrontWarps) * 512 * sizeof(int32_t) + 2 * kFrontBatchPairs * sizeof(int32_t) +
+                         (size_t)kFrontTabExperts * sizeof(GStep);
+      const size_t notab = (size_t)(2 + kFrontWarps) * 1024 * sizeof(int32_t) + 2 * kFrontBatchPairs * sizeof(int32_t);
+      const int big = (int)(tab > notab ? tab : notab);
       attr_err = cudaFuncSetAttribute(moe_front_place_quantize_kernel<uint32_t>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, big);
       if (attr_err == cudaSuccess)
@@ -719,7 +780,8 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
   }
 
   const int qgrid = num_sms * 4;
-  const size_t qsmem = (size_t)a.E * sizeof(float);
+  const size_t qsmem = (size_t)((a.E + 3) & ~3) * sizeof(float) +
+                       (a.E <= kHTabExperts ? (size_t)a.E * sizeof(GStep) : 0);
 
   // 3. gate_up grouped GEMM
   {
@@ -743,11 +805,13 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
     p.amax_h = U32(L.amax_h);
     p.row_pair = I32(L.row_pair);
     if ((e = prepare_moe_kernel<GateUpProblem>()) != cudaSuccess) return e;
+    CUtensorMap tmH;
+    if (encode_store_map_bf16(&tmH, ws + L.h, (uint64_t)a.I, (uint64_t)R) != CUDA_SUCCESS) return cudaErrorInvalidValue;
     int64_t max_tiles = (R / 128) * p.n_tiles;
     const int grid = (int)(max_tiles < num_sms ? max_tiles : num_sms);
     note_launch();
     nvf4_gemm_kernel<GateUpProblem><<<grid, kGemmThreads, gemm_smem_bytes<GateUpProblem>(), s>>>(
-        tmA, tmB, tmA /* output map unused: direct stores */, p, status, kMoeTimeoutNs, 0);
+        tmA, tmB, tmH, p, status, kMoeTimeoutNs, 0);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
 
