@@ -246,69 +246,6 @@ __device__ __forceinline__ void quantize_block_tab(const f32x2 (&xs)[8], float b
   encode_block<kDeq, kErr>(xs, t.d[b.sc], t.r[b.sc], b);
 }
 
-// Block steps of one global scale g for every E4M3 scale code, in 15 entries.
-// For code c = 8E + m the scale is s = ((8+m)/8) * 2^(E-7) (E >= 1) or
-// m * 2^-9 (E == 0, m >= 1), so d = RN(g*s) = RN(g*s') * 2^k with s' the
-// code's significand ((8+m)/8, or m) and k = E-7 (or -9): a power-of-two
-// factor changes neither the rounding of the product nor that of the
-// reciprocal, so d and RN(1/d) come from RN(g*s') and RN(1/RN(g*s')) by an
-// exponent shift, exactly, while every value stays a normal FP32 number (g in
-// [2^-100, 2^100]; gstep_valid). The block-scale divisor RN(6g) and its
-// reciprocal ride along for gstep_scale_code.
-struct GStep {
-  float d[16];  // [0,8): RN(g*(8+m)/8), m = 0..7;  [8,15): RN(g*m), m = 1..7
-  float r[16];  // RN(1/d[i])
-  float div6, inv6;
-};
-
-// Entry i (0..15) of the table of g; entry 15 is unused (written as 1).
-__device__ __forceinline__ void gstep_fill(GStep& t, float g, int i) {
-  const float sig = i < 8 ? __fdiv_rn((float)(8 + i), 8.0f) : (i < 15 ? (float)(i - 7) : 1.0f);
-  const float d = __fmul_rn(g, sig);
-  t.d[i] = d;
-  t.r[i] = __frcp_rn(d);
-  if (i == 0) {
-    t.div6 = __fmul_rn(6.0f, g);
-    t.inv6 = __frcp_rn(t.div6);
-  }
-}
-
-__device__ __forceinline__ bool gstep_valid(float g) { return g >= 0x1p-100f && g <= 0x1p100f; }
-
-// d = RN(g*s) and r = RN(1/d) of scale code c (1..126) from the table.
-__device__ __forceinline__ void gstep_lookup(const GStep& t, uint32_t c, float& d, float& r) {
-  const uint32_t E = c >> 3, m = c & 7u;
-  const uint32_t idx = E ? m : 7u + m;
-  const int32_t k = E ? (int32_t)E - 7 : -9;
-  d = __uint_as_float(__float_as_uint(t.d[idx]) + ((uint32_t)k << 23));
-  r = __uint_as_float(__float_as_uint(t.r[idx]) - ((uint32_t)k << 23));
-}
-
-// Block-scale code for target 6: E4M3(RN(bmax / RN(6g))) floored at 1.
-// bmax * RN(1/RN(6g)) lies within a few ulps of the exact quotient RN(bmax /
-// RN(6g)); the E4M3 rounding of the two differs only when they straddle a
-// rounding midpoint of E4M3 (FP32 significand bits 19..0 equal to 0x80000)
-// or lie in the E4M3 subnormal range (below 2^-6), and there the quotient is
-// computed exactly.
-__device__ __forceinline__ uint32_t gstep_scale_code(const GStep& t, float bmax) {
-  const float tq = __fmul_rn(bmax, t.inv6);
-  const uint32_t lo = __float_as_uint(tq) & 0xFFFFFu;
-  uint32_t c;
-  if (tq < 0.0158f || lo - 0x7FFF0u < 0x20u)
-    c = e4m3_code(__fdiv_rn(bmax, t.div6));
-  else
-    c = e4m3_code(tq);
-  return c > 1u ? c : 1u;
-}
-
-// quantize_block (target 6) with the block step from a GStep table.
-__device__ __forceinline__ void quantize_block_gstep(const f32x2 (&xs)[8], float bmax, const GStep& t, Block& b) {
-  b.sc = gstep_scale_code(t, bmax);
-  float d, r;
-  gstep_lookup(t, b.sc, d, r);
-  encode_block<false, false>(xs, d, r, b);
-}
-
 template <bool kDeq, bool kErr>
 __device__ __forceinline__ void quantize_block(const Raw16& raw, float bmax, float g, float mt, Block& b) {
   f32x2 xs[8];

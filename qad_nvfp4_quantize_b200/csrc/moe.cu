@@ -44,7 +44,6 @@ constexpr int kFrontCtasMax = 256;      // front-end CTAs (each owns a contiguou
 constexpr int kFrontThreads = 512;
 constexpr int kFrontWarps = kFrontThreads / 32;
 constexpr int kFrontBatchPairs = 4096;  // (token, slot) pairs placed and quantized per batch
-constexpr int kFrontTabExperts = 512;   // per-expert block-step tables in shared memory up to this E
 
 // Workspace layout (all regions 256-byte aligned).
 struct MoeLayout {
@@ -245,7 +244,6 @@ __global__ void __launch_bounds__(kFrontThreads, 1) moe_front_place_quantize_ker
   int32_t* wcnt = base + 2 * Ep;                            // [kFrontWarps][Ep]
   int32_t* pos_s = wcnt + kFrontWarps * Ep;                 // [kFrontBatchPairs]
   int32_t* exp_s = pos_s + kFrontBatchPairs;                // [kFrontBatchPairs]
-  GStep* gst = reinterpret_cast<GStep*>(exp_s + kFrontBatchPairs);  // [E] when E <= kFrontTabExperts
   __shared__ int32_t wsum[kFrontWarps];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
@@ -329,9 +327,6 @@ __global__ void __launch_bounds__(kFrontThreads, 1) moe_front_place_quantize_ker
       }
     }
     __syncthreads();
-    if (E <= kFrontTabExperts)
-      for (int i = threadIdx.x; i < E * 16; i += blockDim.x) gstep_fill(gst[i >> 4], g_s[i >> 4], i & 15);
-    __syncthreads();
   }
 
   // ---- placement and quantization, batch by batch
@@ -406,10 +401,7 @@ __global__ void __launch_bounds__(kFrontThreads, 1) moe_front_place_quantize_ker
             if (e < 0) continue;  // warp-uniform
             const Idx row = (Idx)pp[j];
             Block b;
-            if (E <= kFrontTabExperts && gstep_valid(g_s[e]))  // warp-uniform
-              quantize_block_gstep(xs, bmax, gst[e], b);
-            else
-              quantize_block<false, false>(xs, bmax, g_s[e], 6.0f, b);
+            quantize_block<false, false>(xs, bmax, g_s[e], 6.0f, b);
             if (valid) {
               a.xq_codes[(row * (Idx)a.H + (Idx)col) >> 4] = make_uint2(b.q0, b.q1);
               a.xq_scales[(((row >> 7) * (Idx)kgroups + (Idx)(col >> 6)) << 9) + ((row & 31) << 4) +
@@ -435,7 +427,6 @@ __global__ void __launch_bounds__(kFrontThreads, 1) moe_front_place_quantize_ker
 // ----------------------------------------------------------------------------
 constexpr int kRowThreads = 256;
 constexpr int kRowUnroll = 4;
-constexpr int kHTabExperts = 256;  // block-step tables in shared memory up to this E
 
 template <bool kNarrow>
 __global__ void __launch_bounds__(kRowThreads) moe_quantize_h_kernel(
@@ -443,8 +434,7 @@ __global__ void __launch_bounds__(kRowThreads) moe_quantize_h_kernel(
     const int32_t* __restrict__ tile_expert, const int32_t* __restrict__ tile_count,
     const uint32_t* __restrict__ amax_bits, int E, uint2* __restrict__ codes, uint8_t* __restrict__ scales,
     float* __restrict__ g_out, int* status, uint64_t cpr_magic) {
-  extern __shared__ float g_s[];  // [E], then (E <= kHTabExperts) the block-step tables [E]
-  GStep* gst = reinterpret_cast<GStep*>(g_s + ((E + 3) & ~3));
+  extern __shared__ float g_s[];  // [E]
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
     const float amax = __uint_as_float(amax_bits[e]);
     const float g = global_scale_from_amax(amax);
@@ -455,11 +445,6 @@ __global__ void __launch_bounds__(kRowThreads) moe_quantize_h_kernel(
     }
   }
   __syncthreads();
-  const bool tab = E <= kHTabExperts;
-  if (tab) {
-    for (int i = threadIdx.x; i < E * 16; i += blockDim.x) gstep_fill(gst[i >> 4], g_s[i >> 4], i & 15);
-    __syncthreads();
-  }
   using Idx = typename std::conditional<kNarrow, uint32_t, int64_t>::type;
   const int lane = threadIdx.x & 31;
   const int32_t rows = (*tile_count) * 128;
@@ -485,14 +470,7 @@ __global__ void __launch_bounds__(kRowThreads) moe_quantize_h_kernel(
       if (ch0 + u * nwarps >= n_chunks) break;  // warp-uniform
       Block b;
       if (pr[u] >= 0) {
-        const float gv = g_s[ex[u]];
-        if (tab && gstep_valid(gv)) {  // warp-uniform: a chunk lies in one row
-          f32x2 xs[8];
-          unpack_block(vv[u], xs);
-          quantize_block_gstep(xs, block_absmax(vv[u]), gst[ex[u]], b);
-        } else {
-          quantize_block<false, false>(vv[u], block_absmax(vv[u]), gv, 6.0f, b);
-        }
+        quantize_block<false, false>(vv[u], block_absmax(vv[u]), g_s[ex[u]], 6.0f, b);
       } else {
         b.sc = b.q0 = b.q1 = 0u;  // pad row: zero codes and scales, no arithmetic
       }
@@ -743,18 +721,14 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
     fb.xq_codes = reinterpret_cast<uint2*>(ws + L.xq_codes);
     fb.xq_scales = ws + L.xq_scales;
     fb.status = status;
-    const size_t smem = (size_t)(2 + kFrontWarps) * Ep * sizeof(int32_t) + 2 * kFrontBatchPairs * sizeof(int32_t) +
-                        (a.E <= kFrontTabExperts ? (size_t)a.E * sizeof(GStep) : 0);
+    const size_t smem = (size_t)(2 + kFrontWarps) * Ep * sizeof(int32_t) + 2 * kFrontBatchPairs * sizeof(int32_t);
     const bool narrow = narrow_chunks(R, a.H) && narrow_chunks(a.T, a.H);
     const void* kern = narrow ? (const void*)moe_front_place_quantize_kernel<uint32_t>
                               : (const void*)moe_front_place_quantize_kernel<int64_t>;
     static std::once_flag once;
     static cudaError_t attr_err = cudaSuccess;
     std::call_once(once, [] {
-      const size_t tab = (size_t)(2 + kFrontWarps) * 512 * sizeof(int32_t) + 2 * kFrontBatchPairs * sizeof(int32_t) +
-                         (size_t)kFrontTabExperts * sizeof(GStep);
-      const size_t notab = (size_t)(2 + kFrontWarps) * 1024 * sizeof(int32_t) + 2 * kFrontBatchPairs * sizeof(int32_t);
-      const int big = (int)(tab > notab ? tab : notab);
+      const int big = (int)((2 + kFrontWarps) * 1024 * sizeof(int32_t) + 2 * kFrontBatchPairs * sizeof(int32_t));
       attr_err = cudaFuncSetAttribute(moe_front_place_quantize_kernel<uint32_t>,
                                       cudaFuncAttributeMaxDynamicSharedMemorySize, big);
       if (attr_err == cudaSuccess)
@@ -780,8 +754,7 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
   }
 
   const int qgrid = num_sms * 4;
-  const size_t qsmem = (size_t)((a.E + 3) & ~3) * sizeof(float) +
-                       (a.E <= kHTabExperts ? (size_t)a.E * sizeof(GStep) : 0);
+  const size_t qsmem = (size_t)a.E * sizeof(float);
 
   // 3. gate_up grouped GEMM
   {
