@@ -26,6 +26,11 @@
  *    the device (non-finite input, a bounded wait that ran out) are recorded
  *    in a library-owned device status word; read it with
  *    nvfp4_get_device_status(), which synchronizes `stream`.
+ *  - Bounds-checking build: libnvfp4_debug.so (built with
+ *    -DNVFP4_DEBUG_BOUNDS) exports the same calls; its kernels check every
+ *    computed global index against the extent of its buffer, record
+ *    NVFP4_ERR_BOUNDS in the device status word on a violation and skip that
+ *    access (no trap). The regular library carries no checks.
  *  - Requirements: K % 64 == 0; every pointer 16-byte aligned; inputs
  *    row-major and contiguous. The device must be sm_100 (B200-class);
  *    other devices get NVFP4_ERR_UNSUPPORTED_DEVICE (the hardware gate of
@@ -63,7 +68,9 @@ typedef enum {
   NVFP4_ERR_WORKSPACE = 4,          /* workspace missing or too small */
   NVFP4_ERR_NONFINITE_INPUT = 5,    /* device: amax of an input is Inf/NaN */
   NVFP4_ERR_TIMEOUT = 6,            /* device: a bounded wait ran out */
-  NVFP4_ERR_TOO_LARGE = 7           /* input larger than nvfp4_quantize_noalloc's static scratch */
+  NVFP4_ERR_TOO_LARGE = 7,          /* input larger than nvfp4_quantize_noalloc's static scratch */
+  NVFP4_ERR_BOUNDS = 8              /* device, bounds-checking build only: a computed global index
+                                       fell outside its buffer; that access was skipped */
 } nvfp4_status;
 
 typedef enum {

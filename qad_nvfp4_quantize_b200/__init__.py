@@ -30,11 +30,16 @@ _MODES = {"max": MODE_MAX, "four_over_six": MODE_FOUR_OVER_SIX, "mse": MODE_MSE,
           MODE_FOUR_OVER_SIX: MODE_FOUR_OVER_SIX, MODE_MSE: MODE_MSE}
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-library_path = os.path.join(_HERE, "libnvfp4.so")
+# NVFP4_LIBRARY=debug selects the bounds-checking build (libnvfp4_debug.so);
+# any other value is taken as the path of the library to load.
+_choice = os.environ.get("NVFP4_LIBRARY", "")
+library_path = (os.path.join(_HERE, "libnvfp4_debug.so") if _choice == "debug"
+                else (_choice or os.path.join(_HERE, "libnvfp4.so")))
 
 _STATUS = {0: "ok", 1: "invalid argument", 2: "unsupported device", 3: "CUDA error",
            4: "workspace missing or too small", 5: "non-finite input", 6: "device wait timed out",
-           7: "input too large for the no-alloc entry point (M*K > 2^30)"}
+           7: "input too large for the no-alloc entry point (M*K > 2^30)",
+           8: "index outside its buffer (bounds-checking build)"}
 
 
 class NVFP4Error(RuntimeError):

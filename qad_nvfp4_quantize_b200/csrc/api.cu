@@ -100,6 +100,7 @@ const char* nvfp4_status_string(nvfp4_status s) {
     case NVFP4_ERR_NONFINITE_INPUT: return "non-finite input";
     case NVFP4_ERR_TIMEOUT: return "device wait timed out";
     case NVFP4_ERR_TOO_LARGE: return "input larger than the no-alloc entry point's static scratch (M*K > 2^30)";
+    case NVFP4_ERR_BOUNDS: return "a computed index fell outside its buffer (bounds-checking build)";
   }
   return "unknown status";
 }
@@ -213,7 +214,7 @@ nvfp4_status nvfp4_topk_kl(const void* teacher, const void* student, int64_t row
   DeviceInfo* d;
   nvfp4_status st = current_device(&d);
   if (st != NVFP4_OK) return st;
-  return launched(nvfp4::launch_topk_kl(teacher, student, rows, V, k, loss, idx, grad, d->num_sms,
+  return launched(nvfp4::launch_topk_kl(teacher, student, rows, V, k, loss, idx, grad, d->status, d->num_sms,
                                         reinterpret_cast<cudaStream_t>(stream)));
 }
 
@@ -225,7 +226,7 @@ nvfp4_status nvfp4_dequantize(const uint8_t* codes, const uint8_t* scales, const
   nvfp4_status st = current_device(&d);
   if (st != NVFP4_OK) return st;
   if (M == 0) return NVFP4_OK;
-  return launched(nvfp4::launch_dequantize(codes, scales, g, M, K, y, d->num_sms, reinterpret_cast<cudaStream_t>(stream)));
+  return launched(nvfp4::launch_dequantize(codes, scales, g, M, K, y, d->status, d->num_sms, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 nvfp4_status nvfp4_fake_quant_backward(const void* x, const void* grad_y, int64_t M, int64_t K, nvfp4_mode mode,

@@ -29,6 +29,20 @@ NVFP4_DEVINL void record_status(int* status, int code) {
   if (status) atomicCAS(status, 0, code);
 }
 
+// Index check of the bounds-checking build (-DNVFP4_DEBUG_BOUNDS): true when
+// i < n; otherwise records NVFP4_ERR_BOUNDS and returns false so that the
+// caller skips the access. In the regular build it is the constant true.
+NVFP4_DEVINL bool bounds_ok(uint64_t i, uint64_t n, int* status) {
+  if (i < n) return true;
+  record_status(status, NVFP4_ERR_BOUNDS);
+  return false;
+}
+#ifdef NVFP4_DEBUG_BOUNDS
+#define NVFP4_IN_BOUNDS(i, n, status) ::nvfp4::bounds_ok((uint64_t)(i), (uint64_t)(n), (status))
+#else
+#define NVFP4_IN_BOUNDS(i, n, status) true
+#endif
+
 // ----------------------------------------------------------------------------
 // Format conversions.
 // Round-to-nearest-even, saturating conversions of the NVFP4 format: E2M1
@@ -229,6 +243,12 @@ NVFP4_DEVINL void fence_proxy_async_smem() { asm volatile("fence.proxy.async.sha
 NVFP4_DEVINL void st_shared_v4(uint32_t addr, uint4 v) {
   asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(v.x), "r"(v.y), "r"(v.z), "r"(v.w)
                : "memory");
+}
+
+// Barrier `id` (1..15; 0 is __syncthreads) over `nthreads` threads (a
+// multiple of 32) of the CTA.
+NVFP4_DEVINL void named_barrier_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 NVFP4_DEVINL void prefetch_tensormap(const CUtensorMap* map) {

@@ -20,6 +20,7 @@ struct DenseProblem {
   const float* ga;
   const float* gb;
   __nv_bfloat16* C;
+  const uint8_t *sfa_lo, *sfa_hi, *sfb_lo, *sfb_hi;  // scale buffers (bounds-checking build)
 
   __device__ __forceinline__ int num_tiles() const { return m_tiles * n_tiles; }
 
@@ -166,6 +167,10 @@ cudaError_t launch_gemm(const uint8_t* Aq, const uint8_t* As, const float* ga, c
   p.ga = ga;
   p.gb = gb;
   p.C = static_cast<__nv_bfloat16*>(C);
+  p.sfa_lo = As;
+  p.sfa_hi = As + (size_t)p.m_tiles * p.kgroups * kSFAtom;
+  p.sfb_lo = Bs;
+  p.sfb_hi = Bs + (size_t)((N + 127) / 128) * p.kgroups * kSFAtom;
   cudaError_t e = prepare_kernel<DenseProblem>();
   if (e != cudaSuccess) return e;
   CUtensorMap tmC;

@@ -177,11 +177,29 @@ __global__ void __launch_bounds__(kGemmThreads, 1)
         tma_load_2d_elect(sA, &tmA, kt * (kBK / 2), job.a_row, &full[stage]);
         tma_load_2d_elect(sB, &tmB, kt * (kBK / 2), job.b_row0, &full[stage]);
         tma_load_2d_elect(sB + kBHalfBytes, &tmB, kt * (kBK / 2), job.b_row1, &full[stage]);
-        bulk_load_elect(smem + Lay::kSFA + stage * kSFABytes, job.sfa + (size_t)kt * kSFABytes, sf_bytes,
-                        &full[stage]);
+        const uint8_t* pa = job.sfa + (size_t)kt * kSFABytes;
+        const uint8_t* pb0 = job.sfb0 + (size_t)kt * kSFABytes;
+        const uint8_t* pb1 = job.sfb1 ? job.sfb1 + (size_t)kt * kSFABytes : nullptr;
+#ifdef NVFP4_DEBUG_BOUNDS
+        // scale tiles outside their buffers: reported, and read from the
+        // buffer's start instead so that the stage still completes
+        if (pa < prob.sfa_lo || pa + sf_bytes > prob.sfa_hi) {
+          if (lane == 0) record_status(status, NVFP4_ERR_BOUNDS);
+          pa = prob.sfa_lo;
+        }
+        if (pb0 < prob.sfb_lo || pb0 + sf_bytes > prob.sfb_hi) {
+          if (lane == 0) record_status(status, NVFP4_ERR_BOUNDS);
+          pb0 = prob.sfb_lo;
+        }
+        if (pb1 && (pb1 < prob.sfb_lo || pb1 + sf_bytes > prob.sfb_hi)) {
+          if (lane == 0) record_status(status, NVFP4_ERR_BOUNDS);
+          pb1 = prob.sfb_lo;
+        }
+#endif
+        bulk_load_elect(smem + Lay::kSFA + stage * kSFABytes, pa, sf_bytes, &full[stage]);
         uint8_t* sSFB = smem + Lay::kSFB + stage * kSFBBytes;
-        bulk_load_elect(sSFB, job.sfb0 + (size_t)kt * kSFABytes, sf_bytes, &full[stage]);
-        if (job.sfb1) bulk_load_elect(sSFB + kSFABytes, job.sfb1 + (size_t)kt * kSFABytes, sf_bytes, &full[stage]);
+        bulk_load_elect(sSFB, pb0, sf_bytes, &full[stage]);
+        if (pb1) bulk_load_elect(sSFB + kSFABytes, pb1, sf_bytes, &full[stage]);
         if (++stage == kStages) {
           stage = 0;
           phase ^= 1;

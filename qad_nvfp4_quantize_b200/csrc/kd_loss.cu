@@ -214,7 +214,7 @@ __device__ __forceinline__ uint32_t warp_prefix(const KdShared& sh, int w) {
 // Fast path of one row (see the file comment). Returns false, with nothing
 // written, when the row must take the full path. All threads call it.
 __device__ bool kd_fast_row(KdShared& sh, const uint4* trow, const uint16_t* srow16, int64_t nvec, int k,
-                            KdAcc& acc, int32_t* idx_row) {
+                            KdAcc& acc, int32_t* idx_row, int* status) {
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
   const unsigned lt_mask = (1u << lane) - 1u;
 
@@ -411,7 +411,8 @@ __device__ bool kd_fast_row(KdShared& sh, const uint4* trow, const uint16_t* sro
       const bool sel = i < mine && (key > T || (eq && eq_rank + __popc(eqm & lt_mask) < need_eq));
       eq_rank += __popc(eqm);
       const unsigned selm = __ballot_sync(0xFFFFFFFFu, sel);
-      if (sel) idx_row[pos + __popc(selm & lt_mask)] = sh.cidx[warp][i];
+      if (sel && NVFP4_IN_BOUNDS(pos + __popc(selm & lt_mask), k, status))
+        idx_row[pos + __popc(selm & lt_mask)] = sh.cidx[warp][i];
       pos += __popc(selm);
     }
   }
@@ -421,7 +422,9 @@ __device__ bool kd_fast_row(KdShared& sh, const uint4* trow, const uint16_t* sro
 
 // Gradient p_s - p_t of a row the fast path served, written at the same
 // output positions as its idx, from the candidates still in shared memory.
-__device__ void kd_fast_grad(const KdShared& sh, float lse_t, float lse_s, float* grad_row) {
+__device__ void kd_fast_grad(const KdShared& sh, float lse_t, float lse_s, float* grad_row, int k, int* status) {
+  (void)k;
+  (void)status;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const unsigned lt_mask = (1u << lane) - 1u;
   const uint32_t mine = sh.wcount[warp], T = sh.fT, need_eq = sh.fneed;
@@ -434,7 +437,7 @@ __device__ void kd_fast_grad(const KdShared& sh, float lse_t, float lse_s, float
     const bool sel = i < mine && (key > T || (eq && eq_rank + __popc(eqm & lt_mask) < need_eq));
     eq_rank += __popc(eqm);
     const unsigned selm = __ballot_sync(0xFFFFFFFFu, sel);
-    if (sel) {
+    if (sel && NVFP4_IN_BOUNDS(pos + __popc(selm & lt_mask), k, status)) {
       const uint32_t sw = sh.cstu[warp][i];
       const float sv = __uint_as_float((sh.cidx[warp][i] & 1) ? (sw & 0xFFFF0000u) : (sw << 16));
       grad_row[pos + __popc(selm & lt_mask)] = expf(sv - lse_s) - expf(kd_value(key) - lse_t);
@@ -447,7 +450,7 @@ __global__ void __launch_bounds__(kKdThreads, 2) topk_kl_kernel(const uint4* __r
                                                                  const uint4* __restrict__ student, int64_t rows,
                                                                  int64_t V, int k, float* __restrict__ loss,
                                                                  int32_t* __restrict__ idx_out,
-                                                                 float* __restrict__ grad_out) {
+                                                                 float* __restrict__ grad_out, int* status) {
   extern __shared__ __align__(16) uint8_t kd_smem[];
   KdShared& sh = *reinterpret_cast<KdShared*>(kd_smem);
   const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
@@ -459,7 +462,7 @@ __global__ void __launch_bounds__(kKdThreads, 2) topk_kl_kernel(const uint4* __r
     KdAcc acc;
     acc.init();
     const bool fast = kd_fast_row(sh, trow, reinterpret_cast<const uint16_t*>(srow), nvec, k, acc,
-                                  idx_out ? idx_out + row * k : nullptr);
+                                  idx_out ? idx_out + row * k : nullptr, status);
     if (!fast) {
     // ---- pass 1: histogram of the key's high byte
     for (int i = t; i < kKdWarps * 256; i += kKdThreads) (&sh.whist[0][0])[i] = 0u;
@@ -563,7 +566,10 @@ __global__ void __launch_bounds__(kKdThreads, 2) topk_kl_kernel(const uint4* __r
           const float tv = (e & 1) ? bf16_hi(w[e >> 1]) : bf16_lo(w[e >> 1]);
           const float svv = (e & 1) ? bf16_hi(sw[e >> 1]) : bf16_lo(sw[e >> 1]);
           acc.add(tv, svv);
-          if (idx_out) idx_out[row * k + pos++] = (int32_t)(8 * j + e);
+          if (idx_out) {
+            if (NVFP4_IN_BOUNDS(pos, k, status)) idx_out[row * k + pos] = (int32_t)(8 * j + e);
+            ++pos;
+          }
         }
       }
       __syncthreads();  // everyone has read eq_base / sel_base
@@ -616,13 +622,14 @@ __global__ void __launch_bounds__(kKdThreads, 2) topk_kl_kernel(const uint4* __r
 
     // ---- optional pass 4: gradient p_s - p_t at the selected entries
     if (grad_out && idx_out && fast) {
-      kd_fast_grad(sh, sh.red[0][0], sh.red[0][1], grad_out + row * k);
+      kd_fast_grad(sh, sh.red[0][0], sh.red[0][1], grad_out + row * k, k, status);
     } else if (grad_out && idx_out) {
       const float lse_t = sh.red[0][0], lse_s = sh.red[0][1];
       const uint16_t* t16 = reinterpret_cast<const uint16_t*>(trow);
       const uint16_t* s16 = reinterpret_cast<const uint16_t*>(srow);
       for (int i = t; i < k; i += kKdThreads) {
-        const int32_t v = idx_out[row * k + i];
+        int32_t v = idx_out[row * k + i];
+        if (!NVFP4_IN_BOUNDS(v, V, status)) v = 0;
         const float tv = __uint_as_float((uint32_t)t16[v] << 16), svv = __uint_as_float((uint32_t)s16[v] << 16);
         grad_out[row * k + i] = expf(svv - lse_s) - expf(tv - lse_t);
       }
@@ -632,7 +639,7 @@ __global__ void __launch_bounds__(kKdThreads, 2) topk_kl_kernel(const uint4* __r
 }
 
 cudaError_t launch_topk_kl(const void* teacher, const void* student, int64_t rows, int64_t V, int k, float* loss,
-                           int32_t* idx, float* grad, int num_sms, cudaStream_t s) {
+                           int32_t* idx, float* grad, int* status, int num_sms, cudaStream_t s) {
   if (rows == 0) return cudaSuccess;
   static const cudaError_t attr = cudaFuncSetAttribute(topk_kl_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                                        (int)sizeof(KdShared));
@@ -641,7 +648,7 @@ cudaError_t launch_topk_kl(const void* teacher, const void* student, int64_t row
   const int grid = (int)(rows < slots ? rows : slots);
   note_launch();
   topk_kl_kernel<<<grid, kKdThreads, sizeof(KdShared), s>>>(static_cast<const uint4*>(teacher), static_cast<const uint4*>(student),
-                                             rows, V, k, loss, idx, grad);
+                                             rows, V, k, loss, idx, grad, status);
   return cudaGetLastError();
 }
 

@@ -51,10 +51,10 @@ cudaError_t launch_fake_quant_fused(const void* x, int64_t M, int64_t K, bool fo
                                     int* status, int num_sms, cudaStream_t s);
 // Top-k logit KL loss per row (idx / grad nullable; grad needs idx).
 cudaError_t launch_topk_kl(const void* teacher, const void* student, int64_t rows, int64_t V, int k, float* loss,
-                           int32_t* idx, float* grad, int num_sms, cudaStream_t s);
+                           int32_t* idx, float* grad, int* status, int num_sms, cudaStream_t s);
 // y = BF16(g * s * q) from codes and tiled scales.
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t M, int64_t K,
-                              void* y, int num_sms, cudaStream_t s);
+                              void* y, int* status, int num_sms, cudaStream_t s);
 // QAD backward (clipped straight-through estimator); scales as the forward.
 cudaError_t launch_fake_quant_bwd(const void* x, const void* gy, int64_t M, int64_t K, bool fos,
                                   const uint32_t* partial, int n_partial, const float* g_static,

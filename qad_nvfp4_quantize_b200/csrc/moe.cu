@@ -128,8 +128,11 @@ __global__ void __launch_bounds__(kCountThreads) moe_front_count_kernel(
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
         const bool in = i0 + 32 * u < hv;
-        va[u] = in ? ld_stream(row_a + i0 + 32 * u) : make_uint4(0, 0, 0, 0);
-        vb[u] = in && tb < t1 ? ld_stream(row_b + i0 + 32 * u) : make_uint4(0, 0, 0, 0);
+        va[u] = in && NVFP4_IN_BOUNDS(ta * hv + i0 + 32 * u, T * hv, status) ? ld_stream(row_a + i0 + 32 * u)
+                                                                                : make_uint4(0, 0, 0, 0);
+        vb[u] = in && tb < t1 && NVFP4_IN_BOUNDS(tb * hv + i0 + 32 * u, T * hv, status)
+                    ? ld_stream(row_b + i0 + 32 * u)
+                    : make_uint4(0, 0, 0, 0);
       }
 #pragma unroll
       for (int u = 0; u < 8; ++u) {
@@ -161,12 +164,14 @@ __global__ void __launch_bounds__(kCountThreads) moe_front_count_kernel(
         }
       }
       float4* orow = out + t * (H / 4);
-      for (int64_t i = lane; i < H / 4; i += 32) orow[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (NVFP4_IN_BOUNDS(t, T, status))
+        for (int64_t i = lane; i < H / 4; i += 32) orow[i] = make_float4(0.f, 0.f, 0.f, 0.f);
     }
   }
   if (bad) record_status(status, NVFP4_ERR_INVALID_ARG);
   __syncthreads();
   for (int e = threadIdx.x; e < Ep; e += blockDim.x) {
+    if (!NVFP4_IN_BOUNDS((int64_t)blockIdx.x * Ep + e, (int64_t)kFrontCtasMax * Ep, status)) continue;
     cta_count[(int64_t)blockIdx.x * Ep + e] = (int32_t)hist[e];
     cta_amax[(int64_t)blockIdx.x * Ep + e] = amax[e];
   }
@@ -222,6 +227,7 @@ __device__ __forceinline__ int32_t block_excl_scan2(int32_t v0, int32_t v1, int3
 struct FrontB {
   const uint4* x;
   int64_t T, H;
+  int64_t R;               // padded row capacity of the gathered activations
   const int32_t* topk_ids;
   int topk, E, Ep;
   const int32_t* cta_count;
@@ -322,8 +328,10 @@ __global__ void __launch_bounds__(kFrontThreads, 1) moe_front_place_quantize_ker
         }
       }
       if (e % G == c) {
-        for (int32_t t = off / 128; t < (off + padded) / 128; ++t) a.tile_expert[t] = e;
-        for (int32_t r = off + tv[k]; r < off + padded; ++r) a.row_pair[r] = -1;  // pad rows
+        for (int32_t t = off / 128; t < (off + padded) / 128; ++t)
+          if (NVFP4_IN_BOUNDS(t, a.R / 128, a.status)) a.tile_expert[t] = e;
+        for (int32_t r = off + tv[k]; r < off + padded; ++r)
+          if (NVFP4_IN_BOUNDS(r, a.R, a.status)) a.row_pair[r] = -1;  // pad rows
       }
     }
     __syncthreads();
@@ -366,7 +374,7 @@ __global__ void __launch_bounds__(kFrontThreads, 1) moe_front_place_quantize_ker
       int32_t row = -1;
       if (e >= 0) {
         row = wcnt[warp * Ep + e] + rank;
-        a.row_pair[row] = (int32_t)p;
+        if (NVFP4_IN_BOUNDS(row, a.R, a.status)) a.row_pair[row] = (int32_t)p;
       }
       if (p < whi) {
         pos_s[p - pb0] = row;
@@ -386,7 +394,9 @@ __global__ void __launch_bounds__(kFrontThreads, 1) moe_front_place_quantize_ker
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
           const int32_t col = (ch0 + u) * 512 + lane * 16;
-          load_raw16(a.x, (Idx)t * (Idx)hv + (Idx)(col >> 3), ch0 + u < cpr && col < a.H, raw[u]);
+          load_raw16(a.x, (Idx)t * (Idx)hv + (Idx)(col >> 3),
+                     ch0 + u < cpr && col < a.H && NVFP4_IN_BOUNDS(t * hv + (col >> 3) + 1, a.T * hv, a.status),
+                     raw[u]);
         }
 #pragma unroll
         for (int u = 0; u < 4; ++u) {
@@ -403,9 +413,11 @@ __global__ void __launch_bounds__(kFrontThreads, 1) moe_front_place_quantize_ker
             Block b;
             quantize_block<false, false>(xs, bmax, g_s[e], 6.0f, b);
             if (valid) {
-              a.xq_codes[(row * (Idx)a.H + (Idx)col) >> 4] = make_uint2(b.q0, b.q1);
-              a.xq_scales[(((row >> 7) * (Idx)kgroups + (Idx)(col >> 6)) << 9) + ((row & 31) << 4) +
-                          (((row >> 5) & 3) << 2) + (Idx)((col >> 4) & 3)] = (uint8_t)b.sc;
+              const Idx cw = (row * (Idx)a.H + (Idx)col) >> 4;
+              const Idx so = (((row >> 7) * (Idx)kgroups + (Idx)(col >> 6)) << 9) + ((row & 31) << 4) +
+                             (((row >> 5) & 3) << 2) + (Idx)((col >> 4) & 3);
+              if (NVFP4_IN_BOUNDS(cw, a.R * a.H / 16, a.status)) a.xq_codes[cw] = make_uint2(b.q0, b.q1);
+              if (NVFP4_IN_BOUNDS(so, a.R / 128 * kgroups * 512, a.status)) a.xq_scales[so] = (uint8_t)b.sc;
             }
           }
         }
@@ -430,7 +442,7 @@ constexpr int kRowUnroll = 4;
 
 template <bool kNarrow>
 __global__ void __launch_bounds__(kRowThreads) moe_quantize_h_kernel(
-    const uint4* __restrict__ src, int64_t K, const int32_t* __restrict__ row_pair,
+    const uint4* __restrict__ src, int64_t K, int64_t R, const int32_t* __restrict__ row_pair,
     const int32_t* __restrict__ tile_expert, const int32_t* __restrict__ tile_count,
     const uint32_t* __restrict__ amax_bits, int E, uint2* __restrict__ codes, uint8_t* __restrict__ scales,
     float* __restrict__ g_out, int* status, uint64_t cpr_magic) {
@@ -459,12 +471,15 @@ __global__ void __launch_bounds__(kRowThreads) moe_quantize_h_kernel(
     for (int u = 0; u < kRowUnroll; ++u) {
       const int32_t ch = ch0 + u * nwarps;
       cc[u] = chunk_at_t<Idx>(ch < n_chunks ? ch : 0, cpr, cpr_magic, K, lane);
-      pr[u] = ch < n_chunks ? row_pair[cc[u].row] : -1;
-      ex[u] = ch < n_chunks ? tile_expert[cc[u].row >> 7] : 0;
+      const bool in = ch < n_chunks && NVFP4_IN_BOUNDS(cc[u].row, R, status);
+      pr[u] = in ? row_pair[cc[u].row] : -1;
+      ex[u] = in ? tile_expert[cc[u].row >> 7] : 0;
     }
     Raw16 vv[kRowUnroll];
 #pragma unroll
-    for (int u = 0; u < kRowUnroll; ++u) load_raw16(src, cc[u].vec, pr[u] >= 0 && cc[u].valid, vv[u]);
+    for (int u = 0; u < kRowUnroll; ++u)
+      load_raw16(src, cc[u].vec, pr[u] >= 0 && cc[u].valid && NVFP4_IN_BOUNDS(cc[u].vec + 1, R * K / 8, status),
+                 vv[u]);
 #pragma unroll
     for (int u = 0; u < kRowUnroll; ++u) {
       if (ch0 + u * nwarps >= n_chunks) break;  // warp-uniform
@@ -475,8 +490,9 @@ __global__ void __launch_bounds__(kRowThreads) moe_quantize_h_kernel(
         b.sc = b.q0 = b.q1 = 0u;  // pad row: zero codes and scales, no arithmetic
       }
       if (cc[u].valid) {
-        codes[cc[u].vec >> 1] = make_uint2(b.q0, b.q1);
-        scales[block_scale_offset(cc[u], K)] = (uint8_t)b.sc;
+        const int64_t so = block_scale_offset(cc[u], K);
+        if (NVFP4_IN_BOUNDS(cc[u].vec >> 1, R * K / 16, status)) codes[cc[u].vec >> 1] = make_uint2(b.q0, b.q1);
+        if (NVFP4_IN_BOUNDS(so, R / 128 * (K / 64) * 512, status)) scales[so] = (uint8_t)b.sc;
       }
     }
   }
@@ -504,6 +520,9 @@ struct GateUpProblem {
   __nv_bfloat16* h;        // [R][I]
   uint32_t* amax_h;
   const int32_t* row_pair; // -1 marks a pad row
+  int64_t R;               // padded row capacity
+  int* st;
+  const uint8_t *sfa_lo, *sfa_hi, *sfb_lo, *sfb_hi;  // scale buffers (bounds-checking build)
 
   __device__ __forceinline__ int num_tiles() const { return (*tile_count) * n_tiles; }
 
@@ -540,7 +559,8 @@ struct GateUpProblem {
     const float alpha = __fmul_rn(ga[job.expert], gb[job.expert]);
     // pad rows: their gathered activations were never written, so their
     // accumulators are meaningless; h gets zeros and stays out of the amax
-    const uint32_t live = row_pair[row0 + lane] >= 0 ? 0xFFFFFFFFu : 0u;
+    const uint32_t live =
+        NVFP4_IN_BOUNDS(row0 + lane, R, st) && row_pair[row0 + lane] >= 0 ? 0xFFFFFFFFu : 0u;
     const uint32_t sbase = smem_u32(stg);
     uint32_t mx = 0;
 #pragma unroll
@@ -587,17 +607,23 @@ struct GateUpProblem {
 // ----------------------------------------------------------------------------
 // 5. down grouped GEMM problem: out[token] += w * (g_h * g_w2) * acc.
 // The rows of a tile belong to different tokens, so the sum over a token's
-// experts is a reduction into out. Each epilogue lane stages 32 FP32 values
-// of its row (128 bytes, rows 144 bytes apart so the 32 lanes' writes fall on
-// distinct banks) and adds them into out with one bulk reduction
-// (cp.reduce.async.bulk .add.f32: element-wise atomic adds done by the memory
-// system), 1024 per tile instead of 8192 vector atomics.
+// experts is a reduction into out, done by bulk reductions
+// (cp.reduce.async.bulk .add.f32: element-wise adds performed by the memory
+// system). The two epilogue warps of a tensor-memory lane quarter (same 32
+// rows, column halves 0-127 and 128-255) stage whole 256-column row segments
+// (1 KB of FP32) in a shared region of 16 rows, 16 rows at a time, and the
+// first warp's lanes 0..15 add each staged row into out with one 1 KB bulk
+// reduction: 128 reductions of 1 KB per tile. (Each bulk operation has a
+// fixed cost in the copy engine; with 128-byte pieces, 1024 per tile, that
+// cost bound the kernel: halving its grid nearly doubled its time.)
 // ----------------------------------------------------------------------------
-constexpr uint32_t kDownRowStride = 144;  // staged row pitch (128 bytes of data)
+constexpr uint32_t kDownRowStride = 1040;       // staged row pitch: 1 KB of data + 16 B (conflict-free v4 stores)
+constexpr uint32_t kDownGroupRows = 16;         // rows staged per bulk-reduction round
+constexpr uint32_t kDownRegion = kDownGroupRows * kDownRowStride;  // per lane quarter
 
 struct DownProblem {
-  static constexpr int kPipeStages = 3;    // K = I is short: 3 stages cover 1.5 tiles
-  static constexpr uint32_t kEpiWarpBytes = 32 * kDownRowStride;
+  static constexpr int kPipeStages = 2;    // K = I = 512 is two stages; the epilogue regions take the rest
+  static constexpr uint32_t kEpiWarpBytes = kDownRegion / 2;  // a lane quarter's region spans two warp slots
   int K;             // I
   int H;
   int n_tiles;       // ceil(H / 256)
@@ -613,6 +639,9 @@ struct DownProblem {
   const float* ga;         // hq_g [E]
   const float* gb;         // w2_g [E]
   float* out;
+  int64_t R, P;            // padded row capacity, (token, slot) pairs
+  int* st;
+  const uint8_t *sfa_lo, *sfa_hi, *sfb_lo, *sfb_hi;  // scale buffers (bounds-checking build)
 
   __device__ __forceinline__ int num_tiles() const { return (*tile_count) * n_tiles; }
 
@@ -636,31 +665,46 @@ struct DownProblem {
 
   __device__ static constexpr uint32_t tmem_col(int h, int j) { return (uint32_t)(h * 128 + 32 * j); }
 
+  // Epilogue warps 2..9: q = warp & 3 is the lane quarter, hh the column
+  // half; warp slot (warp - 2) = hh*4 + ((q - 2) & 3). The quarter's region
+  // is the two consecutive slots starting at slot 2*((q - 2) & 3), and named
+  // barrier 1 + ((q - 2) & 3) pairs its two warps (64 threads).
   __device__ __forceinline__ void store(const TileJob& job, int q, int hh, int lane,
                                         const uint32_t (&acc)[4][32], uint8_t* stg, const CUtensorMap*) const {
+    const int qi = (q - 2) & 3;
+    uint8_t* epi_base = stg - (uint32_t)(hh * 4 + qi) * kEpiWarpBytes;
+    const uint32_t region = smem_u32(epi_base + (uint32_t)qi * kDownRegion);
     const int row = job.m0 + q * 32 + lane;
-    const int32_t pair = row_pair[row];
+    int32_t pair = NVFP4_IN_BOUNDS(row, R, st) ? row_pair[row] : -1;
+    if (pair >= 0 && !NVFP4_IN_BOUNDS(pair, P, st)) pair = -1;
     const float alpha = __fmul_rn(ga[job.expert], gb[job.expert]);
     const float w = pair >= 0 ? topk_w[pair] : 0.0f;
-    float* orow = out + (size_t)(pair >= 0 ? pair / topk : 0) * H;
-    const uint32_t srow = smem_u32(stg) + lane * kDownRowStride;
+    const int bar_id = 1 + qi;
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int n = job.n0 + hh * 128 + 32 * j;
-      if (n >= H) break;
-      bulk_wait_read_all();  // this lane's previous row segment has left shared memory
+    for (int g = 0; g < 2; ++g) {
+      // the region is free once the previous round's reductions have read it
+      if (hh == 0 && lane < (int)kDownGroupRows) bulk_wait_read_all();
+      named_barrier_sync(bar_id, 64);
+      if ((lane >> 4) == g) {
+        const uint32_t srow = region + (uint32_t)(lane & 15) * kDownRowStride + (uint32_t)hh * 512u;
 #pragma unroll
-      for (int c = 0; c < 32; c += 4) {
-        uint4 v;
-        v.x = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(acc[j][c + 0]), alpha), w));
-        v.y = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(acc[j][c + 1]), alpha), w));
-        v.z = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(acc[j][c + 2]), alpha), w));
-        v.w = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(acc[j][c + 3]), alpha), w));
-        st_shared_v4(srow + c * 4, v);
+        for (int j = 0; j < 4; ++j)
+#pragma unroll
+          for (int c = 0; c < 32; c += 4) {
+            uint4 v;
+            v.x = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(acc[j][c + 0]), alpha), w));
+            v.y = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(acc[j][c + 1]), alpha), w));
+            v.z = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(acc[j][c + 2]), alpha), w));
+            v.w = __float_as_uint(__fmul_rn(__fmul_rn(__uint_as_float(acc[j][c + 3]), alpha), w));
+            st_shared_v4(srow + (uint32_t)(32 * j + c) * 4u, v);
+          }
+        fence_proxy_async_smem();
       }
-      fence_proxy_async_smem();
-      if (pair >= 0) {
-        bulk_reduce_add_f32(orow + n, srow, 128);
+      named_barrier_sync(bar_id, 64);
+      // lanes 0..15 of the first warp add staged rows 16g + lane into out
+      const int32_t p = __shfl_sync(0xFFFFFFFFu, pair, (16 * g + lane) & 31);
+      if (hh == 0 && lane < (int)kDownGroupRows && p >= 0) {
+        bulk_reduce_add_f32(out + (size_t)(p / topk) * H + job.n0, region + (uint32_t)lane * kDownRowStride, 1024);
         bulk_commit_group();
       }
     }
@@ -705,6 +749,7 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
     fb.x = static_cast<const uint4*>(a.x);
     fb.T = a.T;
     fb.H = a.H;
+    fb.R = R;
     fb.topk_ids = a.topk_ids;
     fb.topk = a.topk;
     fb.E = a.E;
@@ -777,6 +822,12 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
     p.h = reinterpret_cast<__nv_bfloat16*>(ws + L.h);
     p.amax_h = U32(L.amax_h);
     p.row_pair = I32(L.row_pair);
+    p.R = R;
+    p.st = status;
+    p.sfa_lo = ws + L.xq_scales;
+    p.sfa_hi = p.sfa_lo + scale_bytes_(R, a.H);
+    p.sfb_lo = a.w13_s;
+    p.sfb_hi = a.w13_s + (size_t)a.E * p.sf_expert_bytes;
     if ((e = prepare_moe_kernel<GateUpProblem>()) != cudaSuccess) return e;
     CUtensorMap tmH;
     if (encode_store_map_bf16(&tmH, ws + L.h, (uint64_t)a.I, (uint64_t)R) != CUDA_SUCCESS) return cudaErrorInvalidValue;
@@ -792,12 +843,12 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
   note_launch();
   if (narrow_chunks(R, a.I))
     moe_quantize_h_kernel<true><<<qgrid, kRowThreads, qsmem, s>>>(
-        reinterpret_cast<const uint4*>(ws + L.h), a.I, I32(L.row_pair), I32(L.tile_expert), I32(L.tile_count),
+        reinterpret_cast<const uint4*>(ws + L.h), a.I, R, I32(L.row_pair), I32(L.tile_expert), I32(L.tile_count),
         U32(L.amax_h), a.E, reinterpret_cast<uint2*>(ws + L.hq_codes), ws + L.hq_scales, F32(L.hq_g), status,
         chunk_magic_narrow(a.I));
   else
     moe_quantize_h_kernel<false><<<qgrid, kRowThreads, qsmem, s>>>(
-        reinterpret_cast<const uint4*>(ws + L.h), a.I, I32(L.row_pair), I32(L.tile_expert), I32(L.tile_count),
+        reinterpret_cast<const uint4*>(ws + L.h), a.I, R, I32(L.row_pair), I32(L.tile_expert), I32(L.tile_count),
         U32(L.amax_h), a.E, reinterpret_cast<uint2*>(ws + L.hq_codes), ws + L.hq_scales, F32(L.hq_g), status,
         chunk_magic(a.I));
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
@@ -824,6 +875,13 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
     p.ga = F32(L.hq_g);
     p.gb = a.w2_g;
     p.out = a.out;
+    p.R = R;
+    p.P = a.T * a.topk;
+    p.st = status;
+    p.sfa_lo = ws + L.hq_scales;
+    p.sfa_hi = p.sfa_lo + scale_bytes_(R, a.I);
+    p.sfb_lo = a.w2_s;
+    p.sfb_hi = a.w2_s + (size_t)a.E * p.sf_expert_bytes;
     if ((e = prepare_moe_kernel<DownProblem>()) != cudaSuccess) return e;
     int64_t max_tiles = (R / 128) * p.n_tiles;
     const int grid = (int)(max_tiles < num_sms ? max_tiles : num_sms);

@@ -109,14 +109,22 @@ __device__ __forceinline__ float resolve_global_scale(const uint32_t* partial, i
   return s_g;
 }
 
+// Buffer extents of an [M x K] tensor for the bounds-checking build: 16-byte
+// vectors of BF16 values, 8-byte words of codes (16 codes), tiled scale bytes.
+__device__ __forceinline__ int64_t n_vec16(int64_t M, int64_t K) { return (M * K) >> 3; }
+__device__ __forceinline__ int64_t n_code_words(int64_t M, int64_t K) { return (M * K) >> 4; }
+__device__ __forceinline__ int64_t n_scale_bytes(int64_t M, int64_t K) { return ((M + 127) >> 7) * (K >> 6) * 512; }
+
 // Zero the scale bytes of the padding rows [M, ceil128(M)).
-__device__ __forceinline__ void zero_pad_scale_rows(uint8_t* scales, int64_t M, int64_t kgroups) {
+__device__ __forceinline__ void zero_pad_scale_rows(uint8_t* scales, int64_t M, int64_t kgroups, int* st) {
   const int64_t pad = ((M + 127) & ~int64_t(127)) - M;
   const int64_t total = pad * kgroups;
   for (int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; i < total;
        i += (int64_t)gridDim.x * blockDim.x) {
     const int64_t row = M + i / kgroups, cg = i % kgroups;
-    *reinterpret_cast<uint32_t*>(scales + scale_offset(row, cg * 4, kgroups)) = 0u;
+    const int64_t off = scale_offset(row, cg * 4, kgroups);
+    if (NVFP4_IN_BOUNDS(off + 3, n_scale_bytes(M, kgroups * 64), st))
+      *reinterpret_cast<uint32_t*>(scales + off) = 0u;
   }
 }
 
@@ -132,6 +140,7 @@ struct QuantOp {
   uint8_t* scales;
   uint8_t* choice;
   int64_t M, K;
+  int* st;  // device status word (bounds-checking build)
 
   template <class C>
   __device__ __forceinline__ void operator()(const Raw16& v, const C& c, float g, int lane) const {
@@ -153,9 +162,10 @@ struct QuantOp {
     }
     (void)lane;
     if (c.valid) {
-      codes[c.vec >> 1] = make_uint2(q0, q1);
-      scales[block_scale_offset(c, K)] = (uint8_t)sc;  // 4 lanes fill one 4-byte group
-      if (kFos && choice) choice[c.vec >> 1] = (uint8_t)pick4;
+      const int64_t off = block_scale_offset(c, K);
+      if (NVFP4_IN_BOUNDS(c.vec >> 1, n_code_words(M, K), st)) codes[c.vec >> 1] = make_uint2(q0, q1);
+      if (NVFP4_IN_BOUNDS(off, n_scale_bytes(M, K), st)) scales[off] = (uint8_t)sc;  // 4 lanes fill one 4-byte group
+      if (kFos && choice && NVFP4_IN_BOUNDS(c.vec >> 1, n_code_words(M, K), st)) choice[c.vec >> 1] = (uint8_t)pick4;
     }
   }
 
@@ -170,7 +180,7 @@ struct QuantOp {
            i += (int64_t)gridDim.x * blockDim.x)
         choice[i] = 0;
     }
-    zero_pad_scale_rows(scales, M, K >> 6);
+    zero_pad_scale_rows(scales, M, K >> 6, st);
   }
 };
 
@@ -179,6 +189,7 @@ template <bool kFos>
 struct FakeOp {
   uint4* y;
   int64_t M, K;
+  int* st;
 
   template <class C>
   __device__ __forceinline__ void operator()(const Raw16& v, const C& c, float g, int lane) const {
@@ -192,11 +203,11 @@ struct FakeOp {
       Block b4;
       quantize_block_tab<true, true, true>(xs, bmax, b4);
       if (b4.err < b6.err) {
-        store_bf16x16(y, c, b4.deq);
+        store_bf16x16(y, c, b4.deq, n_vec16(M, K), st);
         return;
       }
     }
-    store_bf16x16(y, c, b6.deq);
+    store_bf16x16(y, c, b6.deq, n_vec16(M, K), st);
   }
   __device__ __forceinline__ void prepare(float g) const { build_step_table(g); }
   __device__ __forceinline__ void finish() const {}
@@ -208,8 +219,11 @@ struct FakeOp {
   }
 
   template <class C>
-  __device__ static __forceinline__ void store_bf16x16(uint4* y, const C& c, const f32x2 (&out)[8]) {
-    if (!c.valid) return;
+  __device__ static __forceinline__ void store_bf16x16(uint4* y, const C& c, const f32x2 (&out)[8], int64_t n_vec,
+                                                       int* st) {
+    (void)n_vec;
+    (void)st;
+    if (!c.valid || !NVFP4_IN_BOUNDS(c.vec + 1, n_vec, st)) return;
     y[c.vec] = make_uint4(to_bf16x2(out[0]), to_bf16x2(out[1]), to_bf16x2(out[2]), to_bf16x2(out[3]));
     y[c.vec + 1] = make_uint4(to_bf16x2(out[4]), to_bf16x2(out[5]), to_bf16x2(out[6]), to_bf16x2(out[7]));
   }
@@ -220,11 +234,13 @@ struct FrozenFakeOp {
   uint4* y;
   const uint8_t* scales_frozen;
   int64_t M, K;
+  int* st;
 
   template <class C>
   __device__ __forceinline__ void operator()(const Raw16& v, const C& c, float g, int lane) const {
     (void)lane;
-    const uint32_t sc = c.valid ? scales_frozen[block_scale_offset(c, K)] : 1u;
+    const int64_t off = block_scale_offset(c, K);
+    const uint32_t sc = c.valid && NVFP4_IN_BOUNDS(off, n_scale_bytes(M, K), st) ? scales_frozen[off] : 1u;
     const float d = step_table().d[sc & 127u];
     const float r = step_table().r[sc & 127u];
     const f32x2 rr = pack2(r, r), dd = pack2(d, d);
@@ -235,7 +251,7 @@ struct FrozenFakeOp {
     e2m1_unpack4(e2m1_pack4(sv[4], sv[5], sv[6], sv[7]), out + 4);
 #pragma unroll
     for (int i = 0; i < 8; ++i) out[i] = mul2(dd, out[i]);
-    FakeOp<false>::store_bf16x16(y, c, out);
+    FakeOp<false>::store_bf16x16(y, c, out, n_vec16(M, K), st);
   }
   __device__ __forceinline__ void prepare(float g) const { build_step_table(g); }
   __device__ __forceinline__ void finish() const {}
@@ -254,8 +270,10 @@ __device__ __forceinline__ uint32_t ste_word(uint32_t gy, f32x2 xr) {
 
 template <class C>
 __device__ __forceinline__ void ste_store(const uint4* gy, uint4* gx, const C& c, const f32x2 (&xs)[8],
-                                          float r) {
-  if (!c.valid) return;
+                                          float r, int64_t n_vec, int* st) {
+  (void)n_vec;
+  (void)st;
+  if (!c.valid || !NVFP4_IN_BOUNDS(c.vec + 1, n_vec, st)) return;
   const uint4 a = ld_stream(gy + c.vec), b = ld_stream(gy + c.vec + 1);
   const f32x2 rr = pack2(r, r);
   gx[c.vec] = make_uint4(ste_word(a.x, mul2(xs[0], rr)), ste_word(a.y, mul2(xs[1], rr)),
@@ -270,6 +288,7 @@ struct SteOp {
   const uint4* gy;
   uint4* gx;
   int64_t M, K;
+  int* st;
 
   __device__ __forceinline__ void prepare(float g) const { build_step_table(g); }
   template <class C>
@@ -287,7 +306,7 @@ struct SteOp {
     } else {
       sc = block_scale_code(bmax, g, 6.0f);
     }
-    ste_store(gy, gx, c, xs, step_table().r[sc]);
+    ste_store(gy, gx, c, xs, step_table().r[sc], n_vec16(M, K), st);
   }
   __device__ __forceinline__ void finish() const {}
 };
@@ -298,15 +317,17 @@ struct FrozenSteOp {
   uint4* gx;
   const uint8_t* scales_frozen;
   int64_t M, K;
+  int* st;
 
   __device__ __forceinline__ void prepare(float g) const { build_step_table(g); }
   template <class C>
   __device__ __forceinline__ void operator()(const Raw16& v, const C& c, float g, int lane) const {
     (void)lane;
-    const uint32_t sc = c.valid ? scales_frozen[block_scale_offset(c, K)] : 1u;
+    const int64_t off = block_scale_offset(c, K);
+    const uint32_t sc = c.valid && NVFP4_IN_BOUNDS(off, n_scale_bytes(M, K), st) ? scales_frozen[off] : 1u;
     f32x2 xs[8];
     unpack_block(v, xs);
-    ste_store(gy, gx, c, xs, step_table().r[sc & 127u]);
+    ste_store(gy, gx, c, xs, step_table().r[sc & 127u], n_vec16(M, K), st);
   }
   __device__ __forceinline__ void finish() const {}
 };
@@ -324,6 +345,7 @@ struct MseOp {
   uint8_t* scales;
   uint8_t* choice;
   int64_t M, K;
+  int* st;
 
   __device__ __forceinline__ void prepare(float g) const { build_step_table(g); }
 
@@ -355,13 +377,14 @@ struct MseOp {
       }
     }
     if (c.valid) {
-      codes[c.vec >> 1] = make_uint2(q0, q1);
-      scales[block_scale_offset(c, K)] = (uint8_t)best_sc;
-      if (choice) choice[c.vec >> 1] = 0;
+      const int64_t off = block_scale_offset(c, K);
+      if (NVFP4_IN_BOUNDS(c.vec >> 1, n_code_words(M, K), st)) codes[c.vec >> 1] = make_uint2(q0, q1);
+      if (NVFP4_IN_BOUNDS(off, n_scale_bytes(M, K), st)) scales[off] = (uint8_t)best_sc;
+      if (choice && NVFP4_IN_BOUNDS(c.vec >> 1, n_code_words(M, K), st)) choice[c.vec >> 1] = 0;
     }
   }
 
-  __device__ __forceinline__ void finish() const { zero_pad_scale_rows(scales, M, K >> 6); }
+  __device__ __forceinline__ void finish() const { zero_pad_scale_rows(scales, M, K >> 6, st); }
 };
 
 // ----------------------------------------------------------------------------
@@ -395,7 +418,8 @@ __global__ void __launch_bounds__(kQThreads) stream_pass_kernel(const uint4* __r
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
       cc[u] = chunk_at_t<Idx>(ch0 + u * nwarps, cpr, cpr_magic, K, lane);
-      load_raw16(x, cc[u].vec, cc[u].valid && ch0 + u * nwarps < n_chunks, vv[u]);
+      const bool live = cc[u].valid && ch0 + u * nwarps < n_chunks;
+      load_raw16(x, cc[u].vec, live && NVFP4_IN_BOUNDS(cc[u].vec + 1, n_vec16(M, K), status), vv[u]);
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
@@ -486,7 +510,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_dynamic_kernel(const u
       a[u] = b[u] = make_uint4(0, 0, 0, 0);
       if (ch < hi) {
         const ChunkT<Idx> c = chunk_at_t<Idx>(ch, cpr, cpr_magic, K, lane);
-        if (c.valid) {
+        if (c.valid && NVFP4_IN_BOUNDS(c.vec + 1, n_vec16(M, K), status)) {
           a[u] = ld_stream(x + c.vec);
           b[u] = ld_stream(x + c.vec + 1);
         }
@@ -559,7 +583,7 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_dynamic_kernel(const u
         if (k < nkeep) {
           a = keep[k * 64 + lane];
           b = keep[k * 64 + 32 + lane];
-        } else {
+        } else if (NVFP4_IN_BOUNDS(cc[u].vec + 1, n_vec16(M, K), status)) {
           a = ld_stream(x + cc[u].vec);
           b = ld_stream(x + cc[u].vec + 1);
         }
@@ -693,12 +717,12 @@ cudaError_t launch_quantize(const void* x, int64_t M, int64_t K, int mode, const
                             float* g_out, uint8_t* choice, int* status, int num_sms, cudaStream_t s) {
   uint2* c = reinterpret_cast<uint2*>(codes);
   if (mode == 2)
-    return launch_stream(x, M, K, partial, n_partial, g_static, MseOp{c, scales, choice, M, K}, g_out, status,
+    return launch_stream(x, M, K, partial, n_partial, g_static, MseOp{c, scales, choice, M, K, status}, g_out, status,
                          num_sms, s);
   if (mode == 1)
-    return launch_stream(x, M, K, partial, n_partial, g_static, QuantOp<true>{c, scales, choice, M, K}, g_out, status,
+    return launch_stream(x, M, K, partial, n_partial, g_static, QuantOp<true>{c, scales, choice, M, K, status}, g_out, status,
                          num_sms, s);
-  return launch_stream(x, M, K, partial, n_partial, g_static, QuantOp<false>{c, scales, choice, M, K}, g_out, status,
+  return launch_stream(x, M, K, partial, n_partial, g_static, QuantOp<false>{c, scales, choice, M, K, status}, g_out, status,
                        num_sms, s);
 }
 
@@ -707,27 +731,27 @@ cudaError_t launch_fake_quant(const void* x, int64_t M, int64_t K, bool fos, con
                               void* y, int* status, int num_sms, cudaStream_t s) {
   uint4* yv = static_cast<uint4*>(y);
   if (scales_frozen)
-    return launch_stream(x, M, K, partial, n_partial, g_static, FrozenFakeOp{yv, scales_frozen, M, K}, nullptr,
+    return launch_stream(x, M, K, partial, n_partial, g_static, FrozenFakeOp{yv, scales_frozen, M, K, status}, nullptr,
                          status, num_sms, s);
   if (fos)
-    return launch_stream(x, M, K, partial, n_partial, g_static, FakeOp<true>{yv, M, K}, nullptr, status, num_sms, s);
-  return launch_stream(x, M, K, partial, n_partial, g_static, FakeOp<false>{yv, M, K}, nullptr, status, num_sms, s);
+    return launch_stream(x, M, K, partial, n_partial, g_static, FakeOp<true>{yv, M, K, status}, nullptr, status, num_sms, s);
+  return launch_stream(x, M, K, partial, n_partial, g_static, FakeOp<false>{yv, M, K, status}, nullptr, status, num_sms, s);
 }
 
 cudaError_t launch_quantize_fused(const void* x, int64_t M, int64_t K, int mode, uint32_t* ws, uint8_t* codes,
                                   uint8_t* scales, float* g_out, uint8_t* choice, int* status, int num_sms,
                                   cudaStream_t s) {
   uint2* c = reinterpret_cast<uint2*>(codes);
-  if (mode == 2) return launch_fused(x, M, K, ws, MseOp{c, scales, choice, M, K}, g_out, status, num_sms, s);
-  if (mode == 1) return launch_fused(x, M, K, ws, QuantOp<true>{c, scales, choice, M, K}, g_out, status, num_sms, s);
-  return launch_fused(x, M, K, ws, QuantOp<false>{c, scales, choice, M, K}, g_out, status, num_sms, s);
+  if (mode == 2) return launch_fused(x, M, K, ws, MseOp{c, scales, choice, M, K, status}, g_out, status, num_sms, s);
+  if (mode == 1) return launch_fused(x, M, K, ws, QuantOp<true>{c, scales, choice, M, K, status}, g_out, status, num_sms, s);
+  return launch_fused(x, M, K, ws, QuantOp<false>{c, scales, choice, M, K, status}, g_out, status, num_sms, s);
 }
 
 cudaError_t launch_fake_quant_fused(const void* x, int64_t M, int64_t K, bool fos, uint32_t* ws, void* y,
                                     int* status, int num_sms, cudaStream_t s) {
   uint4* yv = static_cast<uint4*>(y);
-  if (fos) return launch_fused(x, M, K, ws, FakeOp<true>{yv, M, K}, nullptr, status, num_sms, s);
-  return launch_fused(x, M, K, ws, FakeOp<false>{yv, M, K}, nullptr, status, num_sms, s);
+  if (fos) return launch_fused(x, M, K, ws, FakeOp<true>{yv, M, K, status}, nullptr, status, num_sms, s);
+  return launch_fused(x, M, K, ws, FakeOp<false>{yv, M, K, status}, nullptr, status, num_sms, s);
 }
 
 cudaError_t launch_convert(const float* in, int64_t n, uint8_t* out, bool e4m3, int num_sms,
@@ -753,12 +777,12 @@ cudaError_t launch_fake_quant_bwd(const void* x, const void* gy, int64_t M, int6
   const uint4* gyv = static_cast<const uint4*>(gy);
   uint4* gxv = static_cast<uint4*>(gx);
   if (scales_frozen)
-    return launch_stream(x, M, K, partial, n_partial, g_static, FrozenSteOp{gyv, gxv, scales_frozen, M, K}, nullptr,
+    return launch_stream(x, M, K, partial, n_partial, g_static, FrozenSteOp{gyv, gxv, scales_frozen, M, K, status}, nullptr,
                          status, num_sms, s);
   if (fos)
-    return launch_stream(x, M, K, partial, n_partial, g_static, SteOp<true>{gyv, gxv, M, K}, nullptr, status,
+    return launch_stream(x, M, K, partial, n_partial, g_static, SteOp<true>{gyv, gxv, M, K, status}, nullptr, status,
                          num_sms, s);
-  return launch_stream(x, M, K, partial, n_partial, g_static, SteOp<false>{gyv, gxv, M, K}, nullptr, status, num_sms,
+  return launch_stream(x, M, K, partial, n_partial, g_static, SteOp<false>{gyv, gxv, M, K, status}, nullptr, status, num_sms,
                        s);
 }
 
@@ -766,8 +790,8 @@ cudaError_t launch_fake_quant_bwd_fused(const void* x, const void* gy, int64_t M
                                         void* gx, int* status, int num_sms, cudaStream_t s) {
   const uint4* gyv = static_cast<const uint4*>(gy);
   uint4* gxv = static_cast<uint4*>(gx);
-  if (fos) return launch_fused(x, M, K, ws, SteOp<true>{gyv, gxv, M, K}, nullptr, status, num_sms, s);
-  return launch_fused(x, M, K, ws, SteOp<false>{gyv, gxv, M, K}, nullptr, status, num_sms, s);
+  if (fos) return launch_fused(x, M, K, ws, SteOp<true>{gyv, gxv, M, K, status}, nullptr, status, num_sms, s);
+  return launch_fused(x, M, K, ws, SteOp<false>{gyv, gxv, M, K, status}, nullptr, status, num_sms, s);
 }
 
 // ----------------------------------------------------------------------------
@@ -781,7 +805,8 @@ template <bool kNarrow>
 __global__ void __launch_bounds__(kQThreads) dequantize_kernel(const uint2* __restrict__ codes,
                                                                 const uint8_t* __restrict__ scales,
                                                                 const float* __restrict__ g_ptr, int64_t M,
-                                                                int64_t K, uint64_t cpr_magic, uint4* __restrict__ y) {
+                                                                int64_t K, uint64_t cpr_magic, uint4* __restrict__ y,
+                                                                int* status) {
   using Idx = typename std::conditional<kNarrow, uint32_t, int64_t>::type;
   const float g = *g_ptr;
   const int32_t cpr = (int32_t)((K + 511) >> 9);
@@ -798,8 +823,10 @@ __global__ void __launch_bounds__(kQThreads) dequantize_kernel(const uint2* __re
       const int32_t ch = ch0 + u * nwarps;
       cc[u] = chunk_at_t<Idx>(ch < n_chunks ? ch : 0, cpr, cpr_magic, K, lane);
       const bool ok = ch < n_chunks && cc[u].valid;
-      q[u] = ok ? codes[cc[u].vec >> 1] : make_uint2(0, 0);
-      sc[u] = ok ? scales[block_scale_offset(cc[u], K)] : 1u;
+      const int64_t off = block_scale_offset(cc[u], K);
+      q[u] = ok && NVFP4_IN_BOUNDS(cc[u].vec >> 1, n_code_words(M, K), status) ? codes[cc[u].vec >> 1]
+                                                                                : make_uint2(0, 0);
+      sc[u] = ok && NVFP4_IN_BOUNDS(off, n_scale_bytes(M, K), status) ? scales[off] : 1u;
     }
 #pragma unroll
     for (int u = 0; u < kUnroll; ++u) {
@@ -811,13 +838,13 @@ __global__ void __launch_bounds__(kQThreads) dequantize_kernel(const uint2* __re
       e2m1_unpack4(q[u].y, v + 4);
 #pragma unroll
       for (int i = 0; i < 8; ++i) v[i] = mul2(dd, v[i]);
-      FakeOp<false>::store_bf16x16(y, cc[u], v);
+      FakeOp<false>::store_bf16x16(y, cc[u], v, n_vec16(M, K), status);
     }
   }
 }
 
 cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const float* g, int64_t M, int64_t K,
-                              void* y, int num_sms, cudaStream_t s) {
+                              void* y, int* status, int num_sms, cudaStream_t s) {
   const int64_t chunks = M * ((K + 511) / 512);
   if (chunks == 0) return cudaSuccess;
   if (chunks >= (int64_t(1) << 30)) return cudaErrorInvalidValue;  // 32-bit chunk loops
@@ -826,10 +853,10 @@ cudaError_t launch_dequantize(const uint8_t* codes, const uint8_t* scales, const
   note_launch();
   if (narrow_chunks(M, K))
     dequantize_kernel<true><<<grid, kQThreads, 0, s>>>(reinterpret_cast<const uint2*>(codes), scales, g, M, K,
-                                                       chunk_magic_narrow(K), static_cast<uint4*>(y));
+                                                       chunk_magic_narrow(K), static_cast<uint4*>(y), status);
   else
     dequantize_kernel<false><<<grid, kQThreads, 0, s>>>(reinterpret_cast<const uint2*>(codes), scales, g, M, K,
-                                                        chunk_magic(K), static_cast<uint4*>(y));
+                                                        chunk_magic(K), static_cast<uint4*>(y), status);
   return cudaGetLastError();
 }
 

@@ -17,6 +17,21 @@ def pytest_collection_modifyitems(config, items):
     pass
 
 
+@pytest.fixture(autouse=True)
+def _no_index_out_of_bounds():
+    """Under the bounds-checking build (NVFP4_LIBRARY=debug), fail a test
+    after which the device status word reads NVFP4_ERR_BOUNDS (8)."""
+    yield
+    if os.environ.get("NVFP4_LIBRARY") != "debug":
+        return
+    import torch
+    if not torch.cuda.is_available():
+        return
+    import qad_nvfp4_quantize_b200 as nv
+    st = nv.device_status(clear=True)
+    assert st != 8, "the bounds-checking build flagged an index outside its buffer"
+
+
 @pytest.fixture(scope="session")
 def golden_dir():
     return os.path.join(ROOT, "tests", "golden")

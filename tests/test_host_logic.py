@@ -56,6 +56,17 @@ def test_library_exports_every_declared_symbol(clib):
     assert len(_header_symbols()) >= 14
 
 
+def test_bounds_checking_build_exports_the_same_symbols():
+    path = os.path.join(ROOT, "qad_nvfp4_quantize_b200", "libnvfp4_debug.so")
+    if not os.path.exists(path):
+        pytest.fail("libnvfp4_debug.so is not built")
+    dbg = ctypes.CDLL(path)
+    missing = [s for s in _header_symbols() if not hasattr(dbg, s)]
+    assert not missing, f"not exported by the bounds-checking build: {missing}"
+    dbg.nvfp4_status_string.restype = ctypes.c_char_p
+    assert dbg.nvfp4_status_string(8).startswith(b"a computed index")
+
+
 def test_host_side_queries_and_validation(clib):
     import qad_nvfp4_quantize_b200 as nv
     L = nv.lib()
