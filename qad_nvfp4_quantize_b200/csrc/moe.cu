@@ -441,7 +441,7 @@ constexpr int kRowThreads = 256;
 constexpr int kRowUnroll = 4;
 
 template <bool kNarrow>
-__global__ void __launch_bounds__(kRowThreads) moe_quantize_h_kernel(
+__global__ void __launch_bounds__(kRowThreads, 4) moe_quantize_h_kernel(
     const uint4* __restrict__ src, int64_t K, int64_t R, const int32_t* __restrict__ row_pair,
     const int32_t* __restrict__ tile_expert, const int32_t* __restrict__ tile_count,
     const uint32_t* __restrict__ amax_bits, int E, uint2* __restrict__ codes, uint8_t* __restrict__ scales,
@@ -798,8 +798,17 @@ cudaError_t launch_moe(const MoeArgs& a, int* status, int num_sms, cudaStream_t 
     if ((e = cudaLaunchKernelExC(&cfg, kern, args)) != cudaSuccess) return e;
   }
 
-  const int qgrid = num_sms * 4;
+  // quantize h: one wave of resident CTAs (a grid beyond what fits leaves a
+  // partial second wave behind the first)
   const size_t qsmem = (size_t)a.E * sizeof(float);
+  auto q_occupancy = [qsmem](auto kern) {
+    int occ = 0;
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kern, kRowThreads, qsmem) == cudaSuccess && occ > 0
+               ? occ
+               : 1;
+  };
+  const int qgrid = num_sms * (narrow_chunks(R, a.I) ? q_occupancy(moe_quantize_h_kernel<true>)
+                                                     : q_occupancy(moe_quantize_h_kernel<false>));
 
   // 3. gate_up grouped GEMM
   {
