@@ -236,6 +236,8 @@ NVFP4_DEVINL void bulk_reduce_add_f32(float* dst, uint32_t smem_src, uint32_t by
 NVFP4_DEVINL void bulk_commit_group() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 // Wait until the bulk stores issued by this thread have finished reading shared memory.
 NVFP4_DEVINL void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// Wait until at most the latest bulk group of this thread may still be reading its source.
+NVFP4_DEVINL void bulk_wait_read_but_one() { asm volatile("cp.async.bulk.wait_group.read 1;" ::: "memory"); }
 // Wait until the bulk stores issued by this thread are complete.
 NVFP4_DEVINL void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 // Make this thread's generic-proxy shared-memory writes visible to the async proxy (TMA).

@@ -136,6 +136,7 @@ __device__ __forceinline__ void zero_pad_scale_rows(uint8_t* scales, int64_t M, 
 // Quantize: codes, tiled block scales and (four_over_six) the choice map.
 template <bool kFos>
 struct QuantOp {
+  static constexpr bool kBulkRefill = false;  // fused pass: phase 2 re-reads through registers
   uint2* codes;
   uint8_t* scales;
   uint8_t* choice;
@@ -187,6 +188,7 @@ struct QuantOp {
 // Fake-quant with block scales computed from the values (max or four_over_six).
 template <bool kFos>
 struct FakeOp {
+  static constexpr bool kBulkRefill = true;  // fused pass: phase 2 refills freed slots by bulk copies
   uint4* y;
   int64_t M, K;
   int* st;
@@ -285,6 +287,7 @@ __device__ __forceinline__ void ste_store(const uint4* gy, uint4* gx, const C& c
 // Backward with the forward's scales recomputed from x (max or four_over_six).
 template <bool kFos>
 struct SteOp {
+  static constexpr bool kBulkRefill = true;
   const uint4* gy;
   uint4* gx;
   int64_t M, K;
@@ -341,6 +344,7 @@ struct FrozenSteOp {
 // whose bound exceeds the best error (it cannot win or tie). d and 1/d per
 // code are tabulated once per CTA.
 struct MseOp {
+  static constexpr bool kBulkRefill = false;
   uint2* codes;
   uint8_t* scales;
   uint8_t* choice;
@@ -435,19 +439,30 @@ __global__ void __launch_bounds__(kQThreads) stream_pass_kernel(const uint4* __r
 //
 // One CTA per SM (cooperative launch, so all CTAs are resident). CTA c owns a
 // contiguous range of chunks. Phase 1 streams the range once, reducing the
-// BF16 magnitude maximum and keeping the first kKeepChunks chunks (up to
-// 200 KB) in shared memory. The CTA maxima meet at a grid-wide barrier (two
-// words in the workspace, returned to zero by every completed barrier, so the
-// workspace must be zero before its first use). Phase 2 walks the range
-// backwards: the chunks that were not kept -- read last in phase 1, so the
-// most likely to still be in L2 -- are read again from global memory, the
-// kept ones come from shared memory. X therefore crosses HBM about once.
+// BF16 magnitude maximum and keeping the first kKeepChunks chunks (224 KB)
+// in shared memory; chunk k of the range goes to slot k, owned by warp k % 32.
+// The CTA maxima meet at a grid-wide barrier (a counter in the workspace that
+// stays a multiple of the grid, so the workspace must be zero before its
+// first use). Phase 2 then re-reads the range, in one of two ways chosen by
+// the op (both read X from HBM about once in total):
+//  * register re-reads (ops with little output: quantize, MSE): each warp
+//    walks the range backwards, two chunks per trip; chunks that were not
+//    kept -- read last in phase 1, so the most likely to still be in L2 --
+//    come from global memory, the kept ones from shared memory;
+//  * bulk refills (ops that write a BF16 tensor: fake-quant, STE): each warp
+//    first processes its kept chunks, and every slot it frees is refilled at
+//    once by one bulk copy (the TMA engine, completion on the slot's
+//    mbarrier) of one of its not-kept chunks, newest first; kSlots chunks per
+//    warp are then in flight while the warp computes and stores. Measured on
+//    16384 x 4096: fake-quant 69.6 -> 63.5 us, STE 90.1 -> 81.9 us, while the
+//    quantize ops were 2-4 us slower this way.
 // ----------------------------------------------------------------------------
 constexpr int kFusedThreads = 1024;
 constexpr int kFusedWarps = kFusedThreads / 32;
-constexpr int kKeepChunks = 200;                       // 1 KB of BF16 per chunk
-constexpr int kFusedSmem = kKeepChunks * 1024;
-constexpr int kFusedUnroll = 2;                        // phase 2: chunks per trip
+constexpr int kSlots = 7;                              // kept / in-flight chunks per warp
+constexpr int kKeepChunks = kSlots * 32;               // 1 KB of BF16 per chunk
+constexpr int kFusedSmem = kKeepChunks * 1024 + kKeepChunks * 8;  // + one mbarrier per slot
+constexpr int kFusedUnroll = 2;                        // register re-reads: chunks per trip
 constexpr int kLoadUnroll = 4;                         // phase 1: chunk loads in flight per warp
 
 // Grid-wide barrier on a 64-bit arrival counter that only grows: CTA arrival
@@ -499,6 +514,13 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_dynamic_kernel(const u
   const int32_t lo = (int32_t)min((int64_t)blockIdx.x * per, (int64_t)n_chunks);
   const int32_t hi = lo + per < n_chunks ? lo + per : n_chunks;
   const int32_t nkeep = hi - lo < kKeepChunks ? (hi - lo > 0 ? hi - lo : 0) : kKeepChunks;
+  uint64_t* slot_bar = reinterpret_cast<uint64_t*>(keep + kKeepChunks * 64);
+  __shared__ int s_abort;
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kKeepChunks; ++i) mbar_init(&slot_bar[i], 1);
+    s_abort = 0;
+    fence_barrier_init();
+  }
 
   // ---- phase 1: magnitude maximum, keep the first nkeep chunks
   uint32_t m2 = 0;
@@ -569,32 +591,128 @@ __global__ void __launch_bounds__(kFusedThreads, 1) fused_dynamic_kernel(const u
 
   grid_dependents_launch();  // a dependent GEMM may set up while phase 2 runs
 
-  // ---- phase 2: backwards, re-read chunks that were not kept, then kept ones
-  for (int32_t top = hi - 1 - warp; top >= lo; top -= kFusedUnroll * kFusedWarps) {
-    Raw16 vv[kFusedUnroll];
-    ChunkT<Idx> cc[kFusedUnroll];
+  if constexpr (!Op::kBulkRefill) {
+    // ---- phase 2, register re-reads: backwards, not-kept chunks from global
+    // memory, then the kept ones
+    for (int32_t top = hi - 1 - warp; top >= lo; top -= kFusedUnroll * kFusedWarps) {
+      Raw16 vv[kFusedUnroll];
+      ChunkT<Idx> cc[kFusedUnroll];
 #pragma unroll
-    for (int u = 0; u < kFusedUnroll; ++u) {
-      const int32_t ch = top - u * kFusedWarps;
-      uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
-      cc[u] = chunk_at_t<Idx>(ch >= lo ? ch : lo, cpr, cpr_magic, K, lane);
-      if (ch >= lo && cc[u].valid) {
-        const int32_t k = ch - lo;
-        if (k < nkeep) {
-          a = keep[k * 64 + lane];
-          b = keep[k * 64 + 32 + lane];
-        } else if (NVFP4_IN_BOUNDS(cc[u].vec + 1, n_vec16(M, K), status)) {
-          a = ld_stream(x + cc[u].vec);
-          b = ld_stream(x + cc[u].vec + 1);
+      for (int u = 0; u < kFusedUnroll; ++u) {
+        const int32_t ch = top - u * kFusedWarps;
+        uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+        cc[u] = chunk_at_t<Idx>(ch >= lo ? ch : lo, cpr, cpr_magic, K, lane);
+        if (ch >= lo && cc[u].valid) {
+          const int32_t k = ch - lo;
+          if (k < nkeep) {
+            a = keep[k * 64 + lane];
+            b = keep[k * 64 + 32 + lane];
+          } else if (NVFP4_IN_BOUNDS(cc[u].vec + 1, n_vec16(M, K), status)) {
+            a = ld_stream(x + cc[u].vec);
+            b = ld_stream(x + cc[u].vec + 1);
+          }
+        }
+        vv[u].w[0] = a.x; vv[u].w[1] = a.y; vv[u].w[2] = a.z; vv[u].w[3] = a.w;
+        vv[u].w[4] = b.x; vv[u].w[5] = b.y; vv[u].w[6] = b.z; vv[u].w[7] = b.w;
+      }
+#pragma unroll
+      for (int u = 0; u < kFusedUnroll; ++u) {
+        if (top - u * kFusedWarps < lo) break;  // warp-uniform
+        op(vv[u], cc[u], g, lane);
+      }
+    }
+  } else {
+    // ---- phase 2: kept chunks first, then the not-kept ones through the freed
+    // slots, each refilled by one bulk copy (1 KB, TMA engine) on the slot's
+    // mbarrier as soon as its kept chunk has been quantized.
+    const int32_t n = hi - lo;
+    int32_t nx = n - 1 - warp;  // next not-kept chunk to fetch (relative to lo)
+    uint32_t armed = 0, par = 0;  // per slot index t: a copy in flight; parity of its next completion
+    const bool full_chunks = (K & 511) == 0;  // then chunk ch is the 1 KB at byte 1024 ch
+    auto fetch_next = [&](int t) {
+      if (nx < nkeep) return;
+      const int32_t s = warp + t * kFusedWarps;
+      Idx vec0;
+      int64_t elems = 512;
+      if (full_chunks) {
+        vec0 = (Idx)(lo + nx) * (Idx)64;
+      } else {
+        const ChunkT<Idx> c0 = chunk_at_t<Idx>(lo + nx, cpr, cpr_magic, K, 0);
+        vec0 = c0.vec;
+        elems = K - c0.col < 512 ? K - c0.col : 512;
+      }
+      const uint32_t bytes = (uint32_t)elems * 2u;
+      if (NVFP4_IN_BOUNDS(vec0 + (Idx)(elems / 8) - 1, n_vec16(M, K), status)) {
+        __syncwarp();  // every lane has consumed the slot's previous contents
+        if (lane == 0) {
+          fence_proxy_async_smem();
+          mbar_arrive_expect_tx(&slot_bar[s], bytes);
+          bulk_load(&keep[s * 64], x + vec0, bytes, &slot_bar[s]);
+        }
+        armed |= 1u << t;
+      }
+      nx -= kFusedWarps;
+    };
+    {
+      int t = 0;
+      for (int32_t s = warp; s < nkeep; s += kFusedWarps, ++t) {
+        const ChunkT<Idx> c = chunk_at_t<Idx>(lo + s, cpr, cpr_magic, K, lane);
+        uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+        if (c.valid) {
+          a = keep[s * 64 + lane];
+          b = keep[s * 64 + 32 + lane];
+        }
+        Raw16 v;
+        v.w[0] = a.x; v.w[1] = a.y; v.w[2] = a.z; v.w[3] = a.w;
+        v.w[4] = b.x; v.w[5] = b.y; v.w[6] = b.z; v.w[7] = b.w;
+        op(v, c, g, lane);
+        fetch_next(t);
+      }
+    }
+    if (n > nkeep) {  // then nkeep == kKeepChunks: every warp owns kSlots slots
+      int t = 0;
+      bool ok = true;
+      for (int32_t cur = n - 1 - warp; cur >= nkeep; cur -= kFusedWarps) {
+        const int32_t s = warp + t * kFusedWarps;
+        if ((armed >> t) & 1u) {
+          if (!mbar_wait_warp(&slot_bar[s], (par >> t) & 1u, &s_abort, timeout_ns)) {
+            ok = false;
+            break;
+          }
+          par ^= 1u << t;
+          armed &= ~(1u << t);
+        }
+        const ChunkT<Idx> c = chunk_at_t<Idx>(lo + cur, cpr, cpr_magic, K, lane);
+        // the copy keeps global order (lane L's 32 bytes at 32 L); lanes 4-7 of
+        // each group of 8 take their halves in the other order, so that each
+        // 16-byte load instruction covers all 32 banks
+        const uint8_t* sb = reinterpret_cast<const uint8_t*>(&keep[s * 64]) + lane * 32;
+        const bool sw = (lane & 4) != 0;
+        uint4 a = make_uint4(0, 0, 0, 0), b = make_uint4(0, 0, 0, 0);
+        if (c.valid) {
+          const uint4 u0 = *reinterpret_cast<const uint4*>(sb + (sw ? 16 : 0));
+          const uint4 u1 = *reinterpret_cast<const uint4*>(sb + (sw ? 0 : 16));
+          a = sw ? u1 : u0;
+          b = sw ? u0 : u1;
+        }
+        Raw16 v;
+        v.w[0] = a.x; v.w[1] = a.y; v.w[2] = a.z; v.w[3] = a.w;
+        v.w[4] = b.x; v.w[5] = b.y; v.w[6] = b.z; v.w[7] = b.w;
+        op(v, c, g, lane);
+        fetch_next(t);
+        t = t + 1 == kSlots ? 0 : t + 1;
+      }
+      if (!ok) {
+        if (lane == 0) record_status(status, NVFP4_ERR_TIMEOUT);
+        // let the copies still in flight land (bounded) before the CTA exits
+        for (int u = 0; u < kSlots; ++u) {
+          if (!((armed >> u) & 1u)) continue;
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(&slot_bar[warp + u * kFusedWarps], (par >> u) & 1u) &&
+                 globaltimer_ns() - t0 < 1000000ull) {
+          }
         }
       }
-      vv[u].w[0] = a.x; vv[u].w[1] = a.y; vv[u].w[2] = a.z; vv[u].w[3] = a.w;
-      vv[u].w[4] = b.x; vv[u].w[5] = b.y; vv[u].w[6] = b.z; vv[u].w[7] = b.w;
-    }
-#pragma unroll
-    for (int u = 0; u < kFusedUnroll; ++u) {
-      if (top - u * kFusedWarps < lo) break;  // warp-uniform
-      op(vv[u], cc[u], g, lane);
     }
   }
   op.finish();
