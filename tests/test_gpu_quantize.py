@@ -259,6 +259,27 @@ def test_ste_backward_dynamic_and_static(nv, mode):
     assert (ref == 0).any()
 
 
+@pytest.mark.parametrize("M,K", [(40000, 64), (12000, 1088), (9000, 2048)])
+def test_fake_quant_and_ste_refill_freed_slots(nv, M, K):
+    # More 512-element chunks per CTA than the 224 it keeps in shared memory,
+    # so phase 2 of the fused pass refills freed slots by bulk copies: partial
+    # chunks (K = 64, and the 64-element tail of K = 1088) and whole 1 KB
+    # chunks (K = 2048), all compared with the oracle bit for bit.
+    rng = np.random.default_rng(M + K)
+    x = inputs.to_bf16((rng.standard_t(3, (M, K)) * 0.3).astype(np.float32))
+    gy = inputs.to_bf16(rng.standard_normal((M, K)).astype(np.float32))
+    cpr = -(-K // 512)
+    per = -(-(M * cpr) // torch.cuda.get_device_properties(0).multi_processor_count)
+    ch = per * 10 + 240  # the 241st chunk of CTA 10's range: not kept
+    x[ch // cpr, (ch % cpr) * 512] = 40.0  # the tensor's amax
+    xd, gyd = x.cuda(), gy.cuda()
+    xf, gf = bf16_np(x), bf16_np(gy)
+    for mode in ("max", "four_over_six"):
+        np.testing.assert_array_equal(bf16_np(nv.fake_quant(xd, mode)), o.fake_quant(xf, mode))
+    np.testing.assert_array_equal(bf16_np(nv.fake_quant_backward(xd, gyd, "max")),
+                                  o.fake_quant_backward(xf, gf, "max"))
+
+
 def test_ste_backward_frozen_scales(nv):
     rng = np.random.default_rng(42)
     M, K = 200, 512
