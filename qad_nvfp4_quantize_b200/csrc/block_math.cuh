@@ -13,6 +13,14 @@
 
 namespace nvfp4 {
 
+// One 32-byte store (two consecutive 16-byte vectors); p must be 32-byte
+// aligned. A warp then writes whole 32-byte sectors in one instruction.
+__device__ __forceinline__ void st_global_32b(uint4* p, uint4 a, uint4 b) {
+  asm volatile("st.global.v8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8};" ::"l"(p), "r"(a.x), "r"(a.y), "r"(a.z),
+               "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+               : "memory");
+}
+
 __device__ __forceinline__ uint4 ld_stream(const uint4* p) {
   uint4 v;
   asm volatile("ld.global.nc.v4.u32 {%0,%1,%2,%3}, [%4];"

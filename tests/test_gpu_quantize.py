@@ -280,6 +280,25 @@ def test_fake_quant_and_ste_refill_freed_slots(nv, M, K):
                                   o.fake_quant_backward(xf, gf, "max"))
 
 
+def test_bf16_outputs_at_16_byte_alignment(nv):
+    # BF16 outputs are written 32 bytes per lane when the buffer is 32-byte
+    # aligned and 16 bytes at a time otherwise; both layouts give the
+    # oracle's values (dynamic and frozen fake-quant, dequantize)
+    rng = np.random.default_rng(5)
+    M, K = 300, 1024
+    x = inputs.to_bf16((rng.standard_t(3, (M, K)) * 0.3).astype(np.float32))
+    xd = x.cuda()
+    base = torch.empty(M * K + 8, dtype=torch.bfloat16, device="cuda")
+    y16 = base[8:].view(M, K)                     # 16 bytes past a 256-byte boundary
+    assert y16.data_ptr() % 32 == 16
+    want = o.fake_quant(bf16_np(x), "max")
+    np.testing.assert_array_equal(bf16_np(nv.fake_quant(xd, "max", out=y16)), want)
+    q = nv.quantize(xd, "max")
+    np.testing.assert_array_equal(bf16_np(nv.fake_quant(xd, g=q.g, scales=q.scales, out=y16)), want)
+    np.testing.assert_array_equal(bf16_np(nv.dequantize(q, out=y16)), want)
+    np.testing.assert_array_equal(bf16_np(nv.dequantize(q)), want)
+
+
 def test_ste_backward_frozen_scales(nv):
     rng = np.random.default_rng(42)
     M, K = 200, 512
