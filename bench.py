@@ -407,7 +407,32 @@ def measure_rows(nv, peaks, flush_buf, stream, spans, iters=10):
     rows["qad_backward_ste_dynamic"] = {"workload": "X 16384x4096 BF16 and dL/dy BF16 -> dL/dx BF16 (clipped STE, "
                                                     "dynamic max scales)", "ms": t * 1e3, "GB/s": alg / t / 1e9,
                                         "frac_hbm": alg / t / 1e9 / hbm, "algorithmic_bytes": alg}
-    del gy, gx
+    # the same ops with scales fixed beforehand (a static global scale, or the
+    # frozen scales of a calibration): one streaming pass each
+    qf = nv.quantize(x)
+    xq_s = nv.quantize(x, "max", g=qf.g)
+    tot, _ = time_loop(lambda ev: nv.quantize(x, "max", g=qf.g, out=xq_s), iters, 2, flush_buf, stream,
+                       name='quantize_static_g_cfg5_x')
+    t = statistics.median(tot) * 1e-3
+    alg = x.numel() * 2.5625
+    rows["quantize_static_g_cfg5_x"] = {"workload": "X 16384x4096 BF16, given global scale", "ms": t * 1e3,
+                                        "GB/s": alg / t / 1e9, "frac_hbm": alg / t / 1e9 / hbm,
+                                        "algorithmic_bytes": alg}
+    tot, _ = time_loop(lambda ev: nv.fake_quant(x, g=qf.g, scales=qf.scales, out=y), iters, 2, flush_buf, stream,
+                       name='fake_quant_frozen')
+    t = statistics.median(tot) * 1e-3
+    alg = x.numel() * (4.0 + 1 / 16)
+    rows["fake_quant_frozen"] = {"workload": "X 16384x4096 BF16 -> BF16 with frozen global and block scales",
+                                 "ms": t * 1e3, "GB/s": alg / t / 1e9, "frac_hbm": alg / t / 1e9 / hbm,
+                                 "algorithmic_bytes": alg}
+    tot, _ = time_loop(lambda ev: nv.fake_quant_backward(x, gy, g=qf.g, scales=qf.scales, out=gx), iters, 2,
+                       flush_buf, stream, name='qad_backward_ste_frozen')
+    t = statistics.median(tot) * 1e-3
+    alg = x.numel() * (6.0 + 1 / 16)
+    rows["qad_backward_ste_frozen"] = {"workload": "as qad_backward_ste_dynamic with frozen global and block scales",
+                                       "ms": t * 1e3, "GB/s": alg / t / 1e9, "frac_hbm": alg / t / 1e9 / hbm,
+                                       "algorithmic_bytes": alg}
+    del gy, gx, qf, xq_s
     xq = nv.quantize(x)
     tot, _ = time_loop(lambda ev: nv.quantize(x, out=xq), iters, 2, flush_buf, stream, name='quantize_dynamic_cfg5_x')
     t = statistics.median(tot) * 1e-3

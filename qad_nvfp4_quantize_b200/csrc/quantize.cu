@@ -287,10 +287,16 @@ __device__ __forceinline__ void ste_store(const uint4* gy, uint4* gx, const C& c
   if (!c.valid || !NVFP4_IN_BOUNDS(c.vec + 1, n_vec, st)) return;
   const uint4 a = ld_stream(gy + c.vec), b = ld_stream(gy + c.vec + 1);
   const f32x2 rr = pack2(r, r);
-  gx[c.vec] = make_uint4(ste_word(a.x, mul2(xs[0], rr)), ste_word(a.y, mul2(xs[1], rr)),
-                         ste_word(a.z, mul2(xs[2], rr)), ste_word(a.w, mul2(xs[3], rr)));
-  gx[c.vec + 1] = make_uint4(ste_word(b.x, mul2(xs[4], rr)), ste_word(b.y, mul2(xs[5], rr)),
-                             ste_word(b.z, mul2(xs[6], rr)), ste_word(b.w, mul2(xs[7], rr)));
+  const uint4 lo = make_uint4(ste_word(a.x, mul2(xs[0], rr)), ste_word(a.y, mul2(xs[1], rr)),
+                              ste_word(a.z, mul2(xs[2], rr)), ste_word(a.w, mul2(xs[3], rr)));
+  const uint4 hi = make_uint4(ste_word(b.x, mul2(xs[4], rr)), ste_word(b.y, mul2(xs[5], rr)),
+                              ste_word(b.z, mul2(xs[6], rr)), ste_word(b.w, mul2(xs[7], rr)));
+  if ((reinterpret_cast<uintptr_t>(gx) & 31u) == 0) {  // as in FakeOp::store_bf16x16
+    st_global_32b(gx + c.vec, lo, hi);
+  } else {
+    gx[c.vec] = lo;
+    gx[c.vec + 1] = hi;
+  }
 }
 
 // Backward with the forward's scales recomputed from x (max or four_over_six).

@@ -283,7 +283,7 @@ def test_fake_quant_and_ste_refill_freed_slots(nv, M, K):
 def test_bf16_outputs_at_16_byte_alignment(nv):
     # BF16 outputs are written 32 bytes per lane when the buffer is 32-byte
     # aligned and 16 bytes at a time otherwise; both layouts give the
-    # oracle's values (dynamic and frozen fake-quant, dequantize)
+    # oracle's values (dynamic and frozen fake-quant, dequantize, STE)
     rng = np.random.default_rng(5)
     M, K = 300, 1024
     x = inputs.to_bf16((rng.standard_t(3, (M, K)) * 0.3).astype(np.float32))
@@ -297,6 +297,12 @@ def test_bf16_outputs_at_16_byte_alignment(nv):
     np.testing.assert_array_equal(bf16_np(nv.fake_quant(xd, g=q.g, scales=q.scales, out=y16)), want)
     np.testing.assert_array_equal(bf16_np(nv.dequantize(q, out=y16)), want)
     np.testing.assert_array_equal(bf16_np(nv.dequantize(q)), want)
+    gy = inputs.to_bf16(rng.standard_normal((M, K)).astype(np.float32))
+    want_gx = o.fake_quant_backward(bf16_np(x), bf16_np(gy), "max")
+    for out in (y16, None):  # dynamic (fused pass) and frozen scales (streaming pass)
+        np.testing.assert_array_equal(bf16_np(nv.fake_quant_backward(xd, gy.cuda(), "max", out=out)), want_gx)
+        np.testing.assert_array_equal(
+            bf16_np(nv.fake_quant_backward(xd, gy.cuda(), g=q.g, scales=q.scales, out=out)), want_gx)
 
 
 def test_ste_backward_frozen_scales(nv):
