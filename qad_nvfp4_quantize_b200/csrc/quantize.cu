@@ -10,7 +10,9 @@
 //
 // Work decomposition: a warp's unit is a 512-element chunk of one row, one
 // 16-element block per lane (block_math.cuh). Codes leave as one 8-byte store
-// per lane, block scales as one byte per lane into the tiled scale layout.
+// per lane, block scales as one byte per lane into the tiled scale layout,
+// BF16 outputs (fake-quant, STE, dequantize) as one 32-byte store per lane
+// when the output is 32-byte aligned.
 // Dynamic calls run as a single cooperative launch (fused_dynamic_kernel);
 // static-scale and frozen-scale calls stream once (stream_pass_kernel).
 #include <type_traits>
