@@ -50,24 +50,6 @@ NVFP4_DEVINL bool bounds_ok(uint64_t i, uint64_t n, int* status) {
 // two-level scaling", num_bits [2,1] and scale_bits [4,3]).
 // ----------------------------------------------------------------------------
 
-// Four pairs of FP32 values -> 8 E2M1 codes in one 32-bit word; element 2j of
-// the group lands in the low nibble of byte j. cvt.e2m1x2 writes its first
-// source operand to the high nibble, so the odd element goes first.
-NVFP4_DEVINL uint32_t e2m1_pack8(const float v[8]) {
-  uint32_t out;
-  asm("{\n\t"
-      ".reg .b8 q0, q1, q2, q3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 q0, %2, %1;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 q1, %4, %3;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 q2, %6, %5;\n\t"
-      "cvt.rn.satfinite.e2m1x2.f32 q3, %8, %7;\n\t"
-      "mov.b32 %0, {q0, q1, q2, q3};\n\t"
-      "}"
-      : "=r"(out)
-      : "f"(v[0]), "f"(v[1]), "f"(v[2]), "f"(v[3]), "f"(v[4]), "f"(v[5]), "f"(v[6]), "f"(v[7]));
-  return out;
-}
-
 // One FP32 value -> E2M1 code in the low nibble.
 NVFP4_DEVINL uint32_t e2m1_code(float v) {
   uint16_t out;
@@ -89,25 +71,11 @@ NVFP4_DEVINL float e2m1_magnitude(uint32_t k) {
   return e ? normal : (m ? 0.5f : 0.0f);
 }
 
-NVFP4_DEVINL float e2m1_value(uint32_t code) {
-  const float mag = e2m1_magnitude(code & 7u);
-  return (code & 8u) ? -mag : mag;
-}
-
 // Non-negative FP32 -> E4M3 code (RNE, satfinite at 448).
 NVFP4_DEVINL uint32_t e4m3_code(float t) {
   uint16_t out;
   asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(out) : "f"(t), "f"(0.0f));
   return out & 0xFFu;
-}
-
-// Value of a non-negative E4M3 code 0..126: exponent field e (bias 7),
-// mantissa m (3 bits); e == 0 is subnormal (m * 2^-9).
-NVFP4_DEVINL float e4m3_value(uint32_t c) {
-  const uint32_t e = (c >> 3) & 15u, m = c & 7u;
-  const float normal = __uint_as_float(((e + 120u) << 23) | (m << 20));
-  const float sub = __fmul_rn((float)m, 0.001953125f);  // m * 2^-9, exact
-  return e ? normal : sub;
 }
 
 // Global scale from amax: g = amax / (6 * 448), FP32, correctly rounded;
@@ -122,12 +90,6 @@ NVFP4_DEVINL uint32_t block_scale_code(float bmax, float g, float mt) {
   const float t = __fdiv_rn(bmax, __fmul_rn(mt, g));
   const uint32_t c = e4m3_code(t);
   return c > 1u ? c : 1u;
-}
-
-// BF16 pair (packed in a 32-bit word) -> two FP32 values (exact).
-NVFP4_DEVINL void bf16x2_to_f32(uint32_t w, float& lo, float& hi) {
-  lo = __uint_as_float(w << 16);
-  hi = __uint_as_float(w & 0xFFFF0000u);
 }
 
 NVFP4_DEVINL uint32_t f32x2_to_bf16x2(float lo, float hi) {
@@ -179,35 +141,6 @@ NVFP4_DEVINL bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
       : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
-}
-
-// Bounded wait on an mbarrier phase. Returns false (and raises *abort) if the
-// phase did not complete within limit_ns or another role already aborted.
-NVFP4_DEVINL bool mbar_wait_bounded(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                    uint64_t limit_ns) {
-  if (mbar_try_wait(bar, parity)) return true;
-  const uint64_t t0 = globaltimer_ns();
-  uint32_t spins = 0;
-  while (true) {
-    if (mbar_try_wait(bar, parity)) return true;
-    if (((++spins) & 63u) == 0) {
-      if (*abort) return false;
-      if (globaltimer_ns() - t0 > limit_ns) {
-        *abort = 1;
-        return false;
-      }
-    }
-  }
-}
-
-// 2-D tiled TMA load into shared memory, completion on an mbarrier.
-NVFP4_DEVINL void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t x, int32_t y,
-                              uint64_t* bar) {
-  asm volatile(
-      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
-      " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(smem_dst)),
-      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
-      : "memory");
 }
 
 // Contiguous bulk copy global -> shared (16-byte aligned, size % 16 == 0).
@@ -284,33 +217,6 @@ NVFP4_DEVINL void tc_fence_after() {
   asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
 
-// Arrive on `bar` once every tcgen05 operation this thread issued so far has
-// completed.
-NVFP4_DEVINL void tc_commit(uint64_t* bar) {
-  asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                   smem_u32(bar))
-               : "memory");
-}
-
-// Shared -> tensor memory copy of one 512-byte scale tile (32 rows of 16
-// bytes), replicated into the four 32-lane quarters of tensor memory.
-NVFP4_DEVINL void tc_copy_scales(uint32_t taddr, uint64_t sdesc) {
-  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
-}
-
-// D[tmem] (+)= A[smem] * B[smem]^T with per-16-element UE4M3 scales read from
-// tensor memory: the block-scaled FP4 MMA (kind::mxf4nvf4, M=128, K=64).
-NVFP4_DEVINL void tc_mma_nvf4(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
-                              uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "tcgen05.mma.cta_group::1.kind::mxf4nvf4.block_scale.block16 [%0], %1, %2, %3, [%5], [%6], p;\n\t"
-      "}" ::"r"(d_tmem),
-      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(sfa_tmem), "r"(sfb_tmem)
-      : "memory");
-}
-
 NVFP4_DEVINL void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // 32 consecutive FP32 columns of this warp's 32 tensor-memory lanes.
@@ -347,6 +253,8 @@ NVFP4_DEVINL uint64_t smem_desc(uint32_t saddr, uint32_t lbo_bytes, uint32_t sbo
 // instruction is predicated on elect.sync, which picks the same single lane
 // every time for a full mask.
 // ----------------------------------------------------------------------------
+// Issue helpers for a converged warp: elect.sync picks one lane, which
+// issues the operation (the same lane every time, so issue order holds).
 #define NVFP4_ELECT_BEGIN "{\n\t.reg .pred e;\n\telect.sync _|e, 0xffffffff;\n\t"
 #define NVFP4_ELECT_END "\n\t}"
 
@@ -355,6 +263,7 @@ NVFP4_DEVINL void mbar_arrive_expect_tx_elect(uint64_t* bar, uint32_t bytes) {
                ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
+// 2-D tiled TMA load into shared memory, completion on an mbarrier.
 NVFP4_DEVINL void tma_load_2d_elect(void* smem_dst, const CUtensorMap* map, int32_t x, int32_t y, uint64_t* bar) {
   asm volatile(NVFP4_ELECT_BEGIN
                "@e cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
@@ -363,6 +272,7 @@ NVFP4_DEVINL void tma_load_2d_elect(void* smem_dst, const CUtensorMap* map, int3
                : "memory");
 }
 
+// Contiguous bulk copy global -> shared, completion on an mbarrier.
 NVFP4_DEVINL void bulk_load_elect(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
   asm volatile(NVFP4_ELECT_BEGIN
                "@e cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];"
@@ -370,11 +280,15 @@ NVFP4_DEVINL void bulk_load_elect(void* smem_dst, const void* src, uint32_t byte
                ::"r"(smem_u32(smem_dst)), "l"(src), "r"(bytes), "r"(smem_u32(bar)) : "memory");
 }
 
+// Shared -> tensor memory copy of one 512-byte scale tile (32 rows of 16
+// bytes), replicated into the four 32-lane quarters of tensor memory.
 NVFP4_DEVINL void tc_copy_scales_elect(uint32_t taddr, uint64_t sdesc) {
   asm volatile(NVFP4_ELECT_BEGIN "@e tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" NVFP4_ELECT_END
                ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
+// D[tmem] (+)= A[smem] * B[smem]^T with per-16-element UE4M3 scales read from
+// tensor memory: the block-scaled FP4 MMA (kind::mxf4nvf4, M=128, K=64).
 NVFP4_DEVINL void tc_mma_nvf4_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                     uint32_t sfa_tmem, uint32_t sfb_tmem, uint32_t accumulate) {
   asm volatile(NVFP4_ELECT_BEGIN ".reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
@@ -384,6 +298,7 @@ NVFP4_DEVINL void tc_mma_nvf4_elect(uint32_t d_tmem, uint64_t a_desc, uint64_t b
                : "memory");
 }
 
+// Arrive on `bar` once every tcgen05 operation issued so far has completed.
 NVFP4_DEVINL void tc_commit_elect(uint64_t* bar) {
   asm volatile(NVFP4_ELECT_BEGIN
                "@e tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" NVFP4_ELECT_END
